@@ -1,0 +1,159 @@
+#pragma once
+// extern "C" entry points of libhlwq (declared and documented in include/hlwq.h).
+// Every argument is validated on the host; nothing is launched on an error.
+
+#include <algorithm>
+#include <cstdint>
+
+#include "hlwq_common.cuh"
+
+namespace hlwq {
+
+
+
+int launch_quantize(const void* W, bool bf16, int64_t rows, int in, const float* codebook, uint8_t* packed,
+                    uint16_t* norms, cudaStream_t stream);
+int launch_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows, int in,
+                      void* out, bool bf16, cudaStream_t stream);
+int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                 const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
+int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                   const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
+                   size_t ws_bytes, cudaStream_t stream);
+size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M);
+size_t moe_workspace_bytes(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk);
+int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+               const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+               const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
+               int topk, int T, const float* logits, const uint16_t* X, void* Y, bool out_bf16, int32_t* ids_out,
+               float* w_out, void* workspace, cudaStream_t stream);
+
+}  // namespace hlwq
+
+namespace {
+
+constexpr int64_t kMaxIn = 1 << 20;  // in-features limit (int indexing inside blocks)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Threshold between the CUDA-core decode path and the tensor-core path.
+constexpr int64_t kTensorCoreMinM = 16;
+
+}  // namespace
+
+extern "C" int hlwq_quantize(const void* W, int wdtype, int64_t rows, int64_t in, const float* codebook,
+                             uint8_t* packed, uint16_t* norms, void* stream) {
+  if (!W || !codebook || !packed || !norms || rows <= 0 || in <= 0 || in > kMaxIn) return HLWQ_EINVAL;
+  if (wdtype != HLWQ_F32 && wdtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || !aligned2(norms) || !aligned2(W) || (wdtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(W) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_quantize(W, wdtype == HLWQ_BF16, rows, static_cast<int>(in), codebook, packed, norms,
+                               as_stream(stream));
+}
+
+extern "C" int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows,
+                               int64_t in, void* W_out, int odtype, void* stream) {
+  if (!W_out || !codebook || !packed || !norms || rows <= 0 || in <= 0 || in > kMaxIn) return HLWQ_EINVAL;
+  if (odtype != HLWQ_F32 && odtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || !aligned2(norms) || !aligned2(W_out) ||
+      (odtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(W_out) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_dequantize(packed, norms, codebook, rows, static_cast<int>(in), W_out, odtype == HLWQ_BF16,
+                                 as_stream(stream));
+}
+
+extern "C" int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
+                         int64_t in, const uint16_t* x, void* y, int ydtype, void* stream) {
+  if (!packed || !norms || !codebook || !x || !y || out <= 0 || in <= 0 || in > kMaxIn) return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || !aligned2(norms) || !aligned2(x) || !aligned2(y) ||
+      (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(y) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_dense(packed, norms, codebook, out, static_cast<int>(in), x, in, 1, y, out,
+                            ydtype == HLWQ_BF16, as_stream(stream));
+}
+
+extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
+                         int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy, int ydtype,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  if (!packed || !norms || !codebook || !X || !Y || out <= 0 || in <= 0 || in > kMaxIn || M <= 0 || M > (1 << 20))
+    return HLWQ_EINVAL;
+  if (ldx < in || ldy < out) return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || !aligned2(norms) || !aligned2(X) || !aligned2(Y) ||
+      (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(Y) & 3u)))
+    return HLWQ_EALIGN;
+  const size_t need = hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0);
+  if (need && (!workspace || ws_bytes < need)) return HLWQ_EWORKSPACE;
+  if (need && !aligned16(workspace)) return HLWQ_EALIGN;
+  if (M >= kTensorCoreMinM)
+    return hlwq::launch_gemm_tc(packed, norms, codebook, out, static_cast<int>(in), X, ldx, static_cast<int>(M), Y,
+                                ldy, ydtype == HLWQ_BF16, workspace, ws_bytes, as_stream(stream));
+  return hlwq::launch_dense(packed, norms, codebook, out, static_cast<int>(in), X, ldx, static_cast<int>(M), Y, ldy,
+                            ydtype == HLWQ_BF16, as_stream(stream));
+}
+
+extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+                             const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                             const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook,
+                             int64_t E, int64_t H, int64_t F, int64_t topk, int64_t T, const float* router_logits,
+                             const uint16_t* X, void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (!gu_packed || !gu_norms || !dn_packed || !dn_norms || !codebook || !router_logits || !X || !Y)
+    return HLWQ_EINVAL;
+  if (E <= 0 || E > 1024 || H <= 0 || H > kMaxIn || F <= 0 || F > kMaxIn || T <= 0 || T > 65535 || topk <= 0 ||
+      topk > 32 || topk > E)
+    return HLWQ_EINVAL;
+  const int shared_given = (sh_gu_packed != nullptr) + (sh_gu_norms != nullptr) + (sh_dn_packed != nullptr) +
+                           (sh_dn_norms != nullptr);
+  if (shared_given != 0 && shared_given != 4) return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(gu_packed) || !aligned16(dn_packed) || (sh_gu_packed && !aligned16(sh_gu_packed)) ||
+      (sh_dn_packed && !aligned16(sh_dn_packed)) || !aligned2(gu_norms) || !aligned2(dn_norms) || !aligned2(X) ||
+      !aligned2(Y) || (reinterpret_cast<uintptr_t>(router_logits) & 3u) ||
+      (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(Y) & 3u)))
+    return HLWQ_EALIGN;
+  const size_t need = hlwq_workspace_bytes(HLWQ_OP_MOE, H, F, T, E, topk);
+  if (!workspace || ws_bytes < need) return HLWQ_EWORKSPACE;
+  if (!aligned16(workspace)) return HLWQ_EALIGN;
+  return hlwq::launch_moe(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+                          sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H), static_cast<int>(F),
+                          static_cast<int>(topk), static_cast<int>(T), router_logits, X, Y, ydtype == HLWQ_BF16,
+                          topk_ids, topk_weights, workspace, as_stream(stream));
+}
+
+extern "C" size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk) {
+  if (a <= 0 || b <= 0 || c <= 0) return 0;
+  if (op == HLWQ_OP_GEMM) return c >= kTensorCoreMinM ? hlwq::gemm_tc_workspace_bytes(a, b, c) : 0;
+  if (op == HLWQ_OP_MOE) {
+    if (E <= 0 || topk <= 0) return 0;
+    return hlwq::moe_workspace_bytes(E, a, b, c, topk);
+  }
+  return 0;
+}
+
+extern "C" int hlwq_device_error(uint32_t* bits) {
+  if (!bits) return HLWQ_EINVAL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return HLWQ_ECUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, hlwq::g_device_error, sizeof(v)) != cudaSuccess) return HLWQ_ECUDA;
+  if (cudaMemcpyToSymbol(hlwq::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return HLWQ_ECUDA;
+  *bits = v;
+  return HLWQ_OK;
+}
+
+extern "C" const char* hlwq_status_string(int status) {
+  switch (status) {
+    case HLWQ_OK: return "ok";
+    case HLWQ_EINVAL: return "invalid argument";
+    case HLWQ_EALIGN: return "misaligned pointer or leading dimension";
+    case HLWQ_EUNSUPPORTED: return "unsupported size or dtype";
+    case HLWQ_ECUDA: return "CUDA runtime error";
+    case HLWQ_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int hlwq_version(void) { return 100; }

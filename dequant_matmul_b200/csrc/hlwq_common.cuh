@@ -1,0 +1,82 @@
+// Shared device helpers for the HLWQ Q5 kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hlwq.h"
+
+namespace hlwq {
+
+constexpr int kBlock = 128;      // weights per block (Method step [1])
+constexpr int kBlockBytes = 80;  // 128 codes x 5 bits (Method step [5])
+constexpr int kLevels = 32;      // centroids (Method step [4])
+
+// Device error word (see hlwq_device_error in hlwq.h).
+__device__ unsigned int g_device_error = 0u;
+
+__device__ __forceinline__ void raise_device_error(unsigned bits) { atomicOr(&g_device_error, bits); }
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// Two bf16 values packed in a 32-bit word -> fp32 (exact).
+__device__ __forceinline__ float bf16x2_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16x2_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t float_to_bf16_bits(float f) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+// Streaming 128-bit load that does not allocate in L1 (data read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// acc + a * b with a, b binary16 and fp32 accumulation (the product is exact).
+__device__ __forceinline__ float fma_f16_f32(uint16_t a, uint16_t b, float acc) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(acc));
+  return d;
+}
+
+// Extract 10 bits starting at bit `sh` of the 64-bit pair (lo, hi).
+template <int SH>
+__device__ __forceinline__ uint32_t bits10(uint32_t lo, uint32_t hi) {
+  if constexpr (SH <= 22) {
+    return (lo >> SH) & 0x3ffu;
+  } else {
+    return __funnelshift_r(lo, hi, SH) & 0x3ffu;
+  }
+}
+
+template <int SH>
+__device__ __forceinline__ uint32_t bits5(uint32_t lo, uint32_t hi) {
+  if constexpr (SH <= 27) {
+    return (lo >> SH) & 0x1fu;
+  } else {
+    return __funnelshift_r(lo, hi, SH) & 0x1fu;
+  }
+}
+
+inline int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+__host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace hlwq

@@ -1,0 +1,7 @@
+// Single translation unit of libhlwq: the kernels share the device error word
+// and are compiled together (no relocatable device code needed).
+#include "quantize.cuh"
+#include "gemv.cuh"
+#include "moe.cuh"
+#include "gemm_tc.cuh"
+#include "api.cuh"

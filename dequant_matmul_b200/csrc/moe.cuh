@@ -1,0 +1,385 @@
+#pragma once
+// Routed mixture-of-experts layer on HLWQ Q5 experts (sm_100a).
+//
+// "Qwen3.6-35B-A3B -- HLWQ Q5" model card: 256 experts per layer, 8 routed +
+// 1 shared per token; "Gemma-4-26B-A4B-it-HLWQ-Q5", Technical Details: 3-D
+// expert tensors (128, 1408, 2816) and (128, 2816, 704), each expert quantized
+// independently.  Per token t:
+//   ids, p = top-k of the router logits (ties: lower id), p = softmax over the
+//            k selected logits;
+//   g || u = w_hat_gu[e] @ x_t (rows [0, F) gate, [F, 2F) up), h = SiLU(g) * u;
+//   Y[t]   = sum_s p_s * w_hat_dn[ids_s] @ h_s  (+ shared expert with weight 1).
+//
+// Four launches, no atomics, deterministic:
+//   1. router (one CTA): top-k + softmax per token, per-expert assignment lists
+//      sorted by (expert, token), and the rotated activations of every token;
+//   2. gate_up: persistent CTAs over units (active expert, 32 intermediate
+//      columns); each unit decodes its gate and up rows against the tokens
+//      routed to that expert (each expert's codes are read once per call) and
+//      writes h = SiLU(g) * u in fp32;
+//   3. down: units (active expert, 128 output rows); h of the expert's tokens is
+//      rotated in the CTA, the weighted result goes to a per-assignment slot;
+//   4. combine: Y[t] = sum over the token's assignment slots in a fixed order.
+
+#include <algorithm>
+
+#include "engine.cuh"
+
+namespace hlwq {
+
+namespace {
+
+constexpr int kRouterThreads = 1024;
+constexpr int kJT = 32;   // intermediate columns per gate_up unit
+constexpr int kHT = 128;  // output rows per down unit
+
+struct MoeWs {
+  int* meta;          // [0] = number of active experts (shared expert last)
+  int* active;        // [E + 1] expert id per active slot (E = shared expert)
+  int* offsets;       // [E + 2] assignment range per active slot
+  int* asg_token;     // [NA]
+  float* asg_weight;  // [NA]
+  int* tok_asg;       // [T][topk + 1] assignment index per (token, slot), -1 = none
+  int* sel_id;        // [T][topk]
+  float* sel_w;       // [T][topk]
+  uint16_t* xt;       // [T][NBh][kXsStride] rotated tokens (binary16)
+  float* xt_inv;      // [T]
+  float* h;           // [NA][F]
+  float* part;        // [NA][H]
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char* base, MoeWs* ws) {
+  const int64_t nbh = ceil_div(H, kBlock);
+  const int64_t na = T * topk + T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  MoeWs w;
+  w.meta = reinterpret_cast<int*>(take(16));
+  w.active = reinterpret_cast<int*>(take(sizeof(int) * (E + 1)));
+  w.offsets = reinterpret_cast<int*>(take(sizeof(int) * (E + 2)));
+  w.asg_token = reinterpret_cast<int*>(take(sizeof(int) * na));
+  w.asg_weight = reinterpret_cast<float*>(take(sizeof(float) * na));
+  w.tok_asg = reinterpret_cast<int*>(take(sizeof(int) * T * (topk + 1)));
+  w.sel_id = reinterpret_cast<int*>(take(sizeof(int) * T * topk));
+  w.sel_w = reinterpret_cast<float*>(take(sizeof(float) * T * topk));
+  w.xt = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * T * nbh * kXsStride));
+  w.xt_inv = reinterpret_cast<float*>(take(sizeof(float) * T));
+  w.h = reinterpret_cast<float*>(take(sizeof(float) * na * F));
+  w.part = reinterpret_cast<float*>(take(sizeof(float) * na * H));
+  if (ws) *ws = w;
+  return off;
+}
+
+__global__ void __launch_bounds__(kRouterThreads, 1)
+router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, int E, int H, int T, int topk,
+              int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
+  __shared__ float red[64];
+  __shared__ int s_count[1025];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_lane = (E + 31) / 32;
+
+  // 1. top-k + softmax, one warp per token.
+  for (int t = warp; t < T; t += kRouterThreads / 32) {
+    const float* lg = logits + static_cast<int64_t>(t) * E;
+    unsigned taken = 0u;  // bit i: element lane + 32 i selected
+    float vmax = 0.0f, wsum = 0.0f;
+    for (int s = 0; s < topk; ++s) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int i = 0; i < per_lane; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u)) {
+          const float v = lg[e];
+          if (v > bv || (v == bv && e < bi) || bi == 0x7fffffff) { bv = v; bi = e; }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (s == 0) vmax = bv;
+      const float ex = expf(bv - vmax);
+      wsum += ex;
+      if (lane == 0) {
+        ws.sel_id[t * topk + s] = bi;
+        ws.sel_w[t * topk + s] = ex;
+      }
+    }
+    __syncwarp();
+    if (lane < topk) {
+      const float wv = ws.sel_w[t * topk + lane] / wsum;
+      ws.sel_w[t * topk + lane] = wv;
+      if (ids_out) ids_out[t * topk + lane] = ws.sel_id[t * topk + lane];
+      if (w_out) w_out[t * topk + lane] = wv;
+    }
+  }
+  __syncthreads();
+
+  // 2. assignments per expert (id E = shared expert, every token).
+  const int nexp = E + (has_shared ? 1 : 0);
+  for (int e = threadIdx.x; e < nexp; e += kRouterThreads) {
+    int c = 0;
+    if (e == E) c = T;
+    else
+      for (int q = 0; q < T * topk; ++q) c += ws.sel_id[q] == e;
+    s_count[e] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int na = 0, off = 0;
+    for (int e = 0; e < nexp; ++e) {
+      if (s_count[e]) {
+        ws.active[na] = e;
+        ws.offsets[na] = off;
+        off += s_count[e];
+        s_count[e] = na;  // reuse: active slot of expert e
+        ++na;
+      } else {
+        s_count[e] = -1;
+      }
+    }
+    ws.offsets[na] = off;
+    ws.meta[0] = na;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < nexp; e += kRouterThreads) {
+    const int slot = s_count[e];
+    if (slot < 0) continue;
+    int pos = ws.offsets[slot];
+    if (e == E) {
+      for (int t = 0; t < T; ++t, ++pos) {
+        ws.asg_token[pos] = t;
+        ws.asg_weight[pos] = 1.0f;
+        ws.tok_asg[t * (topk + 1) + topk] = pos;
+      }
+    } else {
+      for (int q = 0; q < T * topk; ++q) {
+        if (ws.sel_id[q] == e) {
+          ws.asg_token[pos] = q / topk;
+          ws.asg_weight[pos] = ws.sel_w[q];
+          ws.tok_asg[(q / topk) * (topk + 1) + (q % topk)] = pos;
+          ++pos;
+        }
+      }
+    }
+  }
+  if (!has_shared)
+    for (int t = threadIdx.x; t < T; t += kRouterThreads) ws.tok_asg[t * (topk + 1) + topk] = -1;
+
+  // 3. rotated activations of every token (binary16, per-token power-of-two scale).
+  const int nbh = (H + kBlock - 1) / kBlock;
+  for (int t = 0; t < T; ++t)
+    rotate_activations_bf16(X + static_cast<int64_t>(t) * H, H, H, nbh, 1, 1,
+                            ws.xt + static_cast<int64_t>(t) * nbh * kXsStride, ws.xt_inv + t, red);
+}
+
+template <int C>
+__device__ void gate_up_unit_pass(int mt, const uint32_t* tab, const uint16_t* xs, const uint8_t* packed,
+                                  const uint16_t* norms, int nb, int jt, int j0, int F, float* slots) {
+  auto rowfn = [=](int v) { return static_cast<int64_t>(v < jt ? j0 + v : F + j0 + (v - jt)); };
+  switch (mt) {
+    case 1: engine_items<C, 1>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
+    case 2: engine_items<C, 2>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
+    default: engine_items<C, 4>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
+  }
+}
+
+template <int C>
+__device__ void down_unit_pass(int mt, const uint32_t* tab, const uint16_t* xs, const uint8_t* packed,
+                               const uint16_t* norms, int nb, int nr, int r0, float* slots) {
+  auto rowfn = [=](int v) { return static_cast<int64_t>(r0 + v); };
+  switch (mt) {
+    case 1: engine_items<C, 1>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
+    case 2: engine_items<C, 2>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
+    default: engine_items<C, 4>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
+  }
+}
+
+__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : (ntok <= 2 ? 2 : 4); }
+
+template <int C>
+__global__ void __launch_bounds__(kEngineThreads, 1)
+gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict__ gu_norms,
+               const uint8_t* __restrict__ sh_packed, const uint16_t* __restrict__ sh_norms,
+               const float* __restrict__ codebook, int E, int H, int F, MoeWs ws) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nb = (H + kBlock - 1) / kBlock;
+  const int nch = (nb + C - 1) / C;
+  const EngineLayout L = engine_layout(4, nb, 2 * kJT, nch);
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
+  float* slots = reinterpret_cast<float*>(smem + L.slot_off);
+  float* misc = reinterpret_cast<float*>(smem + L.misc_off);
+  float* inv = misc + 48;
+  uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
+  build_pair_table(tab, c16, codebook);
+  __syncthreads();
+
+  const int tiles = (F + kJT - 1) / kJT;
+  const int units = ws.meta[0] * tiles;
+  const int64_t expert_rows = 2 * static_cast<int64_t>(F);
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int a = u / tiles, tile = u - a * tiles;
+    const int e = ws.active[a];
+    const int j0 = tile * kJT, jt = min(kJT, F - j0);
+    const uint8_t* pk = e < E ? gu_packed + e * expert_rows * nb * kBlockBytes : sh_packed;
+    const uint16_t* nm = e < E ? gu_norms + e * expert_rows * nb : sh_norms;
+    const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
+    for (int m0 = 0; m0 < ne; m0 += 4) {
+      const int ntok = min(4, ne - m0), mt = pass_mt(ntok);
+      // stage the tokens' rotated activations
+      const int words = nb * kXsStride / 8;  // uint4 per token
+      for (int q = threadIdx.x; q < mt * words; q += blockDim.x) {
+        const int m = q / words, w = q - m * words;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (m < ntok) {
+          const int t = ws.asg_token[a0 + m0 + m];
+          val = reinterpret_cast<const uint4*>(ws.xt + static_cast<int64_t>(t) * nb * kXsStride)[w];
+        }
+        reinterpret_cast<uint4*>(xs)[q] = val;
+      }
+      if (threadIdx.x < 4) inv[threadIdx.x] = threadIdx.x < ntok ? ws.xt_inv[ws.asg_token[a0 + m0 + threadIdx.x]] : 0.0f;
+      __syncthreads();
+      gate_up_unit_pass<C>(mt, tab, xs, pk, nm, nb, jt, j0, F, slots);
+      __syncthreads();
+      const int nv = 2 * jt;
+      for (int idx = threadIdx.x; idx < ntok * jt; idx += blockDim.x) {
+        const int m = idx / jt, j = idx - m * jt;
+        const float* sg = slots + (m * nv + j) * nch;
+        const float* su = slots + (m * nv + jt + j) * nch;
+        float g = 0.0f, up = 0.0f;
+        for (int ch = 0; ch < nch; ++ch) { g += sg[ch]; up += su[ch]; }
+        g *= inv[m];
+        up *= inv[m];
+        const float hval = g / (1.0f + expf(-g)) * up;
+        ws.h[static_cast<int64_t>(a0 + m0 + m) * F + j0 + j] = hval;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+template <int C>
+__global__ void __launch_bounds__(kEngineThreads, 1)
+down_kernel(const uint8_t* __restrict__ dn_packed, const uint16_t* __restrict__ dn_norms,
+            const uint8_t* __restrict__ sh_packed, const uint16_t* __restrict__ sh_norms,
+            const float* __restrict__ codebook, int E, int H, int F, MoeWs ws) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nb = (F + kBlock - 1) / kBlock;
+  const int nch = (nb + C - 1) / C;
+  const EngineLayout L = engine_layout(4, nb, kHT, nch);
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
+  float* slots = reinterpret_cast<float*>(smem + L.slot_off);
+  float* misc = reinterpret_cast<float*>(smem + L.misc_off);
+  float* inv = misc + 48;
+  uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
+  build_pair_table(tab, c16, codebook);
+  __syncthreads();
+
+  const int tiles = (H + kHT - 1) / kHT;
+  const int units = ws.meta[0] * tiles;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int a = u / tiles, tile = u - a * tiles;
+    const int e = ws.active[a];
+    const int r0 = tile * kHT, nr = min(kHT, H - r0);
+    const uint8_t* pk = e < E ? dn_packed + static_cast<int64_t>(e) * H * nb * kBlockBytes : sh_packed;
+    const uint16_t* nm = e < E ? dn_norms + static_cast<int64_t>(e) * H * nb : sh_norms;
+    const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
+    for (int m0 = 0; m0 < ne; m0 += 4) {
+      const int ntok = min(4, ne - m0), mt = pass_mt(ntok);
+      const float* hbase = ws.h + static_cast<int64_t>(a0 + m0) * F;
+      rotate_activations_f32([=](int m) { return hbase + static_cast<int64_t>(m) * F; }, F, nb, ntok, mt, xs, inv,
+                             misc);
+      down_unit_pass<C>(mt, tab, xs, pk, nm, nb, nr, r0, slots);
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < ntok * nr; idx += blockDim.x) {
+        const int m = idx / nr, v = idx - m * nr;
+        const float* sl = slots + (m * nr + v) * nch;
+        float sum = 0.0f;
+        for (int ch = 0; ch < nch; ++ch) sum += sl[ch];
+        const int asg = a0 + m0 + m;
+        ws.part[static_cast<int64_t>(asg) * H + r0 + v] = sum * inv[m] * ws.asg_weight[asg];
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void combine_kernel(int H, int T, int topk, MoeWs ws, void* __restrict__ Y, int out_bf16) {
+  const int t = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T || i >= H) return;
+  float acc = 0.0f;
+  for (int s = 0; s <= topk; ++s) {
+    const int asg = ws.tok_asg[t * (topk + 1) + s];
+    if (asg >= 0) acc += ws.part[static_cast<int64_t>(asg) * H + i];
+  }
+  const int64_t off = static_cast<int64_t>(t) * H + i;
+  if (out_bf16) static_cast<uint16_t*>(Y)[off] = static_cast<uint16_t>(float_to_bf16_bits(acc));
+  else static_cast<float*>(Y)[off] = acc;
+}
+
+template <typename K>
+bool set_smem_attr(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) == cudaSuccess;
+}
+
+}  // namespace
+
+size_t moe_workspace_bytes(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk) {
+  return moe_layout(E, H, F, T, topk, nullptr, nullptr);
+}
+
+int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+               const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+               const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
+               int topk, int T, const float* logits, const uint16_t* X, void* Y, bool out_bf16, int32_t* ids_out,
+               float* w_out, void* workspace, cudaStream_t stream) {
+  MoeWs ws;
+  moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
+  const bool shared = sh_gu_packed != nullptr;
+  router_kernel<<<1, kRouterThreads, 0, stream>>>(logits, X, E, H, T, topk, shared ? 1 : 0, ids_out, w_out, ws);
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+
+  const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
+  const int cg = pick_chunk(nbh), cd = pick_chunk(nbf);
+  const int smem_g = engine_layout(4, nbh, 2 * kJT, (nbh + cg - 1) / cg).total;
+  const int smem_d = engine_layout(4, nbf, kHT, (nbf + cd - 1) / cd).total;
+  if (smem_g > 227 * 1024 || smem_d > 227 * 1024) return HLWQ_EUNSUPPORTED;
+  const int grid = sm_count();
+  static bool attrs = false;
+  if (!attrs) {
+    bool ok = set_smem_attr(gate_up_kernel<8>) && set_smem_attr(gate_up_kernel<4>) &&
+              set_smem_attr(gate_up_kernel<2>) && set_smem_attr(down_kernel<8>) &&
+              set_smem_attr(down_kernel<4>) && set_smem_attr(down_kernel<2>);
+    if (!ok) return HLWQ_ECUDA;
+    attrs = true;
+  }
+  switch (cg) {
+    case 8: gate_up_kernel<8><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
+    case 4: gate_up_kernel<4><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
+    default: gate_up_kernel<2><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  switch (cd) {
+    case 8: down_kernel<8><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
+    case 4: down_kernel<4><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
+    default: down_kernel<2><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  dim3 cgrid(static_cast<unsigned>(ceil_div(H, 256)), static_cast<unsigned>(T));
+  combine_kernel<<<cgrid, 256, 0, stream>>>(H, T, topk, ws, Y, out_bf16 ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+}
+
+}  // namespace hlwq

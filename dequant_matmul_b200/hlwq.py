@@ -1,0 +1,200 @@
+"""Thin ctypes binding of libhlwq (include/hlwq.h).
+
+Argument marshalling only: every step of the quantizer and of the matmuls runs
+in the library's CUDA kernels.  Tensors must be CUDA tensors; the call is
+enqueued on torch's current stream.  If the shared library is missing or cannot
+be loaded the import fails loudly -- there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhlwq.so")
+
+HLWQ_OK, HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_ECUDA, HLWQ_EWORKSPACE = 0, -1, -2, -3, -4, -5
+HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
+HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
+BLOCK, BLOCK_BYTES, LEVELS = 128, 80, 32
+
+# (name, restype, argtypes) for every symbol include/hlwq.h declares.
+_P, _I, _I64, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+SIGNATURES = {
+    "hlwq_lloyd_codebook": (_I, [_I, _P, _P, _P]),
+    "hlwq_quantize": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
+    "hlwq_gemv": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
+    "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
+    "hlwq_moe_gemv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _I,
+                           _P, _P, _P, _SZ, _P]),
+    "hlwq_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I64, _I64]),
+    "hlwq_device_error": (_I, [_P]),
+    "hlwq_status_string": (ctypes.c_char_p, [_I]),
+    "hlwq_version": (_I, []),
+}
+
+
+class HLWQError(RuntimeError):
+    pass
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libhlwq.so not built ({LIB_PATH}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int, what: str):
+    if status != HLWQ_OK:
+        raise HLWQError(f"{what}: {lib.hlwq_status_string(status).decode()} ({status})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt) -> int:
+    if dt == torch.float32:
+        return HLWQ_F32
+    if dt == torch.bfloat16:
+        return HLWQ_BF16
+    raise HLWQError(f"unsupported dtype {dt}")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise HLWQError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise HLWQError(f"{name} must be contiguous")
+
+
+def n_blocks(in_features: int) -> int:
+    return (in_features + BLOCK - 1) // BLOCK
+
+
+# ------------------------------------------------------------------ host calls
+def lloyd_codebook(levels: int = LEVELS):
+    """Returns (centroids float32[L], midpoints float32[L-1], mse) on the host."""
+    c = (ctypes.c_float * levels)()
+    m = (ctypes.c_float * max(levels - 1, 1))()
+    mse = ctypes.c_double()
+    _check(lib.hlwq_lloyd_codebook(levels, ctypes.cast(c, _P), ctypes.cast(m, _P), ctypes.byref(mse)),
+           "hlwq_lloyd_codebook")
+    return (torch.tensor(list(c), dtype=torch.float32), torch.tensor(list(m)[: levels - 1], dtype=torch.float32),
+            mse.value)
+
+
+def codebook(device="cuda") -> torch.Tensor:
+    return lloyd_codebook(LEVELS)[0].to(device)
+
+
+def workspace_bytes(op: int, a: int, b: int, c: int, E: int = 1, topk: int = 0) -> int:
+    return int(lib.hlwq_workspace_bytes(op, a, b, c, E, topk))
+
+
+def device_error() -> int:
+    bits = ctypes.c_uint32()
+    _check(lib.hlwq_device_error(ctypes.byref(bits)), "hlwq_device_error")
+    return bits.value
+
+
+# ------------------------------------------------------------------ device calls
+def quantize(W: torch.Tensor, cb: torch.Tensor, packed=None, norms=None, stream=None):
+    """W: [..., in] fp32/bf16 CUDA tensor (leading dims are stacked rows).
+    Returns (packed uint8 [..., NB, 80], norms uint16 [..., NB] binary16 bits)."""
+    _cuda(W, "W")
+    in_f = W.shape[-1]
+    rows = W.numel() // in_f
+    nb = n_blocks(in_f)
+    lead = tuple(W.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (nb, BLOCK_BYTES), dtype=torch.uint8, device=W.device)
+    if norms is None:
+        norms = torch.empty(lead + (nb,), dtype=torch.uint16, device=W.device)
+    _check(lib.hlwq_quantize(_ptr(W), _dtype_code(W.dtype), rows, in_f, _ptr(cb), _ptr(packed), _ptr(norms),
+                             _stream(stream)), "hlwq_quantize")
+    return packed, norms
+
+
+def dequantize(packed, norms, cb, in_features: int, out_dtype=torch.float32, out=None, stream=None):
+    _cuda(packed, "packed")
+    nb = packed.shape[-2]
+    lead = tuple(packed.shape[:-2])
+    rows = packed.numel() // (nb * BLOCK_BYTES)
+    if out is None:
+        out = torch.empty(lead + (in_features,), dtype=out_dtype, device=packed.device)
+    _check(lib.hlwq_dequantize(_ptr(packed), _ptr(norms), _ptr(cb), rows, in_features, _ptr(out),
+                               _dtype_code(out.dtype), _stream(stream)), "hlwq_dequantize")
+    return out
+
+
+def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None):
+    """x: bf16 [in].  Returns y [out]."""
+    _cuda(x, "x")
+    out_f = packed.shape[0]
+    if y is None:
+        y = torch.empty(out_f, dtype=out_dtype, device=x.device)
+    _check(lib.hlwq_gemv(_ptr(packed), _ptr(norms), _ptr(cb), out_f, x.shape[-1], _ptr(x), _ptr(y),
+                         _dtype_code(y.dtype), _stream(stream)), "hlwq_gemv")
+    return y
+
+
+def gemm(packed, norms, cb, X: torch.Tensor, out_dtype=torch.bfloat16, Y=None, workspace=None, stream=None):
+    """X: bf16 [M][in] (row pitch X.stride(0)).  Returns Y [M][out]."""
+    _cuda(X, "X")
+    out_f = packed.shape[0]
+    M, in_f = X.shape
+    if Y is None:
+        Y = torch.empty(M, out_f, dtype=out_dtype, device=X.device)
+    need = workspace_bytes(HLWQ_OP_GEMM, out_f, in_f, M)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.hlwq_gemm(_ptr(packed), _ptr(norms), _ptr(cb), out_f, in_f, M, _ptr(X), X.stride(0), _ptr(Y),
+                         Y.stride(0), _dtype_code(Y.dtype), _ptr(workspace), ws_bytes, _stream(stream)), "hlwq_gemm")
+    return Y
+
+
+def moe_gemv(gu, dn, cb, logits, X, topk: int, shared=None, out_dtype=torch.float32, Y=None, ids=None,
+             weights=None, workspace=None, stream=None):
+    """gu = (packed [E][2F][NBh][80], norms [E][2F][NBh]); dn = (packed [E][H][NBf][80], norms [E][H][NBf]);
+    shared = ((packed, norms) of gate_up, (packed, norms) of down) or None.
+    logits fp32 [T][E], X bf16 [T][H].  Returns (Y, ids, weights)."""
+    E, two_f = gu[0].shape[0], gu[0].shape[1]
+    F = two_f // 2
+    H = dn[0].shape[1]
+    T = X.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(T, H, dtype=out_dtype, device=dev)
+    if ids is None:
+        ids = torch.empty(T, topk, dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty(T, topk, dtype=torch.float32, device=dev)
+    need = workspace_bytes(HLWQ_OP_MOE, H, F, T, E, topk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    sg = shared[0] if shared is not None else (None, None)
+    sd = shared[1] if shared is not None else (None, None)
+    _check(lib.hlwq_moe_gemv(_ptr(gu[0]), _ptr(gu[1]), _ptr(dn[0]), _ptr(dn[1]), _ptr(sg[0]), _ptr(sg[1]),
+                             _ptr(sd[0]), _ptr(sd[1]), _ptr(cb), E, H, F, topk, T, _ptr(logits), _ptr(X), _ptr(Y),
+                             _dtype_code(Y.dtype), _ptr(ids), _ptr(weights), _ptr(workspace), workspace.numel(),
+                             _stream(stream)), "hlwq_moe_gemv")
+    return Y, ids, weights

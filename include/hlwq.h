@@ -1,0 +1,172 @@
+/*
+ * hlwq.h -- C ABI of libhlwq, a CUDA (sm_100a) implementation of HLWQ Q5
+ * (Hadamard-Lloyd Weight Quantization, 5 bits) and of the dequant-matmul that
+ * consumes its packed codes directly.
+ *
+ * The method (as described on the "Qwen3.6-35B-A3B -- HLWQ Q5" model card,
+ * section "Method", and restated on the "Qwopus3.6-27B-v2 . HLWQ Q5" card,
+ * "Methodology notes"):
+ *   [1] view W (out x in) as (out, NB, 128), NB = ceil(in / 128), the tail block
+ *       zero-padded;
+ *   [2] n = ||block||_2, stored as fp16;
+ *   [3] y = (block / n) @ H, H the 128 x 128 +-1 Sylvester-Hadamard matrix
+ *       H[i][j] = (-1)^popcount(i & j) (the orthonormal Hadamard x sqrt(128));
+ *   [4] code = index of the nearest of 32 Lloyd-Max centroids for N(0,1), ties
+ *       to the lower index;
+ *   [5] pack 8 codes into 5 bytes: code j of a block occupies bits [5j, 5j+5)
+ *       of the block's 80-byte little-endian bit string, least significant bit
+ *       first.
+ * Dequantisation: w_hat[o][128b + i] = n16[o][b] / 128 * sum_j c[k_obj] H[j][i].
+ *
+ * Storage contract (all row-major, caller-owned):
+ *   packed  uint8  [rows][NB][80]   (0.625 byte per weight, including the pad)
+ *   norms   binary16 bit patterns, uint16 [rows][NB]
+ *   codebook float32 [32], strictly ascending (as hlwq_lloyd_codebook returns)
+ * Activations are bfloat16 bit patterns (uint16).  Output dtype is chosen per
+ * call with hlwq_dtype.
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA device (or managed) memory on the current
+ *     device; "stream" is a cudaStream_t passed as void* (NULL = the legacy
+ *     default stream).  Device calls are asynchronous on that stream; errors
+ *     detected on the host are returned before anything is launched.
+ *   - The library allocates no memory.  Calls that need scratch take a
+ *     caller-provided device workspace sized by hlwq_workspace_bytes().
+ *   - Alignment: packed, W, W_out, X, Y and workspace must be 16-byte aligned
+ *     (torch allocations are); leading dimensions are in elements.
+ *   - Return value: HLWQ_OK (0) or a negative hlwq_status.
+ *   - A kernel never traps.  Conditions it can only see on the device (e.g. a
+ *     codebook that is not ascending) set bits in a device error word that
+ *     hlwq_device_error() reads (synchronously) and clears.
+ */
+#ifndef HLWQ_H
+#define HLWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HLWQ_OK = 0,
+  HLWQ_EINVAL = -1,       /* null pointer, non-positive size, bad levels / topk */
+  HLWQ_EALIGN = -2,       /* a pointer or leading dimension breaks the alignment rule */
+  HLWQ_EUNSUPPORTED = -3, /* a size or dtype combination this build does not handle */
+  HLWQ_ECUDA = -4,        /* a CUDA runtime call (launch, attribute) failed */
+  HLWQ_EWORKSPACE = -5    /* workspace is NULL or smaller than hlwq_workspace_bytes() */
+} hlwq_status;
+
+typedef enum { HLWQ_F32 = 0, HLWQ_BF16 = 1, HLWQ_F16 = 2 } hlwq_dtype;
+
+/* Operations whose scratch size hlwq_workspace_bytes() reports. */
+typedef enum { HLWQ_OP_GEMM = 1, HLWQ_OP_MOE = 2 } hlwq_op;
+
+/* Device error bits (hlwq_device_error). */
+#define HLWQ_DEVERR_CODEBOOK 0x1u  /* codebook not strictly ascending or not finite */
+#define HLWQ_DEVERR_TIMEOUT  0x2u  /* a bounded in-kernel wait gave up */
+
+/*
+ * Lloyd-Max codebook for N(0,1) (Method step [4]: "Lloyd-Max 5-bit quantization
+ * (32 centroids, N(0,1))").  Host-only, synchronous.
+ *   levels      2, 4, 8, 16 or 32 (the device calls use 32)
+ *   centroids   host float[levels], ascending, symmetric (c[L-1-k] = -c[k]):
+ *               the fixed point of Lloyd's conditions rounded to nearest fp32
+ *   midpoints   host float[levels-1] or NULL: (c[k] + c[k+1]) / 2 rounded to fp32
+ *   mse         host double* or NULL: E[(Z - q(Z))^2] of the fp64 fixed point
+ * Errors: HLWQ_EINVAL for another `levels` or a NULL centroids pointer.
+ */
+int hlwq_lloyd_codebook(int levels, float* centroids, float* midpoints, double* mse);
+
+/*
+ * Quantize `rows` x `in` weights (Method steps [1]-[5]); experts are stacked
+ * rows ("Gemma-4-26B-A4B-it-HLWQ-Q5", Technical Details: each expert is
+ * quantized independently -- rows never mix, so E experts of O rows are simply
+ * rows = E * O).
+ *   W         device, wdtype (HLWQ_F32 or HLWQ_BF16), [rows][in], row pitch = in
+ *   codebook  device float[32]
+ *   packed    device uint8 [rows][NB][80]   (output)
+ *   norms     device uint16 [rows][NB]      (output, binary16 bits)
+ * The norm is the exact L2 norm rounded to nearest binary16; codes are the
+ * nearest centroid of the exactly rotated value (decisions within 1e-5 of a
+ * midpoint are re-taken in fp64 on the device).
+ * Errors: HLWQ_EINVAL (NULL, rows/in <= 0), HLWQ_EUNSUPPORTED (wdtype),
+ *         HLWQ_EALIGN (W or packed not 16-byte aligned), HLWQ_ECUDA.
+ */
+int hlwq_quantize(const void* W, int wdtype, int64_t rows, int64_t in,
+                  const float* codebook, uint8_t* packed, uint16_t* norms, void* stream);
+
+/*
+ * Dequantize ("Qwopus3.6-27B-v2 . HLWQ Q5", Pipeline: dequantize per-Linear).
+ *   W_out  device, odtype (HLWQ_F32 or HLWQ_BF16), [rows][in]; pad dropped.
+ * Errors: as hlwq_quantize.
+ */
+int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+                    int64_t rows, int64_t in, void* W_out, int odtype, void* stream);
+
+/*
+ * Decode GEMV: y[o] = sum_i x[i] * w_hat[o][i], fp32 accumulation, without
+ * materialising w_hat (the activation is rotated once per 128-block and dotted
+ * with centroid values in the rotated domain).
+ *   x  device bf16 [in];   y  device ydtype [out] (HLWQ_F32 or HLWQ_BF16)
+ * Errors: HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_ECUDA.
+ */
+int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+              int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype, void* stream);
+
+/*
+ * Small-M GEMM: Y[m][o] = sum_i X[m][i] * w_hat[o][i], fp32 accumulation.
+ *   X  device bf16 [M][ldx] (ldx >= in, ldx % 8 == 0)
+ *   Y  device ydtype [M][ldy] (ldy >= out)
+ *   workspace  device, ws_bytes >= hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
+ * M < 16 runs on the CUDA-core decode path; M >= 16 on the tensor-core path.
+ */
+int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+              int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx,
+              void* Y, int64_t ldy, int ydtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Routed MoE layer ("Qwen3.6-35B-A3B -- HLWQ Q5": 8 routed + 1 shared expert):
+ *   ids, p   = top-k of router_logits[t] (ties: lower expert id), p = softmax
+ *              over the k selected logits;
+ *   g || u   = w_hat_gu[e] @ x_t  (rows [0,F) gate, [F,2F) up);
+ *   h        = SiLU(g) * u (kept fp32);
+ *   Y[t]     = sum_s p_s * w_hat_dn[ids_s] @ h  (+ shared expert, weight 1).
+ *   gu_*  [E][2F][NBh][80] / [E][2F][NBh],  NBh = ceil(H / 128)
+ *   dn_*  [E][H][NBf][80]  / [E][H][NBf],   NBf = ceil(F / 128)
+ *   sh_*  the shared expert's matrices, or all four NULL for none
+ *   router_logits device f32 [T][E];  X device bf16 [T][H];  Y device ydtype [T][H]
+ *   topk_ids / topk_weights  device int32 / f32 [T][topk], or NULL
+ * Errors: HLWQ_EINVAL (sizes, topk > E, topk > 32), HLWQ_EWORKSPACE, ...
+ */
+int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
+                  const uint8_t* dn_packed, const uint16_t* dn_norms,
+                  const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                  const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms,
+                  const float* codebook, int64_t E, int64_t H, int64_t F, int64_t topk,
+                  int64_t T, const float* router_logits, const uint16_t* X,
+                  void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
+                  void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Scratch bytes for an operation (0 when none is needed).
+ *   HLWQ_OP_GEMM: a = out, b = in, c = M
+ *   HLWQ_OP_MOE : a = H,   b = F,  c = T, E = experts, topk
+ */
+size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk);
+
+/* Reads (after synchronising the current device) and clears the device error word. */
+int hlwq_device_error(uint32_t* bits);
+
+/* Static description of a status code. */
+const char* hlwq_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hlwq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HLWQ_H */

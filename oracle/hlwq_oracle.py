@@ -287,7 +287,8 @@ def quantize(W, levels: int = LEVELS, return_rotated: bool = False):
 
     [1] view W as (out, n_blocks, 128), zero-padding the tail (reading R5);
     [2] n = ||block||_2 in fp64, stored as fp16 (reading R3);
-    [3] y = (block / n) @ H (+-1 Sylvester, reading R1); y = 0 for n = 0;
+    [3] y = (block / n) @ H (+-1 Sylvester, reading R1), evaluated as
+        (block @ H) / n; y = 0 for n = 0;
     [4] code = nearest fp32 centroid (ties to the lower index);
     [5] pack 8 codes per 5 bytes (reading R6).
 
@@ -304,8 +305,10 @@ def quantize(W, levels: int = LEVELS, return_rotated: bool = False):
     blocks = wp.reshape(O, nb, BLOCK)
     n = np.sqrt(np.sum(blocks * blocks, axis=-1))
     safe = np.where(n > 0.0, n, 1.0)
-    unit = np.where((n > 0.0)[..., None], blocks / safe[..., None], 0.0)
-    y = unit @ _H64
+    # (block / n) @ H evaluated as (block @ H) / n: the +-1 sum of fp32/bf16
+    # values is exact in fp64, so an exact tie (e.g. y = 0 on a constant block)
+    # stays a tie and is resolved by the tie rule, not by rounding noise.
+    y = np.where((n > 0.0)[..., None], (blocks @ _H64) / safe[..., None], 0.0)
     c32, _, _ = codebook_fp32(levels)
     codes = nearest_centroid(y, c32)
     out = {

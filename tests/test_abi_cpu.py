@@ -1,0 +1,82 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the header
+declares, the host codebook builder agrees bit-for-bit with the oracle, and
+argument validation rejects bad calls before anything is launched."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hl():
+    from dequant_matmul_b200 import build
+    build.build()
+    from dequant_matmul_b200 import hlwq
+    return hlwq
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "hlwq.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(hlwq_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(hl):
+    syms = header_symbols()
+    assert len(syms) >= 9
+    for s in syms:
+        assert hasattr(hl.lib, s), s
+        assert s in hl.SIGNATURES, s
+
+
+@pytest.mark.parametrize("levels", [2, 4, 8, 16, 32])
+def test_host_codebook_equals_oracle(hl, levels):
+    c, m, mse = hl.lloyd_codebook(levels)
+    c32, mid64, b32 = O.codebook_fp32(levels)
+    assert np.array_equal(c.numpy(), c32)
+    assert np.array_equal(m.numpy(), b32)
+    assert mse == pytest.approx(O.lloyd_max_gaussian(levels)["mse"], rel=1e-9)
+
+
+def test_codebook_rejects_bad_levels(hl):
+    buf = (ctypes.c_float * 64)()
+    for bad in (0, 1, 3, 64):
+        assert hl.lib.hlwq_lloyd_codebook(bad, ctypes.cast(buf, ctypes.c_void_p), None, None) == hl.HLWQ_EINVAL
+    assert hl.lib.hlwq_lloyd_codebook(32, None, None, None) == hl.HLWQ_EINVAL
+
+
+def test_validation_before_launch(hl):
+    L = hl.lib
+    p = ctypes.c_void_p(256)        # fake, 16-byte aligned, never dereferenced
+    odd = ctypes.c_void_p(257)
+    assert L.hlwq_quantize(None, hl.HLWQ_BF16, 4, 128, p, p, p, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_quantize(p, hl.HLWQ_BF16, 0, 128, p, p, p, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_quantize(p, hl.HLWQ_F16, 4, 128, p, p, p, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_quantize(p, hl.HLWQ_BF16, 4, 128, p, odd, p, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_dequantize(p, p, p, 4, -1, p, hl.HLWQ_F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_gemv(p, p, p, 4, 128, p, p, 7, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_gemm(p, p, p, 4, 128, 2, p, 64, p, 4, hl.HLWQ_BF16, None, 0, None) == hl.HLWQ_EINVAL  # ldx < in
+    ws = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 8, 256, 8)
+    assert ws > 0
+    args = [p, p, p, p, None, None, None, None, p, 256, 2048, 512, 8, 8, p, p, p, hl.HLWQ_F32, None, None]
+    assert L.hlwq_moe_gemv(*args, p, ws - 1, None) == hl.HLWQ_EWORKSPACE
+    bad_topk = list(args)
+    bad_topk[12] = 300
+    assert L.hlwq_moe_gemv(*bad_topk, p, ws, None) == hl.HLWQ_EINVAL
+    half_shared = list(args)
+    half_shared[4] = p
+    assert L.hlwq_moe_gemv(*half_shared, p, ws, None) == hl.HLWQ_EINVAL
+    assert hl.lib.hlwq_status_string(-5).decode().startswith("workspace")
+    assert hl.lib.hlwq_version() >= 100
+
+
+def test_workspace_sizes(hl):
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 4096, 4096, 1) == 0
+    a = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 1, 256, 8)
+    b = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 64, 256, 8)
+    assert 0 < a < b

@@ -1,0 +1,116 @@
+"""GPU parity: fused dequant GEMV / small-M GEMM against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from dequant_matmul_b200 import synth
+from gpu_helpers import MATMUL_REL, oracle_to_dev, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hl():
+    from dequant_matmul_b200 import hlwq
+    return hlwq
+
+
+@pytest.fixture(scope="module")
+def cb(hl):
+    return hl.codebook("cuda")
+
+
+def _layer(shape, seed):
+    W = synth.student_t(shape, df4_seed=seed)
+    return W, O.quantize(W)
+
+
+def test_gemv_256x512_fp32_outliers(hl, cb):
+    W = synth.gaussian_with_outliers(256, 512, seed=0)
+    q = O.quantize(W)
+    p, n = oracle_to_dev(q)
+    x = synth.activations(1, 512, seed=1)
+    y = hl.gemv(p, n, cb, x[0].cuda())
+    torch.cuda.synchronize()
+    want = O.matmul(q["packed"], q["norms"], 512, x)[0]
+    assert rel_l2(y.cpu().numpy(), want) <= MATMUL_REL
+
+
+@pytest.mark.parametrize("shape", [(5120, 5120), (300, 704), (37, 1000), (1, 128), (4099, 256)])
+def test_gemv_shapes(hl, cb, shape):
+    W, q = _layer(shape, seed=shape[0])
+    p, n = oracle_to_dev(q)
+    x = synth.activations(1, shape[1], seed=2)
+    for odt in (torch.float32, torch.bfloat16):
+        y = hl.gemv(p, n, cb, x[0].cuda(), out_dtype=odt)
+        torch.cuda.synchronize()
+        want = O.matmul(q["packed"], q["norms"], shape[1], x)[0]
+        tol = MATMUL_REL if odt == torch.float32 else MATMUL_REL
+        assert rel_l2(y.double().cpu().numpy(), want) <= tol, odt
+
+
+def test_gemv_activation_scale_extremes(hl, cb):
+    """Activations far from unit scale (the rotated activation is rescaled by a
+    power of two before it is stored in binary16)."""
+    W, q = _layer((128, 512), seed=9)
+    p, n = oracle_to_dev(q)
+    for s in (1e-20, 1e3, 3e4):
+        x = (synth.activations(1, 512, seed=3, dtype=torch.float32) * s).to(torch.bfloat16)
+        y = hl.gemv(p, n, cb, x[0].cuda())
+        torch.cuda.synchronize()
+        want = O.matmul(q["packed"], q["norms"], 512, x)[0]
+        assert rel_l2(y.cpu().numpy(), want) <= MATMUL_REL, s
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 9, 15, 16, 17, 64])
+def test_gemm_small_m(hl, cb, M):
+    W, q = _layer((1024, 5120), seed=21)
+    p, n = oracle_to_dev(q)
+    X = synth.activations(M, 5120, seed=M)
+    Y = hl.gemm(p, n, cb, X.cuda(), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    want = O.matmul(q["packed"], q["norms"], 5120, X)
+    assert rel_l2(Y.double().cpu().numpy(), want) <= MATMUL_REL
+
+
+def test_gemm_ragged_fp32_out_and_pitch(hl, cb):
+    W, q = _layer((200, 704), seed=5)
+    p, n = oracle_to_dev(q)
+    X = synth.activations(6, 720, seed=6)[:, :704]        # row pitch 720 > in
+    Xd = X.cuda()
+    Y = torch.full((6, 208), 7.0, device="cuda")          # row pitch 208 > out
+    hl.gemm(p, n, cb, Xd, Y=Y[:, :200].contiguous(), out_dtype=torch.float32)  # contiguous path
+    Y2 = torch.full((6, 208), 7.0, device="cuda")
+    hl.lib.hlwq_gemm(p.data_ptr(), n.data_ptr(), cb.data_ptr(), 200, 704, 6, Xd.data_ptr(), Xd.stride(0),
+                     Y2.data_ptr(), 208, hl.HLWQ_F32, None, 0, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    want = O.matmul(q["packed"], q["norms"], 704, X)
+    assert rel_l2(Y2[:, :200].cpu().numpy(), want) <= MATMUL_REL
+    assert torch.all(Y2[:, 200:] == 7.0)
+
+
+def test_gemm_m1_equals_gemv(hl, cb):
+    W, q = _layer((512, 1024), seed=8)
+    p, n = oracle_to_dev(q)
+    x = synth.activations(1, 1024, seed=4).cuda()
+    a = hl.gemv(p, n, cb, x[0])
+    b = hl.gemm(p, n, cb, x, out_dtype=torch.float32)[0]
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_gemv_full_27648x5120_sampled_rows(hl, cb):
+    """The 27648 x 5120 layer at full size (GPU-quantized); rows sampled for the
+    oracle, which encodes them itself from the same synthetic weights."""
+    W = synth.student_t((27648, 5120), df4_seed=0)
+    p, n = hl.quantize(W.cuda(), cb)
+    X = synth.activations(4, 5120, seed=11)
+    Y1 = hl.gemv(p, n, cb, X[0].cuda())
+    Y4 = hl.gemm(p, n, cb, X.cuda(), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(0).choice(27648, 384, replace=False))
+    q = O.quantize(W[rows])
+    want = O.matmul(q["packed"], q["norms"], 5120, X)
+    assert rel_l2(Y1.cpu().numpy()[rows], want[0]) <= MATMUL_REL
+    assert rel_l2(Y4.double().cpu().numpy()[:, rows], want) <= MATMUL_REL

@@ -239,3 +239,12 @@ def test_relative_reconstruction_error_is_lloyd_mse():
     rel = ((w_hat - wd) ** 2).sum() / (wd ** 2).sum()
     d = O.lloyd_max_gaussian(32)["mse"]
     assert abs(rel - d) / d < 0.05
+
+
+def test_exact_ties_resolve_low():
+    """Constant blocks: 127 rotated values are exactly 0 (a tie between codes 15
+    and 16 under the symmetric codebook) and must all take code 15."""
+    for v in (0.01, -0.02, 0.3):
+        q = O.quantize(torch.full((2, 256), v), return_rotated=True)
+        assert np.all(q["y"][..., 1:] == 0.0)
+        assert np.all(q["codes"][..., 1:] == 15)
