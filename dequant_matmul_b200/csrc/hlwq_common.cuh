@@ -40,13 +40,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
-// acc + a * b with a, b binary16 and fp32 accumulation (the product is exact).
-__device__ __forceinline__ float fma_f16_f32(uint16_t a, uint16_t b, float acc) {
-  float d;
-  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(acc));
-  return d;
-}
-
 // Extract 10 bits starting at bit `sh` of the 64-bit pair (lo, hi).
 template <int SH>
 __device__ __forceinline__ uint32_t bits10(uint32_t lo, uint32_t hi) {

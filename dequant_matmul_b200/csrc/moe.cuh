@@ -43,7 +43,7 @@ struct MoeWs {
   int* sel_id;        // [T][topk]
   float* sel_w;       // [T][topk]
   uint16_t* xt;       // [T][NBh][kXsStride] rotated tokens (binary16)
-  float* xt_inv;      // [T]
+  float* xt_inv;      // [T][NBh] per-block activation scales
   float* h;           // [NA][F]
   float* part;        // [NA][H]
 };
@@ -69,7 +69,7 @@ size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char
   w.sel_id = reinterpret_cast<int*>(take(sizeof(int) * T * topk));
   w.sel_w = reinterpret_cast<float*>(take(sizeof(float) * T * topk));
   w.xt = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * T * nbh * kXsStride));
-  w.xt_inv = reinterpret_cast<float*>(take(sizeof(float) * T));
+  w.xt_inv = reinterpret_cast<float*>(take(sizeof(float) * T * nbh));
   w.h = reinterpret_cast<float*>(take(sizeof(float) * na * F));
   w.part = reinterpret_cast<float*>(take(sizeof(float) * na * H));
   if (ws) *ws = w;
@@ -175,36 +175,54 @@ router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, 
   if (!has_shared)
     for (int t = threadIdx.x; t < T; t += kRouterThreads) ws.tok_asg[t * (topk + 1) + topk] = -1;
 
-  // 3. rotated activations of every token (binary16, per-token power-of-two scale).
+  // 3. rotated activations of every token (binary16, per-block power-of-two scale).
   const int nbh = (H + kBlock - 1) / kBlock;
-  for (int t = 0; t < T; ++t)
-    rotate_activations_bf16(X + static_cast<int64_t>(t) * H, H, H, nbh, 1, 1,
-                            ws.xt + static_cast<int64_t>(t) * nbh * kXsStride, ws.xt_inv + t, red);
+  rotate_tokens_bf16(X, H, H, nbh, T, T, ws.xt, ws.xt_inv);
 }
 
-template <int C>
-__device__ void gate_up_unit_pass(int mt, const uint32_t* tab, const uint16_t* xs, const uint8_t* packed,
-                                  const uint16_t* norms, int nb, int jt, int j0, int F, float* slots) {
-  auto rowfn = [=](int v) { return static_cast<int64_t>(v < jt ? j0 + v : F + j0 + (v - jt)); };
-  switch (mt) {
-    case 1: engine_items<C, 1>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
-    case 2: engine_items<C, 2>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
-    default: engine_items<C, 4>(tab, xs, packed, norms, nb, 2 * jt, rowfn, slots); break;
+// One pass of up to MT tokens of a gate_up unit: prefetch codes, stage the
+// tokens' rotated activations, decode (results in slots).
+template <int C, int MT, typename RowFn>
+__device__ __forceinline__ void gate_up_pass(const uint8_t* pk, const uint16_t* nm, int nb, int jt, RowFn rowfn,
+                                             const MoeWs& ws, int a_first, int ntok, const uint32_t* tab,
+                                             uint16_t* xs, float* xinv, float* slots) {
+  auto eng = make_engine<C, MT, 2>(pk, nm, nb, 2 * jt, rowfn);
+  eng.prefetch();
+  const int words = nb * kXsStride / 8;  // uint4 per token
+  for (int q = threadIdx.x; q < MT * words; q += blockDim.x) {
+    const int m = q / words, w = q - m * words;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (m < ntok) {
+      const int t = ws.asg_token[a_first + m];
+      val = reinterpret_cast<const uint4*>(ws.xt + static_cast<int64_t>(t) * nb * kXsStride)[w];
+    }
+    reinterpret_cast<uint4*>(xs)[q] = val;
   }
-}
-
-template <int C>
-__device__ void down_unit_pass(int mt, const uint32_t* tab, const uint16_t* xs, const uint8_t* packed,
-                               const uint16_t* norms, int nb, int nr, int r0, float* slots) {
-  auto rowfn = [=](int v) { return static_cast<int64_t>(r0 + v); };
-  switch (mt) {
-    case 1: engine_items<C, 1>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
-    case 2: engine_items<C, 2>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
-    default: engine_items<C, 4>(tab, xs, packed, norms, nb, nr, rowfn, slots); break;
+  for (int q = threadIdx.x; q < MT * nb; q += blockDim.x) {
+    const int m = q / nb, b = q - m * nb;
+    xinv[q] = m < ntok ? ws.xt_inv[static_cast<int64_t>(ws.asg_token[a_first + m]) * nb + b] : 0.0f;
   }
+  __syncthreads();
+  eng.run(tab, xs, xinv, slots);
+  __syncthreads();
 }
 
-__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : (ntok <= 2 ? 2 : 4); }
+// One pass of up to MT assignments of a down unit: prefetch codes, rotate the
+// assignments' h rows in the CTA, decode (results in slots).
+template <int C, int MT, typename RowFn>
+__device__ __forceinline__ void down_pass(const uint8_t* pk, const uint16_t* nm, int nb, int nr, RowFn rowfn,
+                                          const float* hbase, int F, int ntok, const uint32_t* tab, uint16_t* xs,
+                                          float* xinv, float* slots) {
+  auto eng = make_engine<C, MT, 2>(pk, nm, nb, nr, rowfn);
+  eng.prefetch();
+  rotate_tokens_f32([=](int m) { return hbase + static_cast<int64_t>(m) * F; }, F, nb, ntok, MT, xs, xinv);
+  __syncthreads();
+  eng.run(tab, xs, xinv, slots);
+  __syncthreads();
+}
+
+__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : 2; }
+constexpr int kMoePass = 2;  // tokens per decode pass of a unit
 
 template <int C>
 __global__ void __launch_bounds__(kEngineThreads, 1)
@@ -214,12 +232,12 @@ gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict
   extern __shared__ __align__(16) uint8_t smem[];
   const int nb = (H + kBlock - 1) / kBlock;
   const int nch = (nb + C - 1) / C;
-  const EngineLayout L = engine_layout(4, nb, 2 * kJT, nch);
+  const EngineLayout L = engine_layout(kMoePass, nb, 2 * kJT, nch);
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
+  float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
   float* slots = reinterpret_cast<float*>(smem + L.slot_off);
   float* misc = reinterpret_cast<float*>(smem + L.misc_off);
-  float* inv = misc + 48;
   uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
   build_pair_table(tab, c16, codebook);
   __syncthreads();
@@ -234,23 +252,11 @@ gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict
     const uint8_t* pk = e < E ? gu_packed + e * expert_rows * nb * kBlockBytes : sh_packed;
     const uint16_t* nm = e < E ? gu_norms + e * expert_rows * nb : sh_norms;
     const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
-    for (int m0 = 0; m0 < ne; m0 += 4) {
-      const int ntok = min(4, ne - m0), mt = pass_mt(ntok);
-      // stage the tokens' rotated activations
-      const int words = nb * kXsStride / 8;  // uint4 per token
-      for (int q = threadIdx.x; q < mt * words; q += blockDim.x) {
-        const int m = q / words, w = q - m * words;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (m < ntok) {
-          const int t = ws.asg_token[a0 + m0 + m];
-          val = reinterpret_cast<const uint4*>(ws.xt + static_cast<int64_t>(t) * nb * kXsStride)[w];
-        }
-        reinterpret_cast<uint4*>(xs)[q] = val;
-      }
-      if (threadIdx.x < 4) inv[threadIdx.x] = threadIdx.x < ntok ? ws.xt_inv[ws.asg_token[a0 + m0 + threadIdx.x]] : 0.0f;
-      __syncthreads();
-      gate_up_unit_pass<C>(mt, tab, xs, pk, nm, nb, jt, j0, F, slots);
-      __syncthreads();
+    for (int m0 = 0; m0 < ne; m0 += kMoePass) {
+      const int ntok = min(kMoePass, ne - m0), mt = pass_mt(ntok);
+      auto rowfn = [=](int v) { return static_cast<int64_t>(v < jt ? j0 + v : F + j0 + (v - jt)); };
+      if (mt == 1) gate_up_pass<C, 1>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
+      else gate_up_pass<C, 2>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
       const int nv = 2 * jt;
       for (int idx = threadIdx.x; idx < ntok * jt; idx += blockDim.x) {
         const int m = idx / jt, j = idx - m * jt;
@@ -258,8 +264,6 @@ gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict
         const float* su = slots + (m * nv + jt + j) * nch;
         float g = 0.0f, up = 0.0f;
         for (int ch = 0; ch < nch; ++ch) { g += sg[ch]; up += su[ch]; }
-        g *= inv[m];
-        up *= inv[m];
         const float hval = g / (1.0f + expf(-g)) * up;
         ws.h[static_cast<int64_t>(a0 + m0 + m) * F + j0 + j] = hval;
       }
@@ -276,12 +280,12 @@ down_kernel(const uint8_t* __restrict__ dn_packed, const uint16_t* __restrict__ 
   extern __shared__ __align__(16) uint8_t smem[];
   const int nb = (F + kBlock - 1) / kBlock;
   const int nch = (nb + C - 1) / C;
-  const EngineLayout L = engine_layout(4, nb, kHT, nch);
+  const EngineLayout L = engine_layout(kMoePass, nb, kHT, nch);
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
+  float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
   float* slots = reinterpret_cast<float*>(smem + L.slot_off);
   float* misc = reinterpret_cast<float*>(smem + L.misc_off);
-  float* inv = misc + 48;
   uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
   build_pair_table(tab, c16, codebook);
   __syncthreads();
@@ -295,20 +299,19 @@ down_kernel(const uint8_t* __restrict__ dn_packed, const uint16_t* __restrict__ 
     const uint8_t* pk = e < E ? dn_packed + static_cast<int64_t>(e) * H * nb * kBlockBytes : sh_packed;
     const uint16_t* nm = e < E ? dn_norms + static_cast<int64_t>(e) * H * nb : sh_norms;
     const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
-    for (int m0 = 0; m0 < ne; m0 += 4) {
-      const int ntok = min(4, ne - m0), mt = pass_mt(ntok);
+    for (int m0 = 0; m0 < ne; m0 += kMoePass) {
+      const int ntok = min(kMoePass, ne - m0), mt = pass_mt(ntok);
       const float* hbase = ws.h + static_cast<int64_t>(a0 + m0) * F;
-      rotate_activations_f32([=](int m) { return hbase + static_cast<int64_t>(m) * F; }, F, nb, ntok, mt, xs, inv,
-                             misc);
-      down_unit_pass<C>(mt, tab, xs, pk, nm, nb, nr, r0, slots);
-      __syncthreads();
+      auto rowfn = [=](int v) { return static_cast<int64_t>(r0 + v); };
+      if (mt == 1) down_pass<C, 1>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
+      else down_pass<C, 2>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
       for (int idx = threadIdx.x; idx < ntok * nr; idx += blockDim.x) {
         const int m = idx / nr, v = idx - m * nr;
         const float* sl = slots + (m * nr + v) * nch;
         float sum = 0.0f;
         for (int ch = 0; ch < nch; ++ch) sum += sl[ch];
         const int asg = a0 + m0 + m;
-        ws.part[static_cast<int64_t>(asg) * H + r0 + v] = sum * inv[m] * ws.asg_weight[asg];
+        ws.part[static_cast<int64_t>(asg) * H + r0 + v] = sum * ws.asg_weight[asg];
       }
       __syncthreads();
     }
@@ -353,8 +356,8 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
 
   const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
   const int cg = pick_chunk(nbh), cd = pick_chunk(nbf);
-  const int smem_g = engine_layout(4, nbh, 2 * kJT, (nbh + cg - 1) / cg).total;
-  const int smem_d = engine_layout(4, nbf, kHT, (nbf + cd - 1) / cd).total;
+  const int smem_g = engine_layout(kMoePass, nbh, 2 * kJT, (nbh + cg - 1) / cg).total;
+  const int smem_d = engine_layout(kMoePass, nbf, kHT, (nbf + cd - 1) / cd).total;
   if (smem_g > 227 * 1024 || smem_d > 227 * 1024) return HLWQ_EUNSUPPORTED;
   const int grid = sm_count();
   static bool attrs = false;

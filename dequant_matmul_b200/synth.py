@@ -71,3 +71,29 @@ def router_logits(tokens: int, experts: int, seed: int = 2) -> torch.Tensor:
 def uniform(shape, lo: float, hi: float, seed: int) -> np.ndarray:
     """Plain fp64 uniforms (used for rotated-domain probe values in tests)."""
     return _rng(seed).uniform(lo, hi, size=shape)
+
+
+def student_t_device(shape, std: float = 0.02, seed: int = 0, dtype=torch.bfloat16,
+                     device="cuda") -> torch.Tensor:
+    """The same Student-t(4) recipe drawn on the device with torch's seeded
+    generator (a different random stream from ``student_t``): used where the
+    host would take too long to draw a large benchmark workload."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    n = int(np.prod(shape))
+    out = torch.empty(n, dtype=dtype, device=device)
+    scale = std / math.sqrt(2.0)
+    chunk = 1 << 26
+    for s in range(0, n, chunk):
+        m = min(chunk, n - s)
+        z = torch.randn(m, generator=g, device=device)
+        u = torch.rand(2, m, generator=g, device=device)
+        chi2 = -2.0 * torch.log((1.0 - u[0]) * (1.0 - u[1]))
+        out[s:s + m] = (z / torch.sqrt(chi2 / 4.0) * scale).to(dtype)
+    return out.view(shape)
+
+
+def activations_device(rows: int, cols: int, seed: int = 1, dtype=torch.bfloat16, device="cuda") -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn(rows, cols, generator=g, device=device).to(dtype)
