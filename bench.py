@@ -183,9 +183,12 @@ def bench_quantize(hl, cb, peaks, stream):
         hl.quantize(w_dn, cb, p_dn, n_dn, stream=stream)
 
     ms, _ = time_graph(quant_layer, reps=10, warmup=3, stream=stream)
+    ms_gu, _ = time_graph(lambda: hl.quantize(w_gu, cb, p_gu, n_gu, stream=stream), reps=10, warmup=2, stream=stream)
+    ms_dn, _ = time_graph(lambda: hl.quantize(w_dn, cb, p_dn, n_dn, stream=stream), reps=10, warmup=2, stream=stream)
     n_w = E * (GU[0] * GU[1] + DN[0] * DN[1])
     qbytes = 2 * n_w + (p_gu.numel() + p_dn.numel()) + 2 * (n_gu.numel() + n_dn.numel())
     out["quantize"] = {"workload": "128 experts x (1408x2816 + 2816x704) bf16 -> Q5", "ms": round(ms, 4),
+                       "ms_gate_up": round(ms_gu, 4), "ms_down": round(ms_dn, 4),
                        "gweights_per_s": round(n_w / ms / 1e6, 2),
                        "roofline": {"bound": "hbm", "achieved": round(qbytes / ms / 1e6, 1), "peak": peaks["hbm_gbs"],
                                     "unit": "GB/s", "frac": frac(qbytes / ms / 1e6, peaks["hbm_gbs"]),

@@ -73,6 +73,11 @@ __device__ __forceinline__ void build_pair_table(uint32_t* tab, uint16_t* c16, c
   }
 }
 
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+         (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+}
+
 // Rotates one 128-block held 4 values per lane (x_b @ H, Sylvester order:
 // butterflies over the lane's 4 values, then over lanes with shuffles), picks
 // a power-of-two scale 2^k so that max|x_tilde| * 2^k lies in [2^9, 2^10) (so
@@ -125,6 +130,85 @@ __device__ __forceinline__ void rotate_tokens_bf16(const uint16_t* __restrict__ 
   }
 }
 
+// Rotation with four lanes per 128-block (32 consecutive values per lane: five
+// butterfly stages in registers, two across the block's lanes).  Warps
+// [w0, w0 + nw) of the CTA take part; each covers 8 blocks per step.  The
+// block's values are scaled by a power of two so that max |x_tilde| lies in
+// [2^9, 2^10) and stored as binary16; the inverse scale goes to inv_scale[b].
+__device__ __forceinline__ void rotate_row_q4(const uint16_t* __restrict__ X, int in, int nb, uint16_t* xs,
+                                              float* inv_scale, int w0, int nw) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane & 3;
+  if (warp < w0 || warp >= w0 + nw) return;
+  for (int bb = (warp - w0) * 8; bb < nb; bb += nw * 8) {
+    const int b = bb + (lane >> 2);
+    const bool act = b < nb;
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int i = kBlock * b + 32 * q + e;
+      v[e] = (act && i < in) ? bf16_bits_to_float(__ldg(X + i)) : 0.0f;
+    }
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if ((i & h) == 0) {
+          const float a = v[i], c = v[i + h];
+          v[i] = a + c;
+          v[i + h] = a - c;
+        }
+    }
+#pragma unroll
+    for (int lm = 1; lm <= 2; lm <<= 1) {
+      const float sgn = (lane & lm) ? -1.0f : 1.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(v[i], sgn, __shfl_xor_sync(0xffffffffu, v[i], lm));
+    }
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    int ex = 0;
+    if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
+    const int k = max(-120, min(120, 10 - ex));
+    const float sc = ldexpf(1.0f, k);
+    if (act) {
+      uint4* dst = reinterpret_cast<uint4*>(xs + b * kXsStride + 32 * q);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = pack_half2(v[8 * c] * sc, v[8 * c + 1] * sc);
+        u.y = pack_half2(v[8 * c + 2] * sc, v[8 * c + 3] * sc);
+        u.z = pack_half2(v[8 * c + 4] * sc, v[8 * c + 5] * sc);
+        u.w = pack_half2(v[8 * c + 6] * sc, v[8 * c + 7] * sc);
+        dst[c] = u;
+      }
+      if (q == 0) inv_scale[b] = ldexpf(1.0f, -k);
+    }
+  }
+}
+
+// Pair table build by warps [w0, w0 + nw) only (see build_pair_table).
+__device__ __forceinline__ void build_pair_table_warps(uint32_t* tab, const uint16_t* c16, int w0, int nw) {
+  const int warp = threadIdx.x >> 5;
+  if (warp < w0 || warp >= w0 + nw) return;
+  uint4* t4 = reinterpret_cast<uint4*>(tab);
+  for (int q = (warp - w0) * 32 + (threadIdx.x & 31); q < 1024 * 8; q += nw * 32) {
+    const int v = q >> 3;
+    const uint32_t e = static_cast<uint32_t>(c16[v & 31]) | (static_cast<uint32_t>(c16[v >> 5]) << 16);
+    t4[q] = make_uint4(e, e, e, e);
+  }
+}
+
+__device__ __forceinline__ void load_codebook16(uint16_t* c16, const float* __restrict__ codebook) {
+  if (threadIdx.x < kLevels) {
+    const float c = __ldg(codebook + threadIdx.x);
+    c16[threadIdx.x] = __half_as_ushort(__float2half_rn(c));
+    if (threadIdx.x + 1 < kLevels && !(c < __ldg(codebook + threadIdx.x + 1))) raise_device_error(HLWQ_DEVERR_CODEBOOK);
+  }
+}
+
 // Same for fp32 source rows given by rowptr(m) (the MoE intermediate h).
 template <typename RowPtr>
 __device__ __forceinline__ void rotate_tokens_f32(RowPtr rowptr, int in, int nb, int ntok, int mt, uint16_t* xs,
@@ -163,53 +247,99 @@ __device__ __forceinline__ uint32_t comp_of(const uint4& u, int t) {
   }
 }
 
-__device__ __forceinline__ __half2 u2h(uint32_t v) { return *reinterpret_cast<const __half2*>(&v); }
-
-// Table entries of the 8 code pairs of round r8 (pairs 8 r8 .. 8 r8 + 7).
-template <int R8>
-__device__ __forceinline__ void round_entries(const uint4 (&cw)[5], const uint32_t* __restrict__ tab_lane,
-                                              uint32_t (&ent)[8]) {
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const int bit = 80 * R8 + 10 * t, wi = bit >> 5, sh = bit & 31;
-    const uint32_t lo = word_of(cw, wi);
-    const uint32_t hi = (wi + 1 < 20) ? word_of(cw, wi + 1) : 0u;
-    const uint32_t v10 = (sh <= 22) ? ((lo >> sh) & 0x3ffu) : (__funnelshift_r(lo, hi, sh) & 0x3ffu);
-    ent[t] = tab_lane[v10 << 5];
-  }
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
-// sum_t c-pair(ent[t]) . x-pair(x[t]) for 8 pairs: four half2 product chains of
-// two pairs each, combined pairwise in half2 and finally in fp32 (the rotated
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Shared-memory byte address of the table entry of the code pair at bit BIT of
+// a block (20 words): ((pair << 7) + lane_base), the pair field moved to bit 7
+// with one shift (or funnel shift) and masked.
+template <int BIT>
+__device__ __forceinline__ uint32_t pair_addr(const uint4 (&cw)[5], uint32_t lane_base) {
+  constexpr int wi = BIT >> 5, sh = BIT & 31;
+  const uint32_t lo = word_of(cw, wi);
+  uint32_t t;
+  if constexpr (sh > 22) {
+    t = __funnelshift_r(lo, word_of(cw, wi + 1), sh - 7);
+  } else if constexpr (sh >= 7) {
+    t = lo >> (sh - 7);
+  } else {
+    t = lo << (7 - sh);
+  }
+  return (t & (0x3ffu << 7)) + lane_base;
+}
+
+// Table entries (binary16 centroid pairs) of the 8 code pairs of round R8.
+template <int R8>
+__device__ __forceinline__ void round_entries(const uint4 (&cw)[5], uint32_t lane_base, uint32_t (&ent)[8]) {
+  ent[0] = lds_u32(pair_addr<80 * R8 + 0>(cw, lane_base));
+  ent[1] = lds_u32(pair_addr<80 * R8 + 10>(cw, lane_base));
+  ent[2] = lds_u32(pair_addr<80 * R8 + 20>(cw, lane_base));
+  ent[3] = lds_u32(pair_addr<80 * R8 + 30>(cw, lane_base));
+  ent[4] = lds_u32(pair_addr<80 * R8 + 40>(cw, lane_base));
+  ent[5] = lds_u32(pair_addr<80 * R8 + 50>(cw, lane_base));
+  ent[6] = lds_u32(pair_addr<80 * R8 + 60>(cw, lane_base));
+  ent[7] = lds_u32(pair_addr<80 * R8 + 70>(cw, lane_base));
+}
+
+// sum over 8 pairs of c-pair . x-pair: four half2 product chains of two pairs,
+// combined pairwise in half2, the last two halves added in fp32 (the rotated
 // activation is scaled so that |x| < 2^10, far from binary16 overflow).
 __device__ __forceinline__ float round_dot(const uint32_t (&ent)[8], uint32_t x0, uint32_t x1, uint32_t x2,
                                            uint32_t x3, uint32_t x4, uint32_t x5, uint32_t x6, uint32_t x7) {
-  __half2 h0 = __hmul2(u2h(ent[0]), u2h(x0));
-  __half2 h1 = __hmul2(u2h(ent[1]), u2h(x1));
-  __half2 h2 = __hmul2(u2h(ent[2]), u2h(x2));
-  __half2 h3 = __hmul2(u2h(ent[3]), u2h(x3));
-  h0 = __hfma2(u2h(ent[4]), u2h(x4), h0);
-  h1 = __hfma2(u2h(ent[5]), u2h(x5), h1);
-  h2 = __hfma2(u2h(ent[6]), u2h(x6), h2);
-  h3 = __hfma2(u2h(ent[7]), u2h(x7), h3);
-  const float2 f = __half22float2(__hadd2(__hadd2(h0, h1), __hadd2(h2, h3)));
+  uint32_t h0 = hmul2(ent[0], x0);
+  uint32_t h1 = hmul2(ent[1], x1);
+  uint32_t h2 = hmul2(ent[2], x2);
+  uint32_t h3 = hmul2(ent[3], x3);
+  h0 = hfma2(ent[4], x4, h0);
+  h1 = hfma2(ent[5], x5, h1);
+  h2 = hfma2(ent[6], x6, h2);
+  h3 = hfma2(ent[7], x7, h3);
+  const uint32_t hs = hadd2(hadd2(h0, h1), hadd2(h2, h3));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hs));
   return f.x + f.y;
 }
 
 // Dot products of one (row, block) of codes with MT rotated activation blocks
-// stored in shared memory (xb: block base of token 0, xs_tok_stride halves per token).
+// in shared memory (xb_addr: shared address of token 0's block, tok_bytes per token).
 template <int MT>
-__device__ __forceinline__ void block_dot(const uint4 (&cw)[5], const uint32_t* __restrict__ tab_lane,
-                                          const uint16_t* __restrict__ xb, int xs_tok_stride, float (&acc)[MT]) {
+__device__ __forceinline__ void block_dot(const uint4 (&cw)[5], uint32_t lane_base, uint32_t xb_addr, int tok_bytes,
+                                          float (&acc)[MT]) {
 #pragma unroll
   for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
 #define HLWQ_ROUND(R8)                                                                                   \
   {                                                                                                      \
     uint32_t ent[8];                                                                                     \
-    round_entries<R8>(cw, tab_lane, ent);                                                                \
+    round_entries<R8>(cw, lane_base, ent);                                                               \
     _Pragma("unroll") for (int m = 0; m < MT; ++m) {                                                     \
-      const uint4 xa = *reinterpret_cast<const uint4*>(xb + m * xs_tok_stride + 16 * (R8));             \
-      const uint4 xc = *reinterpret_cast<const uint4*>(xb + m * xs_tok_stride + 16 * (R8) + 8);         \
+      const uint4 xa = lds_u128(xb_addr + m * tok_bytes + 32 * (R8));                                    \
+      const uint4 xc = lds_u128(xb_addr + m * tok_bytes + 32 * (R8) + 16);                               \
       acc[m] += round_dot(ent, xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w);                         \
     }                                                                                                    \
   }
@@ -219,13 +349,12 @@ __device__ __forceinline__ void block_dot(const uint4 (&cw)[5], const uint32_t* 
 
 // Single-token dot product with the rotated activation block held in registers
 // (64 half2 words, xr[p] = (x[2p], x[2p+1])).
-__device__ __forceinline__ float block_dot_reg(const uint4 (&cw)[5], const uint32_t* __restrict__ tab_lane,
-                                               const uint32_t (&xr)[64]) {
+__device__ __forceinline__ float block_dot_reg(const uint4 (&cw)[5], uint32_t lane_base, const uint32_t (&xr)[64]) {
   float acc = 0.0f;
 #define HLWQ_ROUND1(R8)                                                                                  \
   {                                                                                                      \
     uint32_t ent[8];                                                                                     \
-    round_entries<R8>(cw, tab_lane, ent);                                                                \
+    round_entries<R8>(cw, lane_base, ent);                                                               \
     acc += round_dot(ent, xr[8 * (R8)], xr[8 * (R8) + 1], xr[8 * (R8) + 2], xr[8 * (R8) + 3],           \
                      xr[8 * (R8) + 4], xr[8 * (R8) + 5], xr[8 * (R8) + 6], xr[8 * (R8) + 7]);           \
   }
@@ -233,6 +362,71 @@ __device__ __forceinline__ float block_dot_reg(const uint4 (&cw)[5], const uint3
   HLWQ_ROUND1(4) HLWQ_ROUND1(5) HLWQ_ROUND1(6) HLWQ_ROUND1(7)
 #undef HLWQ_ROUND1
   return acc;
+}
+
+__device__ __forceinline__ uint32_t word10(const uint2 (&c)[5], int i) {
+  const uint2 u = c[i >> 1];
+  return (i & 1) ? u.y : u.x;
+}
+
+// Address of the table entry of pair p (0..31) of a half block (10 words).
+template <int P>
+__device__ __forceinline__ uint32_t half_pair_addr(const uint2 (&cw)[5], uint32_t lane_base) {
+  constexpr int bit = 10 * P, wi = bit >> 5, sh = bit & 31;
+  const uint32_t lo = word10(cw, wi);
+  uint32_t t;
+  if constexpr (sh > 22) {
+    t = __funnelshift_r(lo, word10(cw, wi + 1), sh - 7);
+  } else if constexpr (sh >= 7) {
+    t = lo >> (sh - 7);
+  } else {
+    t = lo << (7 - sh);
+  }
+  return (t & (0x3ffu << 7)) + lane_base;
+}
+
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 8 pairs: two half2 chains of 4 products each (even / odd pairs), one half2
+// add, widened to fp32 and added to a packed fp32 pair accumulator.
+template <int P0>
+__device__ __forceinline__ void half_round(const uint2 (&cw)[5], uint32_t lane_base, const uint32_t (&xr)[32],
+                                           uint64_t& acc2) {
+  uint32_t e[8];
+  e[0] = lds_u32(half_pair_addr<P0 + 0>(cw, lane_base));
+  e[1] = lds_u32(half_pair_addr<P0 + 1>(cw, lane_base));
+  e[2] = lds_u32(half_pair_addr<P0 + 2>(cw, lane_base));
+  e[3] = lds_u32(half_pair_addr<P0 + 3>(cw, lane_base));
+  e[4] = lds_u32(half_pair_addr<P0 + 4>(cw, lane_base));
+  e[5] = lds_u32(half_pair_addr<P0 + 5>(cw, lane_base));
+  e[6] = lds_u32(half_pair_addr<P0 + 6>(cw, lane_base));
+  e[7] = lds_u32(half_pair_addr<P0 + 7>(cw, lane_base));
+  uint32_t h0 = hmul2(e[0], xr[P0 + 0]);
+  uint32_t h1 = hmul2(e[1], xr[P0 + 1]);
+  h0 = hfma2(e[2], xr[P0 + 2], h0);
+  h1 = hfma2(e[3], xr[P0 + 3], h1);
+  h0 = hfma2(e[4], xr[P0 + 4], h0);
+  h1 = hfma2(e[5], xr[P0 + 5], h1);
+  h0 = hfma2(e[6], xr[P0 + 6], h0);
+  h1 = hfma2(e[7], xr[P0 + 7], h1);
+  const uint32_t hs = hadd2(h0, h1);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hs));
+  acc2 = f32x2_add(acc2, (static_cast<uint64_t>(__float_as_uint(f.y)) << 32) | __float_as_uint(f.x));
+}
+
+// Single-token dot product of a half block (64 codes) with 64 rotated
+// activation values held in registers (xr[p] = (x[2p], x[2p+1])).
+__device__ __forceinline__ float half_dot_reg(const uint2 (&cw)[5], uint32_t lane_base, const uint32_t (&xr)[32]) {
+  uint64_t acc2 = 0;
+  half_round<0>(cw, lane_base, xr, acc2);
+  half_round<8>(cw, lane_base, xr, acc2);
+  half_round<16>(cw, lane_base, xr, acc2);
+  half_round<24>(cw, lane_base, xr, acc2);
+  return __uint_as_float(static_cast<uint32_t>(acc2)) + __uint_as_float(static_cast<uint32_t>(acc2 >> 32));
 }
 
 // Processes all items of a CTA's virtual-row range.  rowfn(vrow) returns the
@@ -283,16 +477,15 @@ struct Engine {
     for (int d = 0; d < kDepth; ++d) fetch(warp + d * kEngineWarps, d);
   }
 
-  __device__ __forceinline__ void consume(int it, int d, const uint32_t* __restrict__ tab_lane,
-                                          const uint16_t* __restrict__ xs, const float* __restrict__ xinv,
-                                          float* __restrict__ slots) {
+  __device__ __forceinline__ void consume(int it, int d, uint32_t lane_base, uint32_t xs_addr,
+                                          const float* __restrict__ xinv, float* __restrict__ slots) {
     const int lane = threadIdx.x & 31;
     const int r = lane / C, s = lane % C;
     const int g = it / nch, ch = it - g * nch;
     const int b = ch * C + s;
     float acc[MT];
     if (ok[d]) {
-      block_dot<MT>(cw[d], tab_lane, xs + b * kXsStride, nb * kXsStride, acc);
+      block_dot<MT>(cw[d], lane_base, xs_addr + b * (kXsStride * 2), nb * kXsStride * 2, acc);
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[m] *= sc[d] * xinv[m * nb + b];
     } else {
@@ -314,13 +507,14 @@ struct Engine {
   __device__ __forceinline__ void run(const uint32_t* __restrict__ tab, const uint16_t* __restrict__ xs,
                                       const float* __restrict__ xinv, float* __restrict__ slots) {
     const int warp = threadIdx.x >> 5;
-    const uint32_t* tab_lane = tab + (threadIdx.x & 31);
+    const uint32_t lane_base = static_cast<uint32_t>(__cvta_generic_to_shared(tab)) + 4u * (threadIdx.x & 31);
+    const uint32_t xs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
     for (int base = warp; base < nitems; base += kDepth * kEngineWarps) {
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         const int it = base + d * kEngineWarps;
         if (it < nitems) {
-          consume(it, d, tab_lane, xs, xinv, slots);
+          consume(it, d, lane_base, xs_addr, xinv, slots);
           fetch(it + kDepth * kEngineWarps, d);
         }
       }

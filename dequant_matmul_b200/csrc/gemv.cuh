@@ -69,11 +69,14 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 }
 
 
-// Single-token GEMV.  256 threads (8 warps) per CTA, one CTA per SM.  A CTA's
-// items are ordered chunk-major and each warp takes a contiguous range of
-// them, so a lane's 128-block of the rotated activation (64 half2 registers)
-// is reloaded only when the warp's range crosses into the next chunk.
-constexpr int kGemv1Threads = 256;
+// Single-token GEMV.  512 threads (16 warps) per CTA, one CTA per SM (the
+// 128 KiB pair table).  A lane owns half a 128-block (64 codes, 40 bytes): lane
+// (r, s, h) takes row r, block s of the chunk and half h, so the 2C lanes of a
+// row read 80 C contiguous bytes.  A CTA's items are ordered chunk-major and
+// each warp takes a contiguous range of them, so a lane's 64 rotated
+// activation values (32 half2 registers) are reloaded only when the range
+// crosses into the next chunk.
+constexpr int kGemv1Threads = 512;
 constexpr int kGemv1Warps = kGemv1Threads / 32;
 
 template <int C>
@@ -82,7 +85,8 @@ gemv1_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
              const float* __restrict__ codebook, int64_t O, int in, int nb, const uint16_t* __restrict__ x,
              void* __restrict__ Y, int out_bf16, int max_rows) {
   extern __shared__ __align__(16) uint8_t smem[];
-  constexpr int G = 32 / C;
+  constexpr int L2C = 2 * C;      // lanes per row
+  constexpr int G = 32 / L2C;     // rows per item
   constexpr int kDepth = 3;
   const int nch = (nb + C - 1) / C;
   const EngineLayout L = engine_layout(1, nb, max_rows, nch);
@@ -100,10 +104,11 @@ gemv1_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
   const int nvrows = static_cast<int>(std::min<int64_t>(g1 * G, O) - row0);
   const int ngr = (nvrows + G - 1) / G;
   const int nitems = ngr * nch;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane / C, s = lane % C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane / L2C, u = lane % L2C, s = u >> 1, hh = u & 1;
   const int it0 = warp * nitems / kGemv1Warps, it1 = (warp + 1) * nitems / kGemv1Warps;
 
-  uint4 cw[kDepth][5];
+  uint2 cw[kDepth][5];
   float sc[kDepth];
   bool ok[kDepth];
   auto fetch = [&](int it, int d) {
@@ -114,9 +119,9 @@ gemv1_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
     const int vrow = g * G + r, b = ch * C + s;
     if (vrow < nvrows && b < nb) {
       const int64_t F = (row0 + vrow) * nb + b;
-      const uint4* src = reinterpret_cast<const uint4*>(packed + F * kBlockBytes);
+      const uint2* src = reinterpret_cast<const uint2*>(packed + F * kBlockBytes + 40 * hh);
 #pragma unroll
-      for (int q = 0; q < 5; ++q) cw[d][q] = ldg_stream(src + q);
+      for (int q = 0; q < 5; ++q) cw[d][q] = __ldg(src + q);
       sc[d] = half_bits_to_float(__ldg(norms + F)) * (1.0f / 128.0f);
       ok[d] = true;
     }
@@ -124,41 +129,51 @@ gemv1_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 #pragma unroll
   for (int d = 0; d < kDepth; ++d) fetch(it0 + d, d);  // code loads in flight during the set-up below
 
-  build_pair_table(tab, c16, codebook);
-  rotate_tokens_bf16(x, in, in, nb, 1, 1, xs, xinv);
+  // Set-up, split over the warps: rotate x (four lanes per block) on some
+  // warps while the others replicate the pair table.
+  load_codebook16(c16, codebook);
+  __syncthreads();
+  const int nrot = min(kGemv1Warps / 2, (nb + 7) / 8);
+  rotate_row_q4(x, in, nb, xs, xinv, 0, nrot);
+  build_pair_table_warps(tab, c16, nrot, kGemv1Warps - nrot);
   __syncthreads();
 
-  const uint32_t* tab_lane = tab + lane;
-  uint32_t xr[64];
+  const uint32_t lane_base = static_cast<uint32_t>(__cvta_generic_to_shared(tab)) + 4u * lane;
+  uint32_t xr[32];
   float xi = 0.0f;
   int cur_ch = -1;
+  int ch_base = it0 / ngr, g_base = it0 - (it0 / ngr) * ngr;  // (chunk, group) of item `base`
   for (int base = it0; base < it1; base += kDepth) {
 #pragma unroll
     for (int d = 0; d < kDepth; ++d) {
       const int it = base + d;
+      int ch = ch_base, g = g_base + d;
+      if (g >= ngr) { g -= ngr; ++ch; }
+      if (g >= ngr) { g -= ngr; ++ch; }
       if (it < it1) {
-        const int ch = it / ngr, g = it - ch * ngr;
         const int b = ch * C + s;
         if (ch != cur_ch) {
           cur_ch = ch;
           if (b < nb) {
-            const uint4* xsrc = reinterpret_cast<const uint4*>(xs + b * kXsStride);
+            const uint4* xsrc = reinterpret_cast<const uint4*>(xs + b * kXsStride + 64 * hh);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const uint4 u = xsrc[q];
-              xr[4 * q] = u.x; xr[4 * q + 1] = u.y; xr[4 * q + 2] = u.z; xr[4 * q + 3] = u.w;
+            for (int q = 0; q < 8; ++q) {
+              const uint4 v = xsrc[q];
+              xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
             }
             xi = xinv[b];
           }
         }
-        float acc = ok[d] ? block_dot_reg(cw[d], tab_lane, xr) * (sc[d] * xi) : 0.0f;
+        float acc = ok[d] ? half_dot_reg(cw[d], lane_base, xr) * (sc[d] * xi) : 0.0f;
 #pragma unroll
-        for (int off = C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        for (int off = L2C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         const int vrow = g * G + r;
-        if (s == 0 && vrow < nvrows) slots[vrow * nch + ch] = acc;
+        if (u == 0 && vrow < nvrows) slots[vrow * nch + ch] = acc;
         fetch(it + kDepth, d);
       }
     }
+    g_base += kDepth;
+    while (g_base >= ngr) { g_base -= ngr; ++ch_base; }
   }
   __syncthreads();
   for (int v = threadIdx.x; v < nvrows; v += blockDim.x) {
@@ -174,7 +189,7 @@ template <int C>
 int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                    const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
-  constexpr int G = 32 / C;
+  constexpr int G = 32 / (2 * C);
   const int64_t ngroups = ceil_div(O, G);
   const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
   const int max_rows = static_cast<int>(ceil_div(ngroups, grid) * G);

@@ -79,7 +79,6 @@ size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char
 __global__ void __launch_bounds__(kRouterThreads, 1)
 router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, int E, int H, int T, int topk,
               int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
-  __shared__ float red[64];
   __shared__ int s_count[1025];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per_lane = (E + 31) / 32;

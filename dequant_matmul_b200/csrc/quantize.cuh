@@ -114,26 +114,40 @@ __device__ void build_quant_tables(const QuantShared& s, const float* __restrict
   __syncthreads();
 }
 
-// Butterfly stage over a lane's 32 values (pairs H apart).
+// Butterfly stage over a lane's 32 values (pairs H apart); for H >= 2 the
+// pairs (v[i], v[i+1]) are processed as packed f32x2.
 template <int H>
 __device__ __forceinline__ void stage32(float (&v)[32]) {
+  if constexpr (H == 1) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if ((i & H) == 0) {
-      const float a = v[i], b = v[i + H];
+    for (int i = 0; i < 32; i += 2) {
+      const float a = v[i], b = v[i + 1];
       v[i] = a + b;
-      v[i + H] = a - b;
+      v[i + 1] = a - b;
     }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2)
+      if ((i & H) == 0) {
+        const float2 a = make_float2(v[i], v[i + 1]), b = make_float2(v[i + H], v[i + H + 1]);
+        const float2 s = add2(a, b), d = sub2(a, b);
+        v[i] = s.x; v[i + 1] = s.y;
+        v[i + H] = d.x; v[i + H + 1] = d.y;
+      }
+  }
 }
 
 // Cross-lane butterfly stage: values 32*LM apart live in lanes LM apart.
 template <int LM>
 __device__ __forceinline__ void stage_x(float (&v)[32], int lane) {
-  const float sgn = (lane & LM) ? -1.0f : 1.0f;
+  const float sg = (lane & LM) ? -1.0f : 1.0f;
+  const float2 sgn = make_float2(sg, sg);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float p = __shfl_xor_sync(0xffffffffu, v[i], LM);
-    v[i] = fmaf(v[i], sgn, p);  // lower lane: v + p; upper lane: p - v
+  for (int i = 0; i < 32; i += 2) {
+    const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, v[i], LM), __shfl_xor_sync(0xffffffffu, v[i + 1], LM));
+    const float2 r = fma2(make_float2(v[i], v[i + 1]), sgn, p);  // lower lane: v + p; upper lane: p - v
+    v[i] = r.x;
+    v[i + 1] = r.y;
   }
 }
 
@@ -181,6 +195,12 @@ __device__ __forceinline__ void load_quarter(const void* __restrict__ base, int 
       v[e] = f;
     }
   }
+}
+
+__device__ __forceinline__ uint32_t lds_u32_q(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 template <bool kBf16>
@@ -237,7 +257,7 @@ quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const 
   constexpr int kEsz = kBf16 ? 2 : 4;
 
   const int lane = threadIdx.x & 31, q = lane & 3;
-  const uint32_t* tab_lane = s.tab + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(__cvta_generic_to_shared(s.tab)) + 4u * lane;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQThreads + threadIdx.x) >> 5;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kQThreads / 32);
   const int64_t nblocks = rows * nb;
@@ -258,15 +278,15 @@ quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const 
     float v[32];
     load_quarter<kBf16, kVec>(wblk + 32 * q * kEsz, qlen, v);
 
-    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    float2 s01 = make_float2(0.0f, 0.0f), s23 = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-      a0 = fmaf(v[e], v[e], a0);
-      a1 = fmaf(v[e + 1], v[e + 1], a1);
-      a2 = fmaf(v[e + 2], v[e + 2], a2);
-      a3 = fmaf(v[e + 3], v[e + 3], a3);
+      const float2 x01 = make_float2(v[e], v[e + 1]), x23 = make_float2(v[e + 2], v[e + 3]);
+      s01 = fma2(x01, x01, s01);
+      s23 = fma2(x23, x23, s23);
     }
-    float ssum = quad_sum((a0 + a1) + (a2 + a3));
+    float ssum = quad_sum((s01.x + s01.y) + (s23.x + s23.y));
+    float a0;
 
     bool zero_block = false, norm_exact = false;
     if (!(ssum >= 0x1p-100f && ssum <= 0x1p100f)) {
@@ -311,17 +331,26 @@ quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const 
 #pragma unroll
       for (int w = 0; w < 5; ++w) p[w] = code15_word(w);
     } else {
+      const float2 inv2 = make_float2(inv, inv), sig2 = make_float2(sigma, sigma);
+      const float2 k64 = make_float2(64.0f, 64.0f), mag2 = make_float2(kQMagic, kQMagic);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float ys = fminf(fmaxf(fmaf(v[e], inv, sigma), -3.0f), 3.0f);
-        const uint32_t idx = __float_as_uint(fmaf(ys, 64.0f, kQMagic)) & 511u;
-        const uint32_t ent = tab_lane[idx << 5];
-        const float thr = __uint_as_float(ent);
-        const uint32_t code = (ent & 31u) + (ys > thr ? 1u : 0u);
-        if (!(fabsf(ys - thr) >= kQGuard)) fm |= 1u << e;
-        const int bit = 5 * e, w = bit >> 5, sh = bit & 31;
-        p[w] |= code << sh;
-        if (sh > 27) p[w + 1] |= code >> (32 - sh);
+      for (int e2 = 0; e2 < 32; e2 += 2) {
+        const float2 y2 = fma2(make_float2(v[e2], v[e2 + 1]), inv2, sig2);
+        const float2 c2 = make_float2(fminf(fmaxf(y2.x, -3.0f), 3.0f), fminf(fmaxf(y2.y, -3.0f), 3.0f));
+        const float2 t2 = fma2(c2, k64, mag2);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = e2 + h;
+          const float ys = h ? c2.y : c2.x;
+          const uint32_t idx = __float_as_uint(h ? t2.y : t2.x) & 511u;
+          const uint32_t ent = lds_u32_q(idx * 128u + lane_base);
+          const float thr = __uint_as_float(ent);
+          const uint32_t code = (ent & 31u) + (ys > thr ? 1u : 0u);
+          if (!(fabsf(ys - thr) >= kQGuard)) fm |= 1u << e;
+          const int bit = 5 * e, w = bit >> 5, sh = bit & 31;
+          p[w] |= code << sh;
+          if (sh > 27) p[w + 1] |= code >> (32 - sh);
+        }
       }
     }
 

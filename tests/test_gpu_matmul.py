@@ -4,6 +4,7 @@ import pytest
 import torch
 
 import oracle as O
+import oracle as O_
 from dequant_matmul_b200 import synth
 from gpu_helpers import MATMUL_REL, oracle_to_dev, rel_l2
 
@@ -114,3 +115,35 @@ def test_gemv_full_27648x5120_sampled_rows(hl, cb):
     want = O.matmul(q["packed"], q["norms"], 5120, X)
     assert rel_l2(Y1.cpu().numpy()[rows], want[0]) <= MATMUL_REL
     assert rel_l2(Y4.double().cpu().numpy()[:, rows], want) <= MATMUL_REL
+
+
+@pytest.mark.parametrize("O,I,M", [(200, 704, 16), (384, 1024, 17), (256, 5120, 256), (130, 256, 48),
+                                   (1024, 5120, 200), (128, 128, 300)])
+def test_gemm_tensor_core_shapes(hl, cb, O, I, M):
+    """M >= 16 runs on the tcgen05 path: partial 128-row tile, ragged K (704 =
+    5.5 blocks), M not a multiple of 16, M = 256, and M > 256 (two token tiles)."""
+    W, q = _layer((O, I), seed=O + I + M)
+    p, n = oracle_to_dev(q)
+    X = synth.activations(M, I, seed=M + 1)
+    for odt in (torch.bfloat16, torch.float32):
+        Y = hl.gemm(p, n, cb, X.cuda(), out_dtype=odt)
+        torch.cuda.synchronize()
+        want = O_.matmul(q["packed"], q["norms"], I, X)
+        assert rel_l2(Y.double().cpu().numpy(), want) <= MATMUL_REL, odt
+    assert hl.device_error() == 0
+
+
+def test_gemm_full_27648x5120_m64_m256_sampled(hl, cb):
+    """The 27648 x 5120 layer at M = 64 and 256 (tensor-core path), rows sampled
+    for the oracle."""
+    W = synth.student_t((27648, 5120), df4_seed=0)
+    p, n = hl.quantize(W.cuda(), cb)
+    rows = np.sort(np.random.default_rng(1).choice(27648, 256, replace=False))
+    q = O_.quantize(W[rows])
+    for M in (64, 256):
+        X = synth.activations(M, 5120, seed=20 + M)
+        Y = hl.gemm(p, n, cb, X.cuda(), out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        want = O_.matmul(q["packed"], q["norms"], 5120, X)
+        assert rel_l2(Y.double().cpu().numpy()[:, rows], want) <= MATMUL_REL, M
+    assert hl.device_error() == 0
