@@ -21,7 +21,8 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return [os.path.join(PKG, "csrc", "libhlwq.cu"), os.path.join(PKG, "csrc", "codebook.cpp")]
+    return [os.path.join(PKG, "csrc", "libhlwq.cu"), os.path.join(PKG, "csrc", "noalloc.cu"),
+            os.path.join(PKG, "csrc", "codebook.cpp")]
 
 
 def needs_build() -> bool:

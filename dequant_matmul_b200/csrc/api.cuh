@@ -152,6 +152,7 @@ extern "C" const char* hlwq_status_string(int status) {
     case HLWQ_EUNSUPPORTED: return "unsupported size or dtype";
     case HLWQ_ECUDA: return "CUDA runtime error";
     case HLWQ_EWORKSPACE: return "workspace missing or too small";
+    case HLWQ_ESCRATCH: return "request exceeds the static scratch of hlwq_gemm_noalloc";
     default: return "unknown status";
   }
 }

@@ -17,6 +17,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhlwq.so")
 
 HLWQ_OK, HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_ECUDA, HLWQ_EWORKSPACE = 0, -1, -2, -3, -4, -5
+HLWQ_ESCRATCH = -6
+NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 + 64 * 1024
 HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
 HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
 BLOCK, BLOCK_BYTES, LEVELS = 128, 80, 32
@@ -31,6 +33,7 @@ SIGNATURES = {
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "hlwq_moe_gemv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _I,
                            _P, _P, _P, _SZ, _P]),
+    "hlwq_gemm_noalloc": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P]),
     "hlwq_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I64, _I64]),
     "hlwq_device_error": (_I, [_P]),
     "hlwq_status_string": (ctypes.c_char_p, [_I]),
@@ -198,3 +201,15 @@ def moe_gemv(gu, dn, cb, logits, X, topk: int, shared=None, out_dtype=torch.floa
                              _dtype_code(Y.dtype), _ptr(ids), _ptr(weights), _ptr(workspace), workspace.numel(),
                              _stream(stream)), "hlwq_moe_gemv")
     return Y, ids, weights
+
+
+def gemm_noalloc(packed, norms, cb, X: torch.Tensor, out_dtype=torch.bfloat16, Y=None, stream=None):
+    """hlwq_gemm_noalloc: the GEMM with the library's static scratch (no workspace)."""
+    _cuda(X, "X")
+    out_f = packed.shape[0]
+    M, in_f = X.shape
+    if Y is None:
+        Y = torch.empty(M, out_f, dtype=out_dtype, device=X.device)
+    _check(lib.hlwq_gemm_noalloc(_ptr(packed), _ptr(norms), _ptr(cb), out_f, in_f, M, _ptr(X), X.stride(0),
+                                 _ptr(Y), Y.stride(0), _dtype_code(Y.dtype), _stream(stream)), "hlwq_gemm_noalloc")
+    return Y

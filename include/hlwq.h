@@ -30,8 +30,9 @@
  *     device; "stream" is a cudaStream_t passed as void* (NULL = the legacy
  *     default stream).  Device calls are asynchronous on that stream; errors
  *     detected on the host are returned before anything is launched.
- *   - The library allocates no memory.  Calls that need scratch take a
- *     caller-provided device workspace sized by hlwq_workspace_bytes().
+ *   - The library allocates no memory at run time.  Calls that need scratch take a
+ *     caller-provided device workspace sized by hlwq_workspace_bytes(), except
+ *     hlwq_gemm_noalloc, which uses a static device array of the library.
  *   - Alignment: packed, W, W_out, X, Y and workspace must be 16-byte aligned
  *     (torch allocations are); leading dimensions are in elements.
  *   - Return value: HLWQ_OK (0) or a negative hlwq_status.
@@ -55,7 +56,8 @@ typedef enum {
   HLWQ_EALIGN = -2,       /* a pointer or leading dimension breaks the alignment rule */
   HLWQ_EUNSUPPORTED = -3, /* a size or dtype combination this build does not handle */
   HLWQ_ECUDA = -4,        /* a CUDA runtime call (launch, attribute) failed */
-  HLWQ_EWORKSPACE = -5    /* workspace is NULL or smaller than hlwq_workspace_bytes() */
+  HLWQ_EWORKSPACE = -5,   /* workspace is NULL or smaller than hlwq_workspace_bytes() */
+  HLWQ_ESCRATCH = -6      /* request needs more than the static scratch of hlwq_gemm_noalloc */
 } hlwq_status;
 
 typedef enum { HLWQ_F32 = 0, HLWQ_BF16 = 1, HLWQ_F16 = 2 } hlwq_dtype;
@@ -155,6 +157,31 @@ int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
  *   HLWQ_OP_MOE : a = H,   b = F,  c = T, E = experts, topk
  */
 size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk);
+
+/* Bytes of library-owned static device memory that hlwq_gemm_noalloc uses as
+ * scratch (held by every GPU that loads the library until process exit). */
+#define HLWQ_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u + 64u * 1024u)
+
+/*
+ * hlwq_gemm without a workspace argument, for callers that cannot allocate
+ * device memory (for example code that runs where allocation is forbidden, or
+ * a plug-in whose host owns every allocation).  No counterpart in the paper:
+ * it is the same computation as hlwq_gemm, taking its scratch from a static
+ * device array of HLWQ_NOALLOC_SCRATCH_BYTES instead of a caller workspace.
+ *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ *   - Requests needing more than HLWQ_NOALLOC_SCRATCH_BYTES of scratch
+ *     (hlwq_workspace_bytes(HLWQ_OP_GEMM, ...)) return HLWQ_ESCRATCH; for the
+ *     tensor-core path that is about M * ceil(in / 128) * 256 bytes.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array: calls whose executions overlap on
+ *     the GPU (other streams, other threads) race on it.
+ * Arguments, layouts and the other errors are those of hlwq_gemm.
+ */
+int hlwq_gemm_noalloc(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+                      int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx,
+                      void* Y, int64_t ldy, int ydtype, void* stream);
 
 /* Reads (after synchronising the current device) and clears the device error word. */
 int hlwq_device_error(uint32_t* bits);

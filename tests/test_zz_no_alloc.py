@@ -1,0 +1,44 @@
+"""hlwq_gemm_noalloc: the GEMM entry point for callers that cannot allocate
+device memory (its scratch is a static device array owned by the library).
+
+Collected last on purpose: it must pass both in a fresh process and after every
+other test has run on the same device."""
+import ctypes
+
+import pytest
+import torch
+
+from dequant_matmul_b200 import synth
+from gpu_helpers import MATMUL_REL, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hl():
+    from dequant_matmul_b200 import hlwq
+    return hlwq
+
+
+def test_noalloc_matches_gemm_on_consecutive_calls(hl):
+    cb = hl.codebook("cuda")
+    W = synth.student_t((1024, 5120), df4_seed=77).cuda()
+    p, n = hl.quantize(W, cb)
+    # two calls in a row with different inputs: the shared scratch keeps the
+    # first call's contents, which must not leak into the second result
+    for M, seed in ((64, 1), (200, 2), (5, 3)):
+        X = synth.activations(M, 5120, seed=seed).cuda()
+        got = hl.gemm_noalloc(p, n, cb, X, out_dtype=torch.float32)
+        want = hl.gemm(p, n, cb, X, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert rel_l2(got.double().cpu().numpy(), want.double().cpu().numpy()) <= MATMUL_REL, M
+    assert hl.device_error() == 0
+
+
+def test_noalloc_rejects_requests_beyond_the_scratch(hl):
+    need = hl.workspace_bytes(hl.HLWQ_OP_GEMM, 128, 65536, 64)
+    assert need > hl.NOALLOC_SCRATCH_BYTES
+    p = ctypes.c_void_p(256)
+    st = hl.lib.hlwq_gemm_noalloc(p, p, p, 128, 65536, 64, p, 65536, p, 128, hl.HLWQ_F32, None)
+    assert st == hl.HLWQ_ESCRATCH
+    assert hl.lib.hlwq_status_string(st).decode().startswith("request exceeds")
