@@ -12,17 +12,19 @@
 //
 // Kernel 1 (rotate_x_kernel): one CTA per token rotates X once per call into
 // the workspace (binary16 B matrix, K-major) and records 1/s_m.
-// Kernel 2 (gemm_tc_kernel): one CTA per 128-row tile of W (and 256-token tile
-// of X).  Roles, 320 threads:
-//   warps 0-7  decode: each lane owns one weight row of the tile and decodes 32
-//              codes of each 64-wide K chunk (code pair -> binary16 centroid
-//              pair from a lane-replicated table, times the block scale) and
-//              writes them straight into tensor memory with tcgen05.st (the A
+// Kernel 2 (gemm_tc_kernel): one CTA per 128-row tile of W (and up to 256-token
+// tile of X).  Roles, 864 threads:
+//   warps 0-23 decode, in G groups of 8 (G = 3, or 2 for 256-token tiles)
+//              taking blocks b = g (mod G): each lane owns one weight row of
+//              the tile and decodes one half block (code -> fp32 centroid from
+//              a shared table, times the block scale, rounded to binary16) and
+//              writes it straight into tensor memory with tcgen05.st (the A
 //              operand lives in TMEM, so decoding costs no shared-memory
 //              bandwidth that the MMA needs for B);
-//   warp 8     TMA producer: 64 x N tiles of B, 128-byte swizzled, into a
-//              3-4 stage shared-memory ring (no multicast);
-//   warp 9     allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
+//   warp 24    TMA producer of the code tiles (128 rows x 80 bytes per block);
+//   warp 26    TMA producer of B: two 64 x N boxes per block, 128-byte swizzled
+//              (no multicast);
+//   warp 25    allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
 //              N = tokens, K = 16) into an fp32 accumulator in TMEM;
 //   warps 0-3  epilogue: tcgen05.ld of the accumulator, scaling, bf16/fp32 store.
 // Stages are handed over with mbarriers; every wait is bounded (2 s), after
@@ -37,11 +39,14 @@ namespace hlwq {
 
 namespace {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcGroups = 3;                       // decode groups (8 warps each) on alternate blocks
+constexpr int kTcDecWarps = 8 * kTcGroups;
+constexpr int kTcWCodes = kTcDecWarps, kTcWMma = kTcDecWarps + 1, kTcWB = kTcDecWarps + 2;
+constexpr int kTcThreads = 32 * (kTcDecWarps + 3);
 constexpr int kTcTileRows = 128;
 constexpr int kTcKChunk = 64;                 // K elements per pipeline stage (one half block)
 constexpr int kTcAccCols = 256;               // TMEM columns reserved for the accumulator
-constexpr int kTcAllocCols = 512;
+constexpr int kTcAllocCols = 512;   // accumulator (256) + 3 A stages of 64
 constexpr uint64_t kTcTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -64,7 +69,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 // Bounded wait for the phase of `parity` to complete; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline) {
-  for (;;) {
+  for (uint32_t n = 1;; ++n) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -74,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
         : "r"(bar), "r"(parity)
         : "memory");
     if (ok) return true;
-    if (globaltimer_ns() > deadline) return false;
+    if ((n & 63u) == 0u && globaltimer_ns() > deadline) return false;
   }
 }
 
@@ -143,6 +148,38 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n) {
          (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
+// Shared address of the fp32 centroid of the code at bit POS of a half block
+// (10 words): the 5-bit field moved to bit 2 with one shift and masked.
+// (pos is a compile-time constant after unrolling.)
+__device__ __forceinline__ uint32_t code_addr(const uint2 (&cw)[5], int pos, uint32_t tab) {
+  const int wi = pos >> 5, sh = pos & 31;
+  const uint32_t lo = word10(cw, wi);
+  uint32_t t;
+  if (sh > 27) {
+    t = __funnelshift_r(lo, word10(cw, wi + 1), sh - 2);
+  } else if (sh >= 2) {
+    t = lo >> (sh - 2);
+  } else {
+    t = lo << (2 - sh);
+  }
+  return (t & 0x7cu) + tab;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 r;
+  asm("{ .reg .b64 pa, pb, pd; mov.b64 pa, {%2, %3}; mov.b64 pb, {%4, %5};\n\t"
+      "mul.rn.f32x2 pd, pa, pb; mov.b64 {%0, %1}, pd; }"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// (lo, hi) -> binary16 pair, round to nearest even.
+__device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 // ---------------------------------------------------------------- rotation
 constexpr int kRotThreads = 256;
 
@@ -195,74 +232,96 @@ rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, uin
 }
 
 // ---------------------------------------------------------------- main kernel
-struct TcSmem {
-  uint32_t tab;     // pair table (128 KiB)
-  uint32_t bstage;  // B stages, each n_box * 128 bytes
-  uint32_t bars;    // full_a[S], full_b[S], empty[S], accum, 8 bytes each
-  uint32_t misc;    // tmem base (4 B), abort flag (4 B), c16 (64 B)
-};
+// Rings: codes (one 128-row x 80-byte block column per stage, TMA) and A/B
+// stages (one 128-wide K block: A decoded into 64 TMEM columns, B as two
+// 64-wide TMA boxes with 128-byte swizzle); see tc_groups for the mapping.
+constexpr int kTcCodeBytes = kTcTileRows * kBlockBytes;  // 10240
+constexpr int kTcAS = 4;   // A stages in TMEM (64 columns each) after the 256-column accumulator
 
-__host__ __device__ inline int tc_stages(int n_box) { return n_box > 128 ? 3 : 4; }
+constexpr int kTcSmemMax = 227 * 1024;
+constexpr int kTcSmemFixed = 1024 /*align slack*/ + 1024 /*centroid table, barriers, misc*/;
+static_assert(4 * kLevels + 8 * (2 * kTcGroups + 4 * kTcGroups + 1) + 8 <= 1024, "barrier block overflows");
+constexpr int kTcMaxNb = 64;  // tile norms in shared memory: 128 x nb binary16 (in <= 8192)
 
-__host__ __device__ inline int tc_smem_bytes(int n_box) {
-  return 1024 /*align slack*/ + kPairTabBytes + tc_stages(n_box) * n_box * 128 + 256 + 128;
+// Decode groups: G groups of 8 warps take blocks b = g (mod G).  Every ring
+// stage belongs to exactly one group, so each stage is consumed in order by a
+// single consumer and mbarrier parity waits are never ambiguous:
+//   A/B stage of block b   = b mod G               (one per group; A in TMEM, B in smem)
+//   code stage of block b  = 2 (b mod G) + (b / G) mod 2   (two per group)
+__host__ __device__ inline int tc_groups(int n_box) { return n_box > 128 ? 2 : kTcGroups; }
+__host__ __device__ inline int tc_cstages(int n_box) { return 2 * tc_groups(n_box); }
+__host__ __device__ inline int tc_stages(int n_box, int) { return tc_groups(n_box); }
+
+__host__ __device__ inline int tc_norm_bytes(int nb) { return (kTcTileRows * nb * 2 + 15) & ~15; }
+
+__host__ __device__ inline int tc_smem_bytes(int n_box, int nb) {
+  return kTcSmemFixed + tc_stages(n_box, nb) * n_box * 256 + tc_cstages(n_box) * kTcCodeBytes + tc_norm_bytes(nb);
 }
 
+__host__ __device__ inline int tc_ab_stage(int b, int G) { return b % G; }
+__host__ __device__ inline uint32_t tc_ab_parity(int b, int G) { return static_cast<uint32_t>(b / G) & 1u; }
+__host__ __device__ inline int tc_code_stage(int b, int G) { return 2 * (b % G) + ((b / G) & 1); }
+__host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static_cast<uint32_t>(b / G / 2) & 1u; }
+
 __global__ void __launch_bounds__(kTcThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restrict__ packed,
+gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
                const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
                const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const int S = tc_stages(n_box);
-  const uint32_t tab = base;
-  const uint32_t bst = base + kPairTabBytes;
-  const uint32_t bars = bst + S * n_box * 128;
-  const uint32_t misc = bars + 8 * (3 * S + 1);
-  uint32_t* tab_g = reinterpret_cast<uint32_t*>(gbase);
+  const int G = tc_groups(n_box), S = tc_stages(n_box, nb), CS = tc_cstages(n_box);
+  const uint32_t tab = base;                 // 32 fp32 centroids
+  const uint32_t bst = base + 1024;
+  const uint32_t cst = bst + S * n_box * 256;
+  const uint32_t nst = cst + CS * kTcCodeBytes;          // tile norms [128][nb] (binary16)
+  const uint32_t bars = base + 4 * kLevels;              // after the table, inside the first 1 KiB
+  // barrier block: full[S] empty[S] c_full[CS] c_empty[CS] accum, then misc
+  // (TMEM base, abort flag): at most 128 + 8 (2 S + 2 CS + 1) + 8 = 288 bytes
+  const uint32_t full0 = bars, empty0 = full0 + 8 * S, c_full0 = empty0 + 8 * S, c_empty0 = c_full0 + 8 * CS,
+                 accum = c_empty0 + 8 * CS;
+  const uint32_t misc = accum + 8;
   volatile uint32_t* misc_g = reinterpret_cast<volatile uint32_t*>(gbase + (misc - base));
-  uint16_t* c16 = reinterpret_cast<uint16_t*>(gbase + (misc - base) + 16);
-  auto full_a = [&](int s) { return bars + 8u * s; };
-  auto full_b = [&](int s) { return bars + 8u * (S + s); };
-  auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
-  const uint32_t accum = bars + 8u * (3 * S);
+  float* c32 = reinterpret_cast<float*>(gbase);
+  const uint8_t* codes_g = gbase + (cst - base);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t o0 = static_cast<int64_t>(blockIdx.x) * kTcTileRows;
   const int n0 = blockIdx.y * n_box;
-  const int nchunks = 2 * nb;
   const uint64_t deadline = globaltimer_ns() + kTcTimeoutNs;
 
-  // ---- set-up: codebook, barriers, TMEM, pair table
+  // ---- set-up: codebook, barriers, TMEM
   if (threadIdx.x < kLevels) {
     const float c = __ldg(codebook + threadIdx.x);
-    c16[threadIdx.x] = __half_as_ushort(__float2half_rn(c));
+    c32[threadIdx.x] = c;
     if (threadIdx.x + 1 < kLevels && !(c < __ldg(codebook + threadIdx.x + 1))) raise_device_error(HLWQ_DEVERR_CODEBOOK);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_a(s), 8);
-      mbar_init(full_b(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(full0 + 8 * s, 9);   // 8 decode warps + the B producer (plus its TMA bytes)
+      mbar_init(empty0 + 8 * s, 1);  // the MMA commit
+    }
+    for (int s = 0; s < CS; ++s) {
+      mbar_init(c_full0 + 8 * s, 1);
+      mbar_init(c_empty0 + 8 * s, 8);
     }
     mbar_init(accum, 1);
     misc_g[1] = 0u;  // abort flag
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == kTcWMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(misc), "r"(kTcAllocCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   __syncthreads();
-  if (warp < 8) {
-    uint4* t4 = reinterpret_cast<uint4*>(tab_g);
-    for (int q = threadIdx.x; q < 1024 * 8; q += 256) {
-      const int v = q >> 3;
-      const uint32_t e = static_cast<uint32_t>(c16[v & 31]) | (static_cast<uint32_t>(c16[v >> 5]) << 16);
-      t4[q] = make_uint4(e, e, e, e);
+  uint16_t* nrm_s = reinterpret_cast<uint16_t*>(gbase + (nst - base));
+  if (warp < kTcDecWarps) {
+    // the tile's norms, row-major [128][nb], coalesced
+    for (int q = threadIdx.x; q < kTcTileRows * nb; q += 32 * kTcDecWarps) {
+      const int rr = q / nb;
+      nrm_s[q] = (o0 + rr < O) ? __ldg(norms + (o0 + rr) * nb + (q - rr * nb)) : static_cast<uint16_t>(0);
     }
   }
   tc_fence_before();
@@ -270,69 +329,54 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restri
   tc_fence_after();
   const uint32_t tmem = misc_g[0];
 
-  if (warp < 8) {
+  if (warp < kTcDecWarps) {
     // ---------------------------------------------------------- decode
-    const int q4 = warp & 3, hh = warp >> 2;
+    // two groups of 8 warps take alternate blocks; in a group, warp (q4, hh)
+    // decodes half block hh of rows 32 q4 + lane
+    const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod kTcGroups
     const int r = 32 * q4 + lane;
     const int64_t o = o0 + r;
     const bool row_ok = o < O;
-    // per-row power of two so that n * 2^-e <= 1
+    const uint16_t* rown = nrm_s + r * nb;
     float nmax = 0.0f;
-    if (row_ok)
-      for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, half_bits_to_float(__ldg(norms + o * nb + b)));
+    for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, half_bits_to_float(rown[b]));
     int erow = 0;
     if (nmax > 0.0f && isfinite(nmax)) frexpf(nmax, &erow);
     const float rs = ldexpf(1.0f, -erow);
-    const uint32_t lane_base = tab + 4u * lane;
     const uint32_t tm_row = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-    const uint8_t* rowp = packed + (row_ok ? o : 0) * static_cast<int64_t>(nb) * kBlockBytes + 20 * hh;
-    const uint16_t* rown = norms + (row_ok ? o : 0) * static_cast<int64_t>(nb);
-
-    constexpr int kD = 4;
-    uint32_t cw[kD][5];
-    float nsc[kD];
-    auto fetch = [&](int i, int d) {
-      if (i < nchunks && row_ok) {
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(rowp + (i >> 1) * kBlockBytes + 40 * (i & 1));
-#pragma unroll
-        for (int k = 0; k < 5; ++k) cw[d][k] = __ldg(src + k);
-        nsc[d] = half_bits_to_float(__ldg(rown + (i >> 1))) * rs;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 5; ++k) cw[d][k] = 0u;
-        nsc[d] = 0.0f;
-      }
-    };
-#pragma unroll
-    for (int d = 0; d < kD; ++d) fetch(d, d);
     bool ok = true;
-    for (int i0 = 0; i0 < nchunks; i0 += kD) {
+    for (int b = dg; b < nb && dg < G; b += G) {
+      const int cs = tc_code_stage(b, G), as = tc_ab_stage(b, G);
+      const float nsc = half_bits_to_float(rown[b]) * rs;
+      uint2 cw[5];
+      if (ok) ok = mbar_wait(c_full0 + 8 * cs, tc_code_parity(b, G), deadline);
+      const uint2* src = reinterpret_cast<const uint2*>(codes_g + cs * kTcCodeBytes + r * kBlockBytes + 40 * hh);
 #pragma unroll
-      for (int d = 0; d < kD; ++d) {
-        const int i = i0 + d;
-        if (i < nchunks) {
-          const int s = i % S;
-          const uint32_t h2 = pack_half2(nsc[d], nsc[d]);
-          uint32_t v[16];
+      for (int k = 0; k < 5; ++k) cw[k] = src[k];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
+      const float2 sc2 = make_float2(nsc, nsc);
+      uint32_t v[32];
 #pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const int bit = 10 * p, wi = bit >> 5, sh = bit & 31;
-            const uint32_t lo = cw[d][wi];
-            const uint32_t hi = (wi + 1 < 5) ? cw[d][wi + 1] : 0u;
-            const uint32_t v10 = (sh <= 22) ? ((lo >> sh) & 0x3ffu) : (__funnelshift_r(lo, hi, sh) & 0x3ffu);
-            v[p] = hmul2(lds_u32(lane_base + (v10 << 7)), h2);
-          }
-          fetch(i + kD, d);
-          if (ok) ok = mbar_wait(empty(s), ((i / S) & 1) ^ 1, deadline);
-          if (ok && misc_g[1] == 0u) {
-            tc_st16(tm_row + kTcAccCols + 32 * s + 16 * hh, v);
-            tc_wait_st();
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(full_a(s));
-        }
+      for (int p = 0; p < 32; ++p) {
+        const float2 c = make_float2(__uint_as_float(lds_u32(code_addr(cw, 10 * p, tab))),
+                                     __uint_as_float(lds_u32(code_addr(cw, 10 * p + 5, tab))));
+        const float2 a = fmul2(c, sc2);
+        v[p] = cvt_half2(a.x, a.y);
       }
+      if (ok) ok = mbar_wait(empty0 + 8 * as, tc_ab_parity(b, G) ^ 1u, deadline);
+      if (ok && misc_g[1] == 0u) {
+        const uint32_t ta = tm_row + kTcAccCols + 64 * as + 32 * hh;
+        uint32_t v0[16], v1[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) { v0[k] = v[k]; v1[k] = v[16 + k]; }
+        tc_st16(ta, v0);
+        tc_st16(ta + 16, v1);
+        tc_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * as);
     }
     if (!ok) {
       misc_g[1] = 1u;
@@ -367,38 +411,61 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restri
         }
       }
     }
-  } else if (warp == 8) {
-    // ---------------------------------------------------------- TMA producer
+  } else if (warp == kTcWCodes) {
+    // ---------------------------------------------------------- TMA producer: code tiles
     if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(n_box) * 128u;
-      for (int i = 0; i < nchunks; ++i) {
-        const int s = i % S;
-        if (!mbar_wait(empty(s), ((i / S) & 1) ^ 1, deadline) || misc_g[1] != 0u) {
-          misc_g[1] = 1u;
-          raise_device_error(HLWQ_DEVERR_TIMEOUT);
-          break;
-        }
-        mbar_arrive_expect_tx(full_b(s), bytes);
-        tma_load_2d(bst + s * n_box * 128, &bmap, kTcKChunk * i, n0, full_b(s));
+      bool ok = true;
+      for (int b = 0; b < nb; ++b) {
+        const int cs = tc_code_stage(b, G);
+        ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b, G) ^ 1u, deadline) && misc_g[1] == 0u;
+        if (!ok) break;
+        mbar_arrive_expect_tx(c_full0 + 8 * cs, kTcCodeBytes);
+        tma_load_2d(cst + cs * kTcCodeBytes, &cmap, kBlockBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
+      }
+      if (!ok) {
+        misc_g[1] = 1u;
+        raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
     }
-  } else {
-    // ---------------------------------------------------------- MMA issuer (warp 9)
+  } else if (warp == kTcWB) {
+    // ---------------------------------------------------------- TMA producer: B tiles
+    if (lane == 0) {
+      const uint32_t half_bytes = static_cast<uint32_t>(n_box) * 128u;
+      bool ok = true;
+      for (int b = 0; b < nb; ++b) {
+        const int st = tc_ab_stage(b, G);
+        ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b, G) ^ 1u, deadline) && misc_g[1] == 0u;
+        if (!ok) break;
+        mbar_arrive_expect_tx(full0 + 8 * st, 2 * half_bytes);
+        const uint32_t dst = bst + st * n_box * 256;
+        tma_load_2d(dst, &bmap, kTcKChunk * (2 * b), n0, full0 + 8 * st);
+        tma_load_2d(dst + half_bytes, &bmap, kTcKChunk * (2 * b + 1), n0, full0 + 8 * st);
+      }
+      if (!ok) {
+        misc_g[1] = 1u;
+        raise_device_error(HLWQ_DEVERR_TIMEOUT);
+      }
+    }
+  } else if (warp == kTcWMma) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(n_box);
       bool ok = true;
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const int s = i % S;
-        const uint32_t par = (i / S) & 1;
-        ok = mbar_wait(full_a(s), par, deadline) && mbar_wait(full_b(s), par, deadline) && misc_g[1] == 0u;
+      for (int b = 0; b < nb; ++b) {
+        const int st = tc_ab_stage(b, G);
+        ok = mbar_wait(full0 + 8 * st, tc_ab_parity(b, G), deadline) && misc_g[1] == 0u;
         if (!ok) break;
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_sw128(bst + s * n_box * 128);
+        const uint32_t bstage = bst + st * n_box * 256;
 #pragma unroll
-        for (int kk = 0; kk < kTcKChunk / 16; ++kk)
-          tc_mma_f16(tmem, tmem + kTcAccCols + 32 * s + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(empty(s));
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t bdesc = smem_desc_sw128(bstage + h * n_box * 128);
+#pragma unroll
+          for (int kk = 0; kk < kTcKChunk / 16; ++kk)
+            tc_mma_f16(tmem, tmem + kTcAccCols + 64 * st + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk),
+                       idesc, (b > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8 * st);  // frees both the A stage (TMEM) and the B stage (shared memory)
       }
       if (!ok) {
         misc_g[1] = 1u;
@@ -410,7 +477,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restri
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kTcWMma) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcAllocCols) : "memory");
   }
@@ -437,10 +504,15 @@ size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
   return ((b_bytes + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(M) * 4 + 256;
 }
 
+int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                 const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
+
 int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                    const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
                    size_t ws_bytes, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
+  // Rows longer than kTcMaxNb blocks do not fit the tile-norm staging: CUDA-core path.
+  if (nb > kTcMaxNb) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
   if (ws_bytes < gemm_tc_workspace_bytes(O, in, M)) return HLWQ_EWORKSPACE;
   uint16_t* B = static_cast<uint16_t*>(workspace);
   const size_t b_bytes = static_cast<size_t>(M) * nb * kBlock * 2;
@@ -456,7 +528,8 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
   rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
 
-  const int n_box = static_cast<int>(std::min<int64_t>(256, (std::min<int64_t>(M, 256) + 15) / 16 * 16));
+  int n_box = static_cast<int>(std::min<int64_t>(256, (std::min<int64_t>(M, 256) + 15) / 16 * 16));
+  while (n_box > 16 && tc_smem_bytes(n_box, nb) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
   CUtensorMap map;
@@ -468,16 +541,25 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
-  const int smem = tc_smem_bytes(n_box);
+  // Codes viewed as a 2-D byte tensor [O][NB * 80]; one box = 128 rows x one 80-byte block.
+  CUtensorMap cmap;
+  const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(nb) * kBlockBytes, static_cast<cuuint64_t>(O)};
+  const cuuint64_t cstride[1] = {static_cast<cuuint64_t>(nb) * kBlockBytes};
+  const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(kTcTileRows)};
+  if (encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), cdim, cstride, cbox, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return HLWQ_ECUDA;
+  const int smem = tc_smem_bytes(n_box, nb);
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return HLWQ_ECUDA;
     attr = true;
   }
-  if (smem > 227 * 1024) return HLWQ_EUNSUPPORTED;
+  if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   dim3 grid(static_cast<unsigned>(ceil_div(O, kTcTileRows)), static_cast<unsigned>(ceil_div(M, n_box)));
-  gemm_tc_kernel<<<grid, kTcThreads, smem, stream>>>(map, packed, norms, codebook, O, nb, M, inv_s, Y, ldy,
+  gemm_tc_kernel<<<grid, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y, ldy,
                                                      out_bf16 ? 1 : 0, n_box);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }

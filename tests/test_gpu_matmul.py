@@ -147,3 +147,16 @@ def test_gemm_full_27648x5120_m64_m256_sampled(hl, cb):
         want = O_.matmul(q["packed"], q["norms"], 5120, X)
         assert rel_l2(Y.double().cpu().numpy()[:, rows], want) <= MATMUL_REL, M
     assert hl.device_error() == 0
+
+
+def test_gemm_long_rows_m256(hl, cb):
+    """in = 8192 at M = 256 (token tile narrowed to fit shared memory) and
+    in = 8320 (longer than the tile-norm staging: CUDA-core path)."""
+    for I in (8192, 8320):
+        W, q = _layer((256, I), seed=I)
+        p, n = oracle_to_dev(q)
+        X = synth.activations(256 if I == 8192 else 20, I, seed=I + 1)
+        Y = hl.gemm(p, n, cb, X.cuda(), out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        want = O_.matmul(q["packed"], q["norms"], I, X)
+        assert rel_l2(Y.double().cpu().numpy(), want) <= MATMUL_REL, I
