@@ -367,9 +367,11 @@ def main():
         ys = torch.empty(LAYERS, O_DIM, dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
 
+    flags = hl.HLWQ_FLAG_WEIGHTS_STATIC   # weights are static across the decode pass
+
     def step():
         for l, (p, n) in enumerate(layers):
-            hl.gemv(p, n, cb, xs[l], y=ys[l], stream=stream)
+            hl.gemv(p, n, cb, xs[l], y=ys[l], stream=stream, flags=flags)
 
     for _ in range(warmup):
         step()
@@ -413,7 +415,7 @@ def main():
     def e2e_step():
         xs.copy_(x_host, non_blocking=True)
         for l, (p, n) in enumerate(layers):
-            hl.gemv(p, n, cb, xs[l], y=ys[l], stream=stream)
+            hl.gemv(p, n, cb, xs[l], y=ys[l], stream=stream, flags=flags)
         y_host.copy_(ys, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -448,6 +450,8 @@ def main():
             "config": {"workload": "dense decode GEMV 5120x5120 HLWQ-Q5 (bf16 Student-t(4) std 0.02 weights, "
                                    "x bf16 N(0,1)), M=1, 64 distinct layers per step",
                        "global_batch": 1, "bytes_per_step_per_gpu": LAYERS * WEIGHT_BYTES,
+                       "launch": "hlwq_gemv_ex(HLWQ_FLAG_WEIGHTS_STATIC): programmatic dependent launch, "
+                                 "x read after the previous kernel completes",
                        "l2": "inputs larger than L2 (64 layers x 16.8 MB = 1.07 GB)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -75,6 +75,18 @@ extern "C" int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const flo
                             ydtype == HLWQ_BF16, as_stream(stream));
 }
 
+extern "C" int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
+                            int64_t in, const uint16_t* x, void* y, int ydtype, unsigned flags, void* stream) {
+  if (flags & ~static_cast<unsigned>(HLWQ_FLAG_WEIGHTS_STATIC)) return HLWQ_EINVAL;
+  if (!packed || !norms || !codebook || !x || !y || out <= 0 || in <= 0 || in > kMaxIn) return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || !aligned2(norms) || !aligned2(x) || !aligned2(y) ||
+      (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(y) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_gemv1(packed, norms, codebook, out, static_cast<int>(in), x, y, ydtype == HLWQ_BF16,
+                            as_stream(stream), flags);
+}
+
 extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
                          int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy, int ydtype,
                          void* workspace, size_t ws_bytes, void* stream) {

@@ -15,8 +15,11 @@
 // deterministic.
 
 #include <algorithm>
+#include <mutex>
+#include <utility>
 
 #include "engine.cuh"
+#include "sm100.cuh"
 
 namespace hlwq {
 
@@ -69,153 +72,421 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 }
 
 
-// Single-token GEMV.  512 threads (16 warps) per CTA, one CTA per SM (the
-// 128 KiB pair table).  A lane owns half a 128-block (64 codes, 40 bytes): lane
-// (r, s, h) takes row r, block s of the chunk and half h, so the 2C lanes of a
-// row read 80 C contiguous bytes.  A CTA's items are ordered chunk-major and
-// each warp takes a contiguous range of them, so a lane's 64 rotated
-// activation values (32 half2 registers) are reloaded only when the range
-// crosses into the next chunk.
-constexpr int kGemv1Threads = 512;
-constexpr int kGemv1Warps = kGemv1Threads / 32;
+// Single-token GEMV.  One CTA of 512 threads per SM (the 128 KiB lane-
+// replicated pair table).  An item is G = 16 / C rows x one chunk of C blocks
+// (always 16 blocks, 1280 bytes of codes); lane (r, s, h) = (lane / 2C,
+// (lane % 2C) / 2, lane % 2) takes row r, block s of the chunk and half h of
+// that block (64 codes, 40 bytes).  A CTA owns a contiguous range of rows; its
+// items are ordered chunk-major and split into 16 contiguous warp ranges, so a
+// lane reloads its 64 rotated activations (32 half2 registers) only when its
+// range crosses into the next chunk.
+//
+// Codes are streamed by TMA: every warp owns a ring of S item slots in shared
+// memory (one 3-D box {80 bytes, C blocks, G rows} per item, one mbarrier per
+// slot) and keeps S items in flight; lane 0 refills a slot as soon as the warp
+// has read it.  Norms travel in a register ring beside it.
+//
+// Per pair of codes: one shift that puts the 10-bit pair index at bit 7, one
+// and-or that forms the byte offset of (entry, lane) in the table, one shared
+// load and one half2 FMA.  The four fp16 chains of a lane (8 products each:
+// at most 8 x 3.27 x 2^10, far below 65504) are widened once per item, scaled
+// by n16 / 128 and the block's activation scale and summed over the row's 2C
+// lanes; the row sums over chunks are formed at the end in a fixed order
+// (deterministic).
+//
+// Launched with programmatic stream serialisation (HLWQ_FLAG_WEIGHTS_STATIC),
+// the set-up -- first code boxes, codebook, pair table -- runs before
+// griddepcontrol.wait, i.e. while the previous kernel on the stream is still
+// finishing; x is read and y written only after it.
+constexpr int kG1Threads = 512;
+constexpr int kG1Warps = kG1Threads / 32;
+constexpr int kG1ItemBytes = 16 * kBlockBytes;  // G rows x C blocks = 16 blocks for every C
 
-template <int C>
-__global__ void __launch_bounds__(kGemv1Threads, 1)
-gemv1_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
+struct G1Layout {
+  int ring_off, xs_off, xinv_off, part_off, c16_off, bar_off, total;
+};
+
+__host__ __device__ inline int round16(int v) { return (v + 15) & ~15; }
+
+__host__ __device__ inline G1Layout g1_layout(int nb, int pass_rows, int nch, int S) {
+  G1Layout L;
+  L.ring_off = kPairTabBytes;  // the table sits at offset 0
+  L.xs_off = L.ring_off + kG1Warps * S * kG1ItemBytes;
+  L.xinv_off = L.xs_off + round16(nb * kXsStride * 2);
+  L.part_off = L.xinv_off + round16(nb * 4);
+  L.c16_off = L.part_off + round16(pass_rows * nch * 4);
+  L.bar_off = L.c16_off + 64;
+  L.total = L.bar_off + kG1Warps * S * 8;
+  return L;
+}
+
+// Byte offset of pair P's table entry for this lane: the 10-bit field at bit
+// 10 P of the half block's 10 words, moved to bit 7, or-ed with lane * 4.
+template <int P>
+__device__ __forceinline__ uint32_t g1_off(const uint2 (&cw)[5], uint32_t lane4) {
+  constexpr int bit = 10 * P, wi = bit >> 5, sh = bit & 31;
+  const uint32_t lo = word10(cw, wi);
+  uint32_t t;
+  if constexpr (sh > 22) {
+    t = __funnelshift_r(lo, word10(cw, wi + 1), sh - 7);
+  } else if constexpr (sh >= 7) {
+    t = lo >> (sh - 7);
+  } else {
+    t = lo << (7 - sh);
+  }
+  return (t & 0x1ff80u) | lane4;
+}
+
+// Pair P goes to fp16 chain P % 4 (four independent chains of 8 products).
+template <int P>
+__device__ __forceinline__ void g1_pair(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
+                                        const uint32_t (&xr)[32], uint32_t (&h)[4]) {
+  const uint32_t e = *reinterpret_cast<const uint32_t*>(tab + g1_off<P>(cw, lane4));
+  if constexpr (P < 4) h[P] = hmul2(e, xr[P]);
+  else h[P & 3] = hfma2(e, xr[P], h[P & 3]);
+}
+
+template <int... P>
+__device__ __forceinline__ float g1_dot(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
+                                        const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
+  uint32_t h[4];
+  (g1_pair<P>(tab, cw, lane4, xr, h), ...);
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h[0]));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h[1]));
+  const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&h[2]));
+  const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&h[3]));
+  return ((f0.x + f1.x) + (f2.x + f3.x)) + ((f0.y + f1.y) + (f2.y + f3.y));
+}
+
+// Rotation of x with eight lanes per 128-block (16 consecutive values per
+// lane: four butterfly stages in registers, three across lanes), all warps.
+// Block b is scaled by 2^k so that max |x_tilde| * 2^k lies in [2^9, 2^10)
+// and stored as binary16; xinv[b] = 2^-k.
+__device__ __forceinline__ void g1_rotate(const uint16_t* __restrict__ x, int in, int nb, bool xvec, uint16_t* xs,
+                                          float* xinv) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane & 7;
+  for (int b0 = 4 * warp; b0 < nb; b0 += 4 * kG1Warps) {
+    const int b = b0 + (lane >> 3);
+    const bool act = b < nb;
+    const int i0 = kBlock * b + 16 * q;
+    float v[16];
+    if (xvec) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (act && i0 + 8 * j < in) w = __ldg(reinterpret_cast<const uint4*>(x + i0 + 8 * j));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[8 * j + 2 * k] = __uint_as_float(ww[k] << 16);
+          v[8 * j + 2 * k + 1] = __uint_as_float(ww[k] & 0xffff0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = (act && i0 + e < in) ? bf16_bits_to_float(__ldg(x + i0 + e)) : 0.0f;
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if ((e & h) == 0) {
+          const float a = v[e], c = v[e + h];
+          v[e] = a + c;
+          v[e + h] = a - c;
+        }
+    }
+#pragma unroll
+    for (int lm = 1; lm < 8; lm <<= 1) {
+      const float sgn = (lane & lm) ? -1.0f : 1.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = fmaf(v[e], sgn, __shfl_xor_sync(0xffffffffu, v[e], lm));
+    }
+    float mx = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
+#pragma unroll
+    for (int lm = 1; lm < 8; lm <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lm));
+    int ex = 0;
+    if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
+    const int k = max(-120, min(120, 10 - ex));
+    const float sc = ldexpf(1.0f, k);
+    if (act) {
+      uint4* dst = reinterpret_cast<uint4*>(xs + b * kXsStride + 16 * q);
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        dst[c] = make_uint4(pack_half2(v[8 * c] * sc, v[8 * c + 1] * sc), pack_half2(v[8 * c + 2] * sc, v[8 * c + 3] * sc),
+                            pack_half2(v[8 * c + 4] * sc, v[8 * c + 5] * sc),
+                            pack_half2(v[8 * c + 6] * sc, v[8 * c + 7] * sc));
+      if (q == 0) xinv[b] = ldexpf(1.0f, -k);
+    }
+  }
+}
+
+template <int C, int S>
+__global__ void __launch_bounds__(kG1Threads, 1)
+gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restrict__ norms,
              const float* __restrict__ codebook, int64_t O, int in, int nb, const uint16_t* __restrict__ x,
-             void* __restrict__ Y, int out_bf16, int max_rows) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  constexpr int L2C = 2 * C;      // lanes per row
-  constexpr int G = 32 / L2C;     // rows per item
-  constexpr int kDepth = 3;
+             void* __restrict__ Y, int out_bf16, int pass_rows, int xvec) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int L2C = 2 * C;   // lanes per row
+  constexpr int G = 32 / L2C;  // rows per item
   const int nch = (nb + C - 1) / C;
-  const EngineLayout L = engine_layout(1, nb, max_rows, nch);
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  const G1Layout L = g1_layout(nb, pass_rows, nch, S);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
   float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
-  float* slots = reinterpret_cast<float*>(smem + L.slot_off);
-  float* misc = reinterpret_cast<float*>(smem + L.misc_off);
-  uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
+  float* part = reinterpret_cast<float*>(smem + L.part_off);
+  uint16_t* c16 = reinterpret_cast<uint16_t*>(smem + L.c16_off);
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
 
   const int64_t ngroups = (O + G - 1) / G;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * ngroups / gridDim.x;
   const int64_t g1 = static_cast<int64_t>(blockIdx.x + 1) * ngroups / gridDim.x;
   const int64_t row0 = g0 * G;
-  const int nvrows = static_cast<int>(std::min<int64_t>(g1 * G, O) - row0);
-  const int ngr = (nvrows + G - 1) / G;
-  const int nitems = ngr * nch;
+  const int nrows = static_cast<int>(std::min<int64_t>(g1 * G, O) - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane / L2C, u = lane % L2C, s = u >> 1, hh = u & 1;
-  const int it0 = warp * nitems / kGemv1Warps, it1 = (warp + 1) * nitems / kGemv1Warps;
+  const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
 
-  uint2 cw[kDepth][5];
-  float sc[kDepth];
-  bool ok[kDepth];
-  auto fetch = [&](int it, int d) {
-    ok[d] = false;
-    sc[d] = 0.0f;
-    if (it >= it1) return;
-    const int ch = it / ngr, g = it - ch * ngr;
-    const int vrow = g * G + r, b = ch * C + s;
-    if (vrow < nvrows && b < nb) {
-      const int64_t F = (row0 + vrow) * nb + b;
-      const uint2* src = reinterpret_cast<const uint2*>(packed + F * kBlockBytes + 40 * hh);
+  // this warp's ring: S slots of one item each, one mbarrier per slot
+  const uint32_t ring = sbase + L.ring_off + warp * (S * kG1ItemBytes);
+  const uint32_t bar = sbase + L.bar_off + warp * (S * 8);
+  const uint8_t* my_codes = smem + L.ring_off + warp * (S * kG1ItemBytes) + 40 * lane;  // slot layout [G][C][80]
+  if (lane == 0) {
 #pragma unroll
-      for (int q = 0; q < 5; ++q) cw[d][q] = __ldg(src + q);
-      sc[d] = half_bits_to_float(__ldg(norms + F)) * (1.0f / 128.0f);
-      ok[d] = true;
+    for (int d = 0; d < S; ++d) mbar_init(bar + 8 * d, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
+  bool ok = true;
+  uint32_t phase = 0;    // parity of the next completion, one bit per slot
+  uint32_t pending = 0;  // slots with a box in flight
+
+  for (int p0 = 0; p0 < nrows; p0 += pass_rows) {
+    const int prow = min(pass_rows, nrows - p0);
+    const int ngr = (prow + G - 1) / G;
+    const int nitems = ngr * nch;
+    const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
+    const int nw = it1 - it0;
+
+    // issue cursor: item (ich, ig) goes to the slot being refilled
+    int ich = it0 / ngr, ig = it0 - (it0 / ngr) * ngr;
+    uint32_t nraw[S];
+    auto issue = [&](int d) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
+        tma_load_3d(ring + d * kG1ItemBytes, &cmap, 0, ich * C, static_cast<int>(row0 + p0 + ig * G), bar + 8 * d);
+      }
+      const int v = ig * G + r, b = ich * C + s;
+      nraw[d] = (v < prow && b < nb) ? static_cast<uint32_t>(__ldg(norms + (row0 + p0 + v) * nb + b)) : 0u;
+      pending |= 1u << d;
+      if (++ig == ngr) { ig = 0; ++ich; }
+    };
+#pragma unroll
+    for (int d = 0; d < S; ++d)
+      if (d < nw) issue(d);
+
+    if (p0 == 0) {
+      // set-up while the first boxes are in flight
+      load_codebook16(c16, codebook);
+      __syncthreads();
+      build_pair_table_warps(reinterpret_cast<uint32_t*>(smem), c16, 0, kG1Warps);
+      pdl_wait();  // x may be produced by the previous kernel on the stream
+      g1_rotate(x, in, nb, xvec != 0, xs, xinv);
+      __syncthreads();
+      pdl_trigger();
     }
-  };
-#pragma unroll
-  for (int d = 0; d < kDepth; ++d) fetch(it0 + d, d);  // code loads in flight during the set-up below
 
-  // Set-up, split over the warps: rotate x (four lanes per block) on some
-  // warps while the others replicate the pair table.
-  load_codebook16(c16, codebook);
-  __syncthreads();
-  const int nrot = min(kGemv1Warps / 2, (nb + 7) / 8);
-  rotate_row_q4(x, in, nb, xs, xinv, 0, nrot);
-  build_pair_table_warps(tab, c16, nrot, kGemv1Warps - nrot);
-  __syncthreads();
-
-  const uint32_t lane_base = static_cast<uint32_t>(__cvta_generic_to_shared(tab)) + 4u * lane;
-  uint32_t xr[32];
-  float xi = 0.0f;
-  int cur_ch = -1;
-  int ch_base = it0 / ngr, g_base = it0 - (it0 / ngr) * ngr;  // (chunk, group) of item `base`
-  for (int base = it0; base < it1; base += kDepth) {
+    int cch = it0 / ngr, cg = it0 - (it0 / ngr) * ngr, xch = -1;
+    uint32_t xr[32];
+    float xi = 0.0f;
+    for (int base = 0; base < nw; base += S) {
 #pragma unroll
-    for (int d = 0; d < kDepth; ++d) {
-      const int it = base + d;
-      int ch = ch_base, g = g_base + d;
-      if (g >= ngr) { g -= ngr; ++ch; }
-      if (g >= ngr) { g -= ngr; ++ch; }
-      if (it < it1) {
-        const int b = ch * C + s;
-        if (ch != cur_ch) {
-          cur_ch = ch;
-          if (b < nb) {
-            const uint4* xsrc = reinterpret_cast<const uint4*>(xs + b * kXsStride + 64 * hh);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint4 v = xsrc[q];
-              xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
+      for (int d = 0; d < S; ++d) {
+        const int k = base + d;
+        if (k < nw) {
+          const uint32_t nr = nraw[d];
+          if (ok && ((pending >> d) & 1u)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
+            if (ok) {
+              phase ^= 1u << d;
+              pending &= ~(1u << d);
             }
-            xi = xinv[b];
           }
-        }
-        float acc = ok[d] ? half_dot_reg(cw[d], lane_base, xr) * (sc[d] * xi) : 0.0f;
+          uint2 cw[5];
+          const uint2* src = reinterpret_cast<const uint2*>(my_codes + d * kG1ItemBytes);
 #pragma unroll
-        for (int off = L2C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        const int vrow = g * G + r;
-        if (u == 0 && vrow < nvrows) slots[vrow * nch + ch] = acc;
-        fetch(it + kDepth, d);
+          for (int q = 0; q < 5; ++q) cw[q] = src[q];
+          __syncwarp();
+          if (ok && k + S < nw) {
+            if (lane == 0) fence_proxy_async();  // the slot's reads precede the refill
+            issue(d);
+          }
+          if (cch != xch) {
+            xch = cch;
+            const int b = cch * C + s;
+            if (b < nb) {
+              const uint4* xsrc = reinterpret_cast<const uint4*>(xs + b * kXsStride + 64 * hh);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint4 w = xsrc[q];
+                xr[4 * q] = w.x; xr[4 * q + 1] = w.y; xr[4 * q + 2] = w.z; xr[4 * q + 3] = w.w;
+              }
+              xi = xinv[b] * (1.0f / 128.0f);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 32; ++q) xr[q] = 0u;
+              xi = 0.0f;
+            }
+          }
+          float acc = g1_dot(smem, cw, lane4, xr, std::make_integer_sequence<int, 32>{});
+          acc *= half_bits_to_float(static_cast<uint16_t>(nr)) * xi;
+#pragma unroll
+          for (int off = L2C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+          const int v = cg * G + r;
+          if (u == 0 && v < prow) part[v * nch + cch] = acc;
+          if (++cg == ngr) { cg = 0; ++cch; }
+        }
       }
     }
-    g_base += kDepth;
-    while (g_base >= ngr) { g_base -= ngr; ++ch_base; }
-  }
-  __syncthreads();
-  for (int v = threadIdx.x; v < nvrows; v += blockDim.x) {
-    const float* sl = slots + v * nch;
-    float sum = 0.0f;
-    for (int ch = 0; ch < nch; ++ch) sum += sl[ch];
-    if (out_bf16) static_cast<uint16_t*>(Y)[row0 + v] = static_cast<uint16_t>(float_to_bf16_bits(sum));
-    else static_cast<float*>(Y)[row0 + v] = sum;
+    if (!ok) {
+      // a box never arrived: drain what is still in flight (bounded), then stop
+      const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
+      for (int d = 0; d < S; ++d)
+        if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
+      if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < prow; v += kG1Threads) {
+      const float* pr = part + v * nch;
+      float sum = 0.0f;
+      for (int ch = 0; ch < nch; ++ch) sum += pr[ch];
+      const int64_t o = row0 + p0 + v;
+      if (out_bf16) static_cast<uint16_t*>(Y)[o] = static_cast<uint16_t>(float_to_bf16_bits(sum));
+      else static_cast<float*>(Y)[o] = sum;
+    }
+    __syncthreads();
+    if (__syncthreads_or(!ok)) break;
   }
 }
 
-template <int C>
-int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
-                   const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream) {
-  const int nb = static_cast<int>(ceil_div(in, kBlock));
-  constexpr int G = 32 / (2 * C);
-  const int64_t ngroups = ceil_div(O, G);
-  const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
-  const int max_rows = static_cast<int>(ceil_div(ngroups, grid) * G);
-  const EngineLayout L = engine_layout(1, nb, max_rows, (nb + C - 1) / C);
-  if (L.total > 227 * 1024) return HLWQ_EUNSUPPORTED;
+// Tensor map of the codes viewed as a 3-D byte tensor {80, NB, O}; one box is
+// one item {80, C, G}.  Encoding costs host time, so the last few maps are
+// kept (a map depends only on the pointer and the shape).
+struct CodesMapEntry {
+  const void* ptr;
+  int64_t O;
+  int nb, C;
+  CUtensorMap map;
+};
+
+inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, CUtensorMap* out) {
+  static std::mutex mu;
+  static CodesMapEntry cache[8];
+  static int used = 0, next = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int k = 0; k < used; ++k) {
+    const CodesMapEntry& e = cache[k];
+    if (e.ptr == packed && e.O == O && e.nb == nb && e.C == C) {
+      *out = e.map;
+      return HLWQ_OK;
+    }
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+  if (!encode) return HLWQ_ECUDA;
+  const int G = 16 / C;
+  const cuuint64_t dim[3] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb),
+                             static_cast<cuuint64_t>(O)};
+  const cuuint64_t stride[2] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb) * kBlockBytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(C),
+                             static_cast<cuuint32_t>(G)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap m;
+  if (encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dim, stride, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return HLWQ_ECUDA;
+  CodesMapEntry& e = cache[next];
+  e.ptr = packed;
+  e.O = O;
+  e.nb = nb;
+  e.C = C;
+  e.map = m;
+  next = (next + 1) % 8;
+  used = std::min(used + 1, 8);
+  *out = m;
+  return HLWQ_OK;
+}
+
+// Rows of a CTA handled per pass for ring depth S (0 if the layout does not fit).
+inline int g1_pass_rows(int nb, int C, int S, int rows_cta) {
+  const int G = 16 / C, nch = (nb + C - 1) / C;
+  const int fixed = g1_layout(nb, 0, nch, S).total;
+  const int cap = (227 * 1024 - fixed - 16) / (nch * 4) / G * G;
+  return cap < G ? 0 : std::min(rows_cta, cap);
+}
+
+template <int C, int S>
+int launch_gemv1_cs(const CUtensorMap& map, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                    int nb, const uint16_t* x, void* Y, bool out_bf16, unsigned flags, int grid, int pass_rows,
+                    cudaStream_t stream) {
+  const G1Layout L = g1_layout(nb, pass_rows, (nb + C - 1) / C, S);
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(gemv1_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+    if (cudaFuncSetAttribute(gemv1_kernel<C, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
         cudaSuccess)
       return HLWQ_ECUDA;
     attr_set = true;
   }
-  gemv1_kernel<C><<<grid, kGemv1Threads, L.total, stream>>>(packed, norms, codebook, O, in, nb, x, Y,
-                                                           out_bf16 ? 1 : 0, max_rows);
-  return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+  const int xvec = (reinterpret_cast<uintptr_t>(x) % 16 == 0 && in % 8 == 0) ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kG1Threads);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & HLWQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
+  const int ob = out_bf16 ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, gemv1_kernel<C, S>, map, norms, codebook, O, in, nb, x, Y, ob, pass_rows, xvec) !=
+      cudaSuccess)
+    return HLWQ_ECUDA;
+  return HLWQ_OK;
+}
+
+template <int C>
+int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                   const uint16_t* x, void* Y, bool out_bf16, unsigned flags, cudaStream_t stream) {
+  const int nb = static_cast<int>(ceil_div(in, kBlock));
+  constexpr int G = 16 / C;
+  const int64_t ngroups = ceil_div(O, G);
+  const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
+  const int rows_cta = static_cast<int>(ceil_div(ngroups, grid) * G);
+  CUtensorMap map;
+  const int st = codes_map(packed, O, nb, C, &map);
+  if (st != HLWQ_OK) return st;
+  // deepest ring that fits beside the table and the rotated activation
+  if (const int pr = g1_pass_rows(nb, C, 4, rows_cta))
+    return launch_gemv1_cs<C, 4>(map, norms, codebook, O, in, nb, x, Y, out_bf16, flags, grid, pr, stream);
+  if (const int pr = g1_pass_rows(nb, C, 2, rows_cta))
+    return launch_gemv1_cs<C, 2>(map, norms, codebook, O, in, nb, x, Y, out_bf16, flags, grid, pr, stream);
+  if (const int pr = g1_pass_rows(nb, C, 1, rows_cta))
+    return launch_gemv1_cs<C, 1>(map, norms, codebook, O, in, nb, x, Y, out_bf16, flags, grid, pr, stream);
+  return HLWQ_EUNSUPPORTED;
 }
 
 }  // namespace
 
 int launch_gemv1(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
-                 const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream) {
+                 const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream, unsigned flags) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
   switch (pick_chunk(nb)) {
-    case 8: return launch_gemv1_c<8>(packed, norms, codebook, O, in, x, Y, out_bf16, stream);
-    case 4: return launch_gemv1_c<4>(packed, norms, codebook, O, in, x, Y, out_bf16, stream);
-    default: return launch_gemv1_c<2>(packed, norms, codebook, O, in, x, Y, out_bf16, stream);
+    case 8: return launch_gemv1_c<8>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
+    case 4: return launch_gemv1_c<4>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
+    default: return launch_gemv1_c<2>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
   }
 }
 
@@ -271,7 +542,7 @@ int dense_smem_bytes(int64_t O, int in, int mt) {
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
-  if (M == 1) return launch_gemv1(packed, norms, codebook, O, in, X, Y, out_bf16, stream);
+  if (M == 1) return launch_gemv1(packed, norms, codebook, O, in, X, Y, out_bf16, stream, 0u);
   int mt = M >= 3 ? 4 : M;
   while (mt > 1 && dense_smem_bytes(O, in, mt) > 227 * 1024) mt >>= 1;
   switch (pick_chunk(nb)) {

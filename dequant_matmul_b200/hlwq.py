@@ -21,6 +21,7 @@ HLWQ_ESCRATCH = -6
 NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 + 64 * 1024
 HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
 HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
+HLWQ_FLAG_WEIGHTS_STATIC = 1
 BLOCK, BLOCK_BYTES, LEVELS = 128, 80, 32
 
 # (name, restype, argtypes) for every symbol include/hlwq.h declares.
@@ -30,6 +31,7 @@ SIGNATURES = {
     "hlwq_quantize": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
     "hlwq_gemv": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
+    "hlwq_gemv_ex": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, ctypes.c_uint, _P]),
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "hlwq_moe_gemv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _I,
                            _P, _P, _P, _SZ, _P]),
@@ -148,14 +150,20 @@ def dequantize(packed, norms, cb, in_features: int, out_dtype=torch.float32, out
     return out
 
 
-def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None):
-    """x: bf16 [in].  Returns y [out]."""
+def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None, flags: int = 0):
+    """x: bf16 [in].  Returns y [out].  flags != 0 calls hlwq_gemv_ex (e.g.
+    HLWQ_FLAG_WEIGHTS_STATIC: the weights are not written by earlier work still
+    running on the stream, so the kernel's set-up may overlap it)."""
     _cuda(x, "x")
     out_f = packed.shape[0]
     if y is None:
         y = torch.empty(out_f, dtype=out_dtype, device=x.device)
-    _check(lib.hlwq_gemv(_ptr(packed), _ptr(norms), _ptr(cb), out_f, x.shape[-1], _ptr(x), _ptr(y),
-                         _dtype_code(y.dtype), _stream(stream)), "hlwq_gemv")
+    if flags:
+        _check(lib.hlwq_gemv_ex(_ptr(packed), _ptr(norms), _ptr(cb), out_f, x.shape[-1], _ptr(x), _ptr(y),
+                                _dtype_code(y.dtype), flags, _stream(stream)), "hlwq_gemv_ex")
+    else:
+        _check(lib.hlwq_gemv(_ptr(packed), _ptr(norms), _ptr(cb), out_f, x.shape[-1], _ptr(x), _ptr(y),
+                             _dtype_code(y.dtype), _stream(stream)), "hlwq_gemv")
     return y
 
 

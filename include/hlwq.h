@@ -65,6 +65,9 @@ typedef enum { HLWQ_F32 = 0, HLWQ_BF16 = 1, HLWQ_F16 = 2 } hlwq_dtype;
 /* Operations whose scratch size hlwq_workspace_bytes() reports. */
 typedef enum { HLWQ_OP_GEMM = 1, HLWQ_OP_MOE = 2 } hlwq_op;
 
+/* Launch flags of the *_ex calls. */
+typedef enum { HLWQ_FLAG_WEIGHTS_STATIC = 1 } hlwq_flags;
+
 /* Device error bits (hlwq_device_error). */
 #define HLWQ_DEVERR_CODEBOOK 0x1u  /* codebook not strictly ascending or not finite */
 #define HLWQ_DEVERR_TIMEOUT  0x2u  /* a bounded in-kernel wait gave up */
@@ -116,6 +119,21 @@ int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, const float* c
  */
 int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook,
               int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype, void* stream);
+
+/*
+ * hlwq_gemv with launch flags (bitwise or of hlwq_flags; 0 = hlwq_gemv).
+ *   HLWQ_FLAG_WEIGHTS_STATIC: the caller guarantees that packed, norms and
+ *     codebook are not written by any work enqueued earlier on `stream` that
+ *     may still be running (true of the weights of a decode loop).  The kernel
+ *     is then launched with programmatic stream serialisation: its set-up
+ *     (first code loads, codebook, decode table) may run while the previous
+ *     kernel on the stream is finishing; x is read and y written only after
+ *     that kernel has completed and its writes are visible.
+ * Errors: as hlwq_gemv; unknown flag bits -> HLWQ_EINVAL.
+ */
+int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+                 int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype,
+                 unsigned flags, void* stream);
 
 /*
  * Small-M GEMM: Y[m][o] = sum_i X[m][i] * w_hat[o][i], fp32 accumulation.

@@ -64,6 +64,64 @@ def test_gemv_activation_scale_extremes(hl, cb):
         assert rel_l2(y.cpu().numpy(), want) <= MATMUL_REL, s
 
 
+def test_gemv_ex_weights_static_chain(hl, cb):
+    """hlwq_gemv_ex with HLWQ_FLAG_WEIGHTS_STATIC on a chain of square layers in
+    which every GEMV reads the bf16 output of the kernel before it (the decode
+    pattern; each launch's set-up overlaps the previous kernel), with a torch
+    kernel producing the input of every other layer.  Bit-identical to plain
+    launches, and each layer matches the oracle on the input it was given."""
+    D = 2048
+    layers = [_layer((D, D), seed=40 + l) for l in range(4)]
+    devs = [oracle_to_dev(q) for _, q in layers]
+    x0 = synth.activations(1, D, seed=41)[0].cuda()
+    outs = {}
+    for flags in (0, hl.HLWQ_FLAG_WEIGHTS_STATIC):
+        x, ins, ys = x0.clone(), [], []
+        for l, (p, n) in enumerate(devs):
+            if l % 2:
+                x = (x.float() * 1.0).to(torch.bfloat16)   # a torch kernel writes this layer's input
+            ins.append(x)
+            x = hl.gemv(p, n, cb, x, out_dtype=torch.bfloat16, flags=flags)
+            ys.append(x)
+        torch.cuda.synchronize()
+        outs[flags] = (ins, ys)
+    for a, b in zip(outs[0][1], outs[hl.HLWQ_FLAG_WEIGHTS_STATIC][1]):
+        assert torch.equal(a, b)
+    for (W, q), xin, y in zip(layers, *outs[hl.HLWQ_FLAG_WEIGHTS_STATIC]):
+        want = O.matmul(q["packed"], q["norms"], D, xin.cpu()[None])[0]
+        assert rel_l2(y.double().cpu().numpy(), want) <= MATMUL_REL
+
+
+def test_gemv_ex_rejects_unknown_flags(hl, cb):
+    W, q = _layer((64, 256), seed=3)
+    p, n = oracle_to_dev(q)
+    x = synth.activations(1, 256, seed=3)[0].cuda()
+    y = torch.empty(64, device="cuda")
+    st = hl.lib.hlwq_gemv_ex(p.data_ptr(), n.data_ptr(), cb.data_ptr(), 64, 256, x.data_ptr(), y.data_ptr(),
+                             hl.HLWQ_F32, 0x2, torch.cuda.current_stream().cuda_stream)
+    assert st == hl.HLWQ_EINVAL
+
+
+def test_gemv_long_rows_several_passes(hl, cb):
+    """in = 32768 (256 blocks): the rotated activation takes most of shared
+    memory, so the code ring is one slot deep and each CTA covers its ~160 rows
+    in several passes (rows sampled for the oracle, including the first and
+    last rows of the matrix and rows around pass boundaries)."""
+    Od, I = 11700, 32768
+    W = synth.student_t_device((Od, I), seed=12)
+    p, n = hl.quantize(W, cb)
+    x = synth.activations(1, I, seed=13)
+    y = hl.gemv(p, n, cb, x[0].cuda())
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.arange(0, 24), np.arange(70, 90), np.arange(150, 170),
+                                     np.arange(Od - 16, Od),
+                                     np.random.default_rng(1).choice(Od, 24, replace=False)]))
+    q = O.quantize(W[torch.as_tensor(rows, device=W.device)].cpu())
+    del W
+    want = O.matmul(q["packed"], q["norms"], I, x)[0]
+    assert rel_l2(y.cpu().numpy()[rows], want) <= MATMUL_REL
+
+
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 9, 15, 16, 17, 64])
 def test_gemm_small_m(hl, cb, M):
     W, q = _layer((1024, 5120), seed=21)
