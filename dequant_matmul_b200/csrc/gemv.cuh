@@ -73,25 +73,28 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 
 
 // Single-token GEMV.  One CTA of 512 threads per SM (the 128 KiB lane-
-// replicated pair table).  An item is G = 16 / C rows x one chunk of C blocks
-// (always 16 blocks, 1280 bytes of codes); lane (r, s, h) = (lane / 2C,
-// (lane % 2C) / 2, lane % 2) takes row r, block s of the chunk and half h of
-// that block (64 codes, 40 bytes).  A CTA owns a contiguous range of rows; its
-// items are ordered chunk-major and split into 16 contiguous warp ranges, so a
-// lane reloads its 64 rotated activations (32 half2 registers) only when its
+// replicated pair table).  An item is 2G rows (G = 16 / C) x one chunk of C
+// blocks (always 32 blocks, 2560 bytes of codes); lane (r, s, h) = (lane / 2C,
+// (lane % 2C) / 2, lane % 2) takes rows r and r + G, block s of the chunk and
+// half h of that block (2 x 64 codes), so the two rows share the lane's 64
+// rotated activations (32 half2 registers) and the per-item costs (wait,
+// refill, reduction) are paid once per 64 code pairs.  A CTA owns a contiguous
+// range of rows; its items are ordered chunk-major and split into 16
+// contiguous warp ranges, so a lane reloads its activations only when its
 // range crosses into the next chunk.
 //
 // Codes are streamed by TMA: every warp owns a ring of S item slots in shared
-// memory (one 3-D box {80 bytes, C blocks, G rows} per item, one mbarrier per
+// memory (one 3-D box {80 bytes, C blocks, 2G rows} per item, one mbarrier per
 // slot) and keeps S items in flight; lane 0 refills a slot as soon as the warp
 // has read it.  Norms travel in a register ring beside it.
 //
 // Per pair of codes: one shift that puts the 10-bit pair index at bit 7, one
 // and-or that forms the byte offset of (entry, lane) in the table, one shared
-// load and one half2 FMA.  The four fp16 chains of a lane (8 products each:
-// at most 8 x 3.27 x 2^10, far below 65504) are widened once per item, scaled
+// load and one half2 FMA.  The four fp16 chains of a lane (8 products each)
+// are added pairwise in fp16 and widened once per item, scaled
 // by n16 / 128 and the block's activation scale and summed over the row's 2C
-// lanes; the row sums over chunks are formed at the end in a fixed order
+// lanes (the two rows of a lane are reduced together: log2(2C) shuffles); the
+// row sums over chunks are formed at the end in a fixed order
 // (deterministic).
 //
 // Launched with programmatic stream serialisation (HLWQ_FLAG_WEIGHTS_STATIC),
@@ -100,7 +103,12 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 // finishing; x is read and y written only after it.
 constexpr int kG1Threads = 512;
 constexpr int kG1Warps = kG1Threads / 32;
-constexpr int kG1ItemBytes = 16 * kBlockBytes;  // G rows x C blocks = 16 blocks for every C
+constexpr int kG1ItemBytes = 32 * kBlockBytes;  // 2G rows x C blocks = 32 blocks for every C
+// Rotated activation: 256 bytes per block, its sixteen 16-byte chunks stored
+// at chunk (j ^ (b & 7)) so that the lanes of a row (blocks b, b + 1, ...)
+// reload their halves from different banks.
+constexpr int kG1XsBytes = 256;
+__host__ __device__ inline int g1_xs_chunk(int b, int j) { return b * 16 + (j ^ (b & 7)); }
 
 struct G1Layout {
   int ring_off, xs_off, xinv_off, part_off, c16_off, bar_off, total;
@@ -112,7 +120,7 @@ __host__ __device__ inline G1Layout g1_layout(int nb, int pass_rows, int nch, in
   G1Layout L;
   L.ring_off = kPairTabBytes;  // the table sits at offset 0
   L.xs_off = L.ring_off + kG1Warps * S * kG1ItemBytes;
-  L.xinv_off = L.xs_off + round16(nb * kXsStride * 2);
+  L.xinv_off = L.xs_off + nb * kG1XsBytes;
   L.part_off = L.xinv_off + round16(nb * 4);
   L.c16_off = L.part_off + round16(pass_rows * nch * 4);
   L.bar_off = L.c16_off + 64;
@@ -151,75 +159,84 @@ __device__ __forceinline__ float g1_dot(const uint8_t* tab, const uint2 (&cw)[5]
                                         const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
   uint32_t h[4];
   (g1_pair<P>(tab, cw, lane4, xr, h), ...);
-  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h[0]));
-  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h[1]));
-  const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&h[2]));
-  const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&h[3]));
-  return ((f0.x + f1.x) + (f2.x + f3.x)) + ((f0.y + f1.y) + (f2.y + f3.y));
+  // two chains at a time are added in fp16 (16 products: the codes of a block
+  // have sum c^2 ~ 128, so |sum| <= sqrt(135) * 4 * 2^10 < 65504), then widened
+  const uint32_t h01 = hadd2(h[0], h[1]), h23 = hadd2(h[2], h[3]);
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+  return (f0.x + f1.x) + (f0.y + f1.y);
 }
 
 // Rotation of x with eight lanes per 128-block (16 consecutive values per
-// lane: four butterfly stages in registers, three across lanes), all warps.
-// Block b is scaled by 2^k so that max |x_tilde| * 2^k lies in [2^9, 2^10)
-// and stored as binary16; xinv[b] = 2^-k.
-__device__ __forceinline__ void g1_rotate(const uint16_t* __restrict__ x, int in, int nb, bool xvec, uint16_t* xs,
-                                          float* xinv) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane & 7;
-  for (int b0 = 4 * warp; b0 < nb; b0 += 4 * kG1Warps) {
-    const int b = b0 + (lane >> 3);
-    const bool act = b < nb;
-    const int i0 = kBlock * b + 16 * q;
-    float v[16];
-    if (xvec) {
+// lane: four butterfly stages in registers, three across lanes); a warp covers
+// blocks b0 .. b0 + 3.  Block b is scaled by 2^k so that max |x_tilde| * 2^k
+// lies in [2^9, 2^10) and stored as binary16; xinv[b] = 2^-k.  The load is a
+// separate step so that its latency can overlap other set-up work.
+__device__ __forceinline__ void g1_rot_load(const uint16_t* __restrict__ x, int in, int nb, bool xvec, int b0,
+                                            uint32_t (&w)[8]) {
+  const int lane = threadIdx.x & 31, q = lane & 7;
+  const int b = b0 + (lane >> 3);
+  const bool act = b < nb;
+  const int i0 = kBlock * b + 16 * q;
+  if (xvec) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint4 w = make_uint4(0, 0, 0, 0);
-        if (act && i0 + 8 * j < in) w = __ldg(reinterpret_cast<const uint4*>(x + i0 + 8 * j));
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int j = 0; j < 2; ++j) {
+      uint4 t = make_uint4(0, 0, 0, 0);
+      if (act && i0 + 8 * j < in) t = __ldg(reinterpret_cast<const uint4*>(x + i0 + 8 * j));
+      w[4 * j] = t.x; w[4 * j + 1] = t.y; w[4 * j + 2] = t.z; w[4 * j + 3] = t.w;
+    }
+  } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[8 * j + 2 * k] = __uint_as_float(ww[k] << 16);
-          v[8 * j + 2 * k + 1] = __uint_as_float(ww[k] & 0xffff0000u);
-        }
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t lo = (act && i0 + 2 * e < in) ? __ldg(x + i0 + 2 * e) : 0u;
+      const uint32_t hi = (act && i0 + 2 * e + 1 < in) ? __ldg(x + i0 + 2 * e + 1) : 0u;
+      w[e] = lo | (hi << 16);
+    }
+  }
+}
+
+__device__ __forceinline__ void g1_rot_store(const uint32_t (&w)[8], int nb, int b0, uint16_t* xs, float* xinv) {
+  const int lane = threadIdx.x & 31, q = lane & 7;
+  const int b = b0 + (lane >> 3);
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      if ((e & h) == 0) {
+        const float a = v[e], c = v[e + h];
+        v[e] = a + c;
+        v[e + h] = a - c;
       }
-    } else {
+  }
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = (act && i0 + e < in) ? bf16_bits_to_float(__ldg(x + i0 + e)) : 0.0f;
-    }
+  for (int lm = 1; lm < 8; lm <<= 1) {
+    const float sgn = (lane & lm) ? -1.0f : 1.0f;
 #pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
+    for (int e = 0; e < 16; ++e) v[e] = fmaf(v[e], sgn, __shfl_xor_sync(0xffffffffu, v[e], lm));
+  }
+  float mx = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if ((e & h) == 0) {
-          const float a = v[e], c = v[e + h];
-          v[e] = a + c;
-          v[e + h] = a - c;
-        }
-    }
+  for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
 #pragma unroll
-    for (int lm = 1; lm < 8; lm <<= 1) {
-      const float sgn = (lane & lm) ? -1.0f : 1.0f;
+  for (int lm = 1; lm < 8; lm <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lm));
+  int ex = 0;
+  if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
+  const int k = max(-120, min(120, 10 - ex));
+  const float sc = ldexpf(1.0f, k);
+  if (b < nb) {
+    uint4* dst = reinterpret_cast<uint4*>(xs);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = fmaf(v[e], sgn, __shfl_xor_sync(0xffffffffu, v[e], lm));
-    }
-    float mx = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
-#pragma unroll
-    for (int lm = 1; lm < 8; lm <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lm));
-    int ex = 0;
-    if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
-    const int k = max(-120, min(120, 10 - ex));
-    const float sc = ldexpf(1.0f, k);
-    if (act) {
-      uint4* dst = reinterpret_cast<uint4*>(xs + b * kXsStride + 16 * q);
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        dst[c] = make_uint4(pack_half2(v[8 * c] * sc, v[8 * c + 1] * sc), pack_half2(v[8 * c + 2] * sc, v[8 * c + 3] * sc),
-                            pack_half2(v[8 * c + 4] * sc, v[8 * c + 5] * sc),
-                            pack_half2(v[8 * c + 6] * sc, v[8 * c + 7] * sc));
-      if (q == 0) xinv[b] = ldexpf(1.0f, -k);
-    }
+    for (int c = 0; c < 2; ++c)
+      dst[g1_xs_chunk(b, 2 * q + c)] =
+          make_uint4(pack_half2(v[8 * c] * sc, v[8 * c + 1] * sc), pack_half2(v[8 * c + 2] * sc, v[8 * c + 3] * sc),
+                     pack_half2(v[8 * c + 4] * sc, v[8 * c + 5] * sc), pack_half2(v[8 * c + 6] * sc, v[8 * c + 7] * sc));
+    if (q == 0) xinv[b] = ldexpf(1.0f, -k);
   }
 }
 
@@ -230,7 +247,8 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
              void* __restrict__ Y, int out_bf16, int pass_rows, int xvec) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int L2C = 2 * C;   // lanes per row
-  constexpr int G = 32 / L2C;  // rows per item
+  constexpr int G = 32 / L2C;  // rows of one half item
+  constexpr int RG = 2 * G;    // rows per item
   const int nch = (nb + C - 1) / C;
   const G1Layout L = g1_layout(nb, pass_rows, nch, S);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
@@ -239,11 +257,11 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
   uint16_t* c16 = reinterpret_cast<uint16_t*>(smem + L.c16_off);
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
 
-  const int64_t ngroups = (O + G - 1) / G;
+  const int64_t ngroups = (O + RG - 1) / RG;
   const int64_t g0 = static_cast<int64_t>(blockIdx.x) * ngroups / gridDim.x;
   const int64_t g1 = static_cast<int64_t>(blockIdx.x + 1) * ngroups / gridDim.x;
-  const int64_t row0 = g0 * G;
-  const int nrows = static_cast<int>(std::min<int64_t>(g1 * G, O) - row0);
+  const int64_t row0 = g0 * RG;
+  const int nrows = static_cast<int>(std::min<int64_t>(g1 * RG, O) - row0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane / L2C, u = lane % L2C, s = u >> 1, hh = u & 1;
   const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
@@ -251,13 +269,14 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
   // this warp's ring: S slots of one item each, one mbarrier per slot
   const uint32_t ring = sbase + L.ring_off + warp * (S * kG1ItemBytes);
   const uint32_t bar = sbase + L.bar_off + warp * (S * 8);
-  const uint8_t* my_codes = smem + L.ring_off + warp * (S * kG1ItemBytes) + 40 * lane;  // slot layout [G][C][80]
+  const uint8_t* my_codes = smem + L.ring_off + warp * (S * kG1ItemBytes) + 40 * lane;  // slot layout [2G][C][80]
   if (lane == 0) {
 #pragma unroll
     for (int d = 0; d < S; ++d) mbar_init(bar + 8 * d, 1);
     fence_barrier_init();
   }
   __syncwarp();
+  load_codebook16(c16, codebook);  // read by all warps after the first CTA barrier
   const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
   bool ok = true;
   uint32_t phase = 0;    // parity of the next completion, one bit per slot
@@ -265,35 +284,55 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
 
   for (int p0 = 0; p0 < nrows; p0 += pass_rows) {
     const int prow = min(pass_rows, nrows - p0);
-    const int ngr = (prow + G - 1) / G;
+    const int ngr = (prow + RG - 1) / RG;
     const int nitems = ngr * nch;
     const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
     const int nw = it1 - it0;
+    const int64_t prow0 = row0 + p0;
 
-    // issue cursor: item (ich, ig) goes to the slot being refilled
+    // issue cursor: item (ich, ig) goes to the slot being refilled; nptr
+    // points at the norm of (row ig * RG + r, block ich * C + s)
     int ich = it0 / ngr, ig = it0 - (it0 / ngr) * ngr;
+    const uint16_t* nptr = norms + (prow0 + ig * RG + r) * nb + ich * C + s;
     uint32_t nraw[S];
     auto issue = [&](int d) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
-        tma_load_3d(ring + d * kG1ItemBytes, &cmap, 0, ich * C, static_cast<int>(row0 + p0 + ig * G), bar + 8 * d);
+        tma_load_3d(ring + d * kG1ItemBytes, &cmap, 0, ich * C, static_cast<int>(prow0 + ig * RG), bar + 8 * d);
       }
-      const int v = ig * G + r, b = ich * C + s;
-      nraw[d] = (v < prow && b < nb) ? static_cast<uint32_t>(__ldg(norms + (row0 + p0 + v) * nb + b)) : 0u;
+      const int v = ig * RG + r;
+      const bool bok = ich * C + s < nb;
+      const uint32_t n0 = (bok && v < prow) ? static_cast<uint32_t>(__ldg(nptr)) : 0u;
+      const uint32_t n1 = (bok && v + G < prow) ? static_cast<uint32_t>(__ldg(nptr + G * nb)) : 0u;
+      nraw[d] = n0 | (n1 << 16);
       pending |= 1u << d;
-      if (++ig == ngr) { ig = 0; ++ich; }
+      if (++ig == ngr) {
+        ig = 0;
+        ++ich;
+        nptr = norms + (prow0 + r) * nb + ich * C + s;
+      } else {
+        nptr += RG * nb;
+      }
     };
 #pragma unroll
     for (int d = 0; d < S; ++d)
       if (d < nw) issue(d);
 
     if (p0 == 0) {
-      // set-up while the first boxes are in flight
-      load_codebook16(c16, codebook);
-      __syncthreads();
-      build_pair_table_warps(reinterpret_cast<uint32_t*>(smem), c16, 0, kG1Warps);
+      // set-up while the first boxes are in flight: the first round of x
+      // loads is issued before the pair table is built, so its latency
+      // overlaps the table stores
       pdl_wait();  // x may be produced by the previous kernel on the stream
-      g1_rotate(x, in, nb, xvec != 0, xs, xinv);
+      uint32_t xw[8];
+      const int rb0 = 4 * warp;
+      if (rb0 < nb) g1_rot_load(x, in, nb, xvec != 0, rb0, xw);
+      __syncthreads();  // c16
+      build_pair_table_warps(reinterpret_cast<uint32_t*>(smem), c16, 0, kG1Warps);
+      if (rb0 < nb) g1_rot_store(xw, nb, rb0, xs, xinv);
+      for (int b0 = rb0 + 4 * kG1Warps; b0 < nb; b0 += 4 * kG1Warps) {
+        g1_rot_load(x, in, nb, xvec != 0, b0, xw);
+        g1_rot_store(xw, nb, b0, xs, xinv);
+      }
       __syncthreads();
       pdl_trigger();
     }
@@ -308,16 +347,19 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
         if (k < nw) {
           const uint32_t nr = nraw[d];
           if (ok && ((pending >> d) & 1u)) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar + 8 * d, (phase >> d) & 1u, deadline));
             if (ok) {
               phase ^= 1u << d;
               pending &= ~(1u << d);
             }
           }
-          uint2 cw[5];
+          uint2 cw0[5], cw1[5];
           const uint2* src = reinterpret_cast<const uint2*>(my_codes + d * kG1ItemBytes);
 #pragma unroll
-          for (int q = 0; q < 5; ++q) cw[q] = src[q];
+          for (int q = 0; q < 5; ++q) {
+            cw0[q] = src[q];
+            cw1[q] = src[q + kG1ItemBytes / 16];  // row r + G: half a slot further
+          }
           __syncwarp();
           if (ok && k + S < nw) {
             if (lane == 0) fence_proxy_async();  // the slot's reads precede the refill
@@ -327,10 +369,10 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
             xch = cch;
             const int b = cch * C + s;
             if (b < nb) {
-              const uint4* xsrc = reinterpret_cast<const uint4*>(xs + b * kXsStride + 64 * hh);
+              const uint4* xsrc = reinterpret_cast<const uint4*>(xs);
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
-                const uint4 w = xsrc[q];
+                const uint4 w = xsrc[g1_xs_chunk(b, 8 * hh + q)];
                 xr[4 * q] = w.x; xr[4 * q + 1] = w.y; xr[4 * q + 2] = w.z; xr[4 * q + 3] = w.w;
               }
               xi = xinv[b] * (1.0f / 128.0f);
@@ -340,12 +382,18 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
               xi = 0.0f;
             }
           }
-          float acc = g1_dot(smem, cw, lane4, xr, std::make_integer_sequence<int, 32>{});
-          acc *= half_bits_to_float(static_cast<uint16_t>(nr)) * xi;
+          const float a0 = g1_dot(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+                           (half_bits_to_float(static_cast<uint16_t>(nr)) * xi);
+          const float a1 = g1_dot(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+                           (half_bits_to_float(static_cast<uint16_t>(nr >> 16)) * xi);
+          // reduce both rows over the 2C lanes: the first exchange leaves row
+          // r's partial on lanes with bit C clear and row r + G's on the others
+          const bool hi = (u & C) != 0;
+          float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
 #pragma unroll
-          for (int off = L2C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-          const int v = cg * G + r;
-          if (u == 0 && v < prow) part[v * nch + cch] = acc;
+          for (int off = C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+          const int v = cg * RG + r + (hi ? G : 0);
+          if ((u & (C - 1)) == 0 && v < prow) part[v * nch + cch] = acc;
           if (++cg == ngr) { cg = 0; ++cch; }
         }
       }
@@ -354,7 +402,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       // a box never arrived: drain what is still in flight (bounded), then stop
       const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
       for (int d = 0; d < S; ++d)
-        if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
+        if ((pending >> d) & 1u) mbar_wait_sleep(bar + 8 * d, (phase >> d) & 1u, dl);
       if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
     }
     __syncthreads();
@@ -362,7 +410,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       const float* pr = part + v * nch;
       float sum = 0.0f;
       for (int ch = 0; ch < nch; ++ch) sum += pr[ch];
-      const int64_t o = row0 + p0 + v;
+      const int64_t o = prow0 + v;
       if (out_bf16) static_cast<uint16_t*>(Y)[o] = static_cast<uint16_t>(float_to_bf16_bits(sum));
       else static_cast<float*>(Y)[o] = sum;
     }
@@ -395,12 +443,12 @@ inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, CUtensorMa
   }
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
-  const int G = 16 / C;
+  const int RG = 32 / C;  // rows per item
   const cuuint64_t dim[3] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb),
                              static_cast<cuuint64_t>(O)};
   const cuuint64_t stride[2] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb) * kBlockBytes};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(C),
-                             static_cast<cuuint32_t>(G)};
+                             static_cast<cuuint32_t>(RG)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUtensorMap m;
   if (encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dim, stride, box, estr,
@@ -421,10 +469,10 @@ inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, CUtensorMa
 
 // Rows of a CTA handled per pass for ring depth S (0 if the layout does not fit).
 inline int g1_pass_rows(int nb, int C, int S, int rows_cta) {
-  const int G = 16 / C, nch = (nb + C - 1) / C;
+  const int RG = 32 / C, nch = (nb + C - 1) / C;
   const int fixed = g1_layout(nb, 0, nch, S).total;
-  const int cap = (227 * 1024 - fixed - 16) / (nch * 4) / G * G;
-  return cap < G ? 0 : std::min(rows_cta, cap);
+  const int cap = (227 * 1024 - fixed - 16) / (nch * 4) / RG * RG;
+  return cap < RG ? 0 : std::min(rows_cta, cap);
 }
 
 template <int C, int S>
@@ -461,16 +509,14 @@ template <int C>
 int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                    const uint16_t* x, void* Y, bool out_bf16, unsigned flags, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
-  constexpr int G = 16 / C;
-  const int64_t ngroups = ceil_div(O, G);
+  constexpr int RG = 32 / C;
+  const int64_t ngroups = ceil_div(O, RG);
   const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
-  const int rows_cta = static_cast<int>(ceil_div(ngroups, grid) * G);
+  const int rows_cta = static_cast<int>(ceil_div(ngroups, grid) * RG);
   CUtensorMap map;
   const int st = codes_map(packed, O, nb, C, &map);
   if (st != HLWQ_OK) return st;
   // deepest ring that fits beside the table and the rotated activation
-  if (const int pr = g1_pass_rows(nb, C, 4, rows_cta))
-    return launch_gemv1_cs<C, 4>(map, norms, codebook, O, in, nb, x, Y, out_bf16, flags, grid, pr, stream);
   if (const int pr = g1_pass_rows(nb, C, 2, rows_cta))
     return launch_gemv1_cs<C, 2>(map, norms, codebook, O, in, nb, x, Y, out_bf16, flags, grid, pr, stream);
   if (const int pr = g1_pass_rows(nb, C, 1, rows_cta))
@@ -480,14 +526,22 @@ int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* co
 
 }  // namespace
 
+int launch_dense_m1(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                    const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream);
+
 int launch_gemv1(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream, unsigned flags) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
+  int st;
   switch (pick_chunk(nb)) {
-    case 8: return launch_gemv1_c<8>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
-    case 4: return launch_gemv1_c<4>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
-    default: return launch_gemv1_c<2>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream);
+    case 8: st = launch_gemv1_c<8>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream); break;
+    case 4: st = launch_gemv1_c<4>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream); break;
+    default: st = launch_gemv1_c<2>(packed, norms, codebook, O, in, x, Y, out_bf16, flags, stream); break;
   }
+  // rows too long for the code ring beside the table and the activation:
+  // the CUDA-core decode kernel (no ring) takes them
+  if (st == HLWQ_EUNSUPPORTED) st = launch_dense_m1(packed, norms, codebook, O, in, x, Y, out_bf16, stream);
+  return st;
 }
 
 namespace {
@@ -537,6 +591,17 @@ int dense_smem_bytes(int64_t O, int in, int mt) {
   const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
   const int max_rows = static_cast<int>(ceil_div(ngroups, grid) * G);
   return engine_layout(mt, nb, max_rows, (nb + C - 1) / C).total;
+}
+
+int launch_dense_m1(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                    const uint16_t* x, void* Y, bool out_bf16, cudaStream_t stream) {
+  const int nb = static_cast<int>(ceil_div(in, kBlock));
+  if (dense_smem_bytes(O, in, 1) > 227 * 1024) return HLWQ_EUNSUPPORTED;
+  switch (pick_chunk(nb)) {
+    case 8: return launch_dense_c<8>(1, packed, norms, codebook, O, in, x, in, 1, Y, O, out_bf16, stream);
+    case 4: return launch_dense_c<4>(1, packed, norms, codebook, O, in, x, in, 1, Y, O, out_bf16, stream);
+    default: return launch_dense_c<2>(1, packed, norms, codebook, O, in, x, in, 1, Y, O, out_bf16, stream);
+  }
 }
 
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,

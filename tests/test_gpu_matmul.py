@@ -102,24 +102,36 @@ def test_gemv_ex_rejects_unknown_flags(hl, cb):
     assert st == hl.HLWQ_EINVAL
 
 
-def test_gemv_long_rows_several_passes(hl, cb):
-    """in = 32768 (256 blocks): the rotated activation takes most of shared
-    memory, so the code ring is one slot deep and each CTA covers its ~160 rows
-    in several passes (rows sampled for the oracle, including the first and
-    last rows of the matrix and rows around pass boundaries)."""
-    Od, I = 11700, 32768
-    W = synth.student_t_device((Od, I), seed=12)
+def _sampled_gemv(hl, cb, Od, I, seed, rows):
+    W = synth.student_t_device((Od, I), seed=seed)
     p, n = hl.quantize(W, cb)
-    x = synth.activations(1, I, seed=13)
+    x = synth.activations(1, I, seed=seed + 1)
     y = hl.gemv(p, n, cb, x[0].cuda())
     torch.cuda.synchronize()
-    rows = np.unique(np.concatenate([np.arange(0, 24), np.arange(70, 90), np.arange(150, 170),
-                                     np.arange(Od - 16, Od),
-                                     np.random.default_rng(1).choice(Od, 24, replace=False)]))
     q = O.quantize(W[torch.as_tensor(rows, device=W.device)].cpu())
-    del W
+    del W, p, n
     want = O.matmul(q["packed"], q["norms"], I, x)[0]
-    assert rel_l2(y.cpu().numpy()[rows], want) <= MATMUL_REL
+    return rel_l2(y.cpu().numpy()[rows], want)
+
+
+def test_gemv_long_rows_several_passes(hl, cb):
+    """in = 27648 (216 blocks): the rotated activation takes most of shared
+    memory, so the code ring is one slot deep and a CTA covers its 44 rows in
+    two passes of 36 and 8 (rows sampled for the oracle: the first CTAs' pass
+    boundaries, the last rows and random rows)."""
+    Od, I = 6000, 27648
+    rows = np.unique(np.concatenate([np.arange(0, 48), np.arange(80, 92), np.arange(Od - 16, Od),
+                                     np.random.default_rng(1).choice(Od, 24, replace=False)]))
+    assert _sampled_gemv(hl, cb, Od, I, 12, rows) <= MATMUL_REL
+
+
+def test_gemv_rows_too_long_for_the_ring(hl, cb):
+    """in = 32768 (256 blocks): no code ring fits beside the table and the
+    activation; the CUDA-core decode kernel takes the call."""
+    Od, I = 600, 32768
+    rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(Od - 8, Od),
+                                     np.random.default_rng(2).choice(Od, 24, replace=False)]))
+    assert _sampled_gemv(hl, cb, Od, I, 14, rows) <= MATMUL_REL
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 9, 15, 16, 17, 64])
