@@ -51,12 +51,28 @@ def load_peaks():
 
 
 def load_traffic():
-    """Per-launch DRAM bytes from the committed ncu summary (profiles/), if any."""
+    """Per-launch DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from
+    the committed ncu summaries (profiles/traffic.json).  An entry counts only
+    while the kernel sources it was measured on are unchanged (sha1 of the
+    listed files); otherwise its traffic is reported as null."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return json.load(f)
-    return {}
+    if not os.path.exists(p):
+        return {}
+    with open(p) as f:
+        entries = json.load(f)
+    out = {}
+    for key, e in entries.items():
+        m = hashlib.sha1()
+        try:
+            for name in e["sources"]:
+                with open(os.path.join(ROOT, "dequant_matmul_b200", "csrc", name), "rb") as src:
+                    m.update(src.read())
+        except OSError:
+            continue
+        if m.hexdigest() == e.get("source_sha1"):
+            out[key] = e["dram_bytes_per_launch"]
+    return out
 
 
 class ClockSampler:
