@@ -130,6 +130,16 @@ extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
   const size_t need = hlwq_workspace_bytes(HLWQ_OP_MOE, H, F, T, E, topk);
   if (!workspace || ws_bytes < need) return HLWQ_EWORKSPACE;
   if (!aligned16(workspace)) return HLWQ_EALIGN;
+  // few tokens: two fused kernels on the TMA-fed decode engine; otherwise (or
+  // when the pairs' activations do not fit in shared memory) the four-kernel
+  // path that reads each active expert once for all its tokens
+  hlwq::MoeWs ws;
+  hlwq::moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
+  const int st = hlwq::launch_moe1(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+                                   sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H),
+                                   static_cast<int>(F), static_cast<int>(topk), static_cast<int>(T), router_logits, X,
+                                   Y, ydtype == HLWQ_BF16, topk_ids, topk_weights, ws.h, as_stream(stream));
+  if (st != HLWQ_EUNSUPPORTED) return st;
   return hlwq::launch_moe(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
                           sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H), static_cast<int>(F),
                           static_cast<int>(topk), static_cast<int>(T), router_logits, X, Y, ydtype == HLWQ_BF16,

@@ -145,65 +145,125 @@ __device__ __forceinline__ uint32_t g1_off(const uint2 (&cw)[5], uint32_t lane4)
   return (t & 0x1ff80u) | lane4;
 }
 
-// Pair P goes to fp16 chain P % 4 (four independent chains of 8 products).
-template <int P>
+// Pair P goes to fp16 chain P % NC.  NC = 4: four chains of 8 products, added
+// pairwise in fp16 (a block's codes have sum c^2 ~ 128, so a 16-product sum
+// stays below sqrt(135) * 4 * 2^10 < 65504 for |x_tilde| < 2^10) and widened
+// once.  NC = 8: eight chains of 4 products, each widened to fp32 (smaller
+// rounding error, for chained products such as the MoE layer).
+template <int NC, int P>
 __device__ __forceinline__ void g1_pair(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
-                                        const uint32_t (&xr)[32], uint32_t (&h)[4]) {
+                                        const uint32_t (&xr)[32], uint32_t (&h)[NC]) {
   const uint32_t e = *reinterpret_cast<const uint32_t*>(tab + g1_off<P>(cw, lane4));
-  if constexpr (P < 4) h[P] = hmul2(e, xr[P]);
-  else h[P & 3] = hfma2(e, xr[P], h[P & 3]);
+  if constexpr (P < NC) h[P] = hmul2(e, xr[P]);
+  else h[P % NC] = hfma2(e, xr[P], h[P % NC]);
+}
+
+__device__ __forceinline__ float2 half2_to_float2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
+template <int NC, int... P>
+__device__ __forceinline__ float g1_dot_n(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
+                                          const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
+  uint32_t h[NC];
+  (g1_pair<NC, P>(tab, cw, lane4, xr, h), ...);
+  if constexpr (NC == 4) {
+    const float2 f0 = half2_to_float2(hadd2(h[0], h[1]));
+    const float2 f1 = half2_to_float2(hadd2(h[2], h[3]));
+    return (f0.x + f1.x) + (f0.y + f1.y);
+  } else {
+    float2 f[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) f[c] = half2_to_float2(h[c]);
+#pragma unroll
+    for (int w = NC / 2; w > 0; w >>= 1)
+#pragma unroll
+      for (int c = 0; c < w; ++c) f[c] = make_float2(f[c].x + f[c + w].x, f[c].y + f[c + w].y);
+    return f[0].x + f[0].y;
+  }
 }
 
 template <int... P>
 __device__ __forceinline__ float g1_dot(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
-                                        const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
-  uint32_t h[4];
-  (g1_pair<P>(tab, cw, lane4, xr, h), ...);
-  // two chains at a time are added in fp16 (16 products: the codes of a block
-  // have sum c^2 ~ 128, so |sum| <= sqrt(135) * 4 * 2^10 < 65504), then widened
-  const uint32_t h01 = hadd2(h[0], h[1]), h23 = hadd2(h[2], h[3]);
-  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-  return (f0.x + f1.x) + (f0.y + f1.y);
+                                        const uint32_t (&xr)[32], std::integer_sequence<int, P...> seq) {
+  return g1_dot_n<4>(tab, cw, lane4, xr, seq);
 }
 
-// Rotation of x with eight lanes per 128-block (16 consecutive values per
-// lane: four butterfly stages in registers, three across lanes); a warp covers
-// blocks b0 .. b0 + 3.  Block b is scaled by 2^k so that max |x_tilde| * 2^k
-// lies in [2^9, 2^10) and stored as binary16; xinv[b] = 2^-k.  The load is a
-// separate step so that its latency can overlap other set-up work.
-__device__ __forceinline__ void g1_rot_load(const uint16_t* __restrict__ x, int in, int nb, bool xvec, int b0,
-                                            uint32_t (&w)[8]) {
-  const int lane = threadIdx.x & 31, q = lane & 7;
-  const int b = b0 + (lane >> 3);
-  const bool act = b < nb;
-  const int i0 = kBlock * b + 16 * q;
+// Lane l's centroid c[l] as binary16 (warp 0 also checks that the codebook is
+// strictly ascending and raises HLWQ_DEVERR_CODEBOOK otherwise).
+__device__ __forceinline__ uint32_t g1_codebook_lane(const float* __restrict__ codebook) {
+  const int lane = threadIdx.x & 31;
+  const float c = __ldg(codebook + lane);
+  if (threadIdx.x < 32) {
+    const float next = __shfl_down_sync(0xffffffffu, c, 1);
+    if (lane + 1 < kLevels && !(c < next)) raise_device_error(HLWQ_DEVERR_CODEBOOK);
+  }
+  return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(c)));
+}
+
+// Warps [w0, w0 + nw) write the lane-replicated pair table, word (v * 32 +
+// lane) = half2(c[v & 31], c[v >> 5]), from the centroids in their lanes (no
+// shared copy of the codebook, so no CTA barrier before the table is built).
+__device__ __forceinline__ void g1_build_table(uint8_t* smem, uint32_t c16r, int w0, int nw) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < w0 || warp >= w0 + nw) return;
+  uint4* t4 = reinterpret_cast<uint4*>(smem);
+  for (int q = (warp - w0) * 32 + lane; q < 1024 * 8; q += nw * 32) {  // same trip count on every lane
+    const int v = q >> 3;
+    const uint32_t e = __shfl_sync(0xffffffffu, c16r, v & 31) | (__shfl_sync(0xffffffffu, c16r, v >> 5) << 16);
+    t4[q] = make_uint4(e, e, e, e);
+  }
+}
+
+// Rotation of activation vectors with eight lanes per 128-block (16
+// consecutive values per lane: four butterfly stages in registers, three
+// across lanes).  Blocks are numbered gb = vector * nb + block over nvec
+// vectors of `in` values (row pitch ld); a warp covers blocks gb0 .. gb0 + 3.
+// Block gb is scaled by 2^k so that max |x_tilde| * 2^k lies in [2^9, 2^10)
+// and stored as binary16 at chunks g1_xs_chunk(gb, .); xinv[gb] = 2^-k.  The
+// load is a separate step so that its latency can overlap other set-up work.
+struct RotBlock {
+  int gb, vec, b, i0;
+  bool act;
+};
+
+__device__ __forceinline__ RotBlock g1_rot_block(int nb, int nblocks, int gb0) {
+  const int lane = threadIdx.x & 31;
+  RotBlock B;
+  B.gb = gb0 + (lane >> 3);
+  B.act = B.gb < nblocks;
+  B.vec = B.act ? B.gb / nb : 0;
+  B.b = B.gb - B.vec * nb;
+  B.i0 = kBlock * B.b + 16 * (lane & 7);
+  return B;
+}
+
+// bf16 source: the 16 values as 8 words (kept packed while other work runs).
+__device__ __forceinline__ void g1_rot_load(const uint16_t* __restrict__ x, int64_t ld, int in, int nb, int nblocks,
+                                            bool xvec, int gb0, uint32_t (&w)[8]) {
+  const RotBlock B = g1_rot_block(nb, nblocks, gb0);
+  const uint16_t* row = x + B.vec * ld;
   if (xvec) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       uint4 t = make_uint4(0, 0, 0, 0);
-      if (act && i0 + 8 * j < in) t = __ldg(reinterpret_cast<const uint4*>(x + i0 + 8 * j));
+      if (B.act && B.i0 + 8 * j < in) t = __ldg(reinterpret_cast<const uint4*>(row + B.i0 + 8 * j));
       w[4 * j] = t.x; w[4 * j + 1] = t.y; w[4 * j + 2] = t.z; w[4 * j + 3] = t.w;
     }
   } else {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const uint32_t lo = (act && i0 + 2 * e < in) ? __ldg(x + i0 + 2 * e) : 0u;
-      const uint32_t hi = (act && i0 + 2 * e + 1 < in) ? __ldg(x + i0 + 2 * e + 1) : 0u;
+      const uint32_t lo = (B.act && B.i0 + 2 * e < in) ? __ldg(row + B.i0 + 2 * e) : 0u;
+      const uint32_t hi = (B.act && B.i0 + 2 * e + 1 < in) ? __ldg(row + B.i0 + 2 * e + 1) : 0u;
       w[e] = lo | (hi << 16);
     }
   }
 }
 
-__device__ __forceinline__ void g1_rot_store(const uint32_t (&w)[8], int nb, int b0, uint16_t* xs, float* xinv) {
+__device__ __forceinline__ void g1_rot_core(float (&v)[16], int nb, int nblocks, int gb0, uint16_t* xs,
+                                            float* xinv) {
   const int lane = threadIdx.x & 31, q = lane & 7;
-  const int b = b0 + (lane >> 3);
-  float v[16];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    v[2 * k] = __uint_as_float(w[k] << 16);
-    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-  }
+  const RotBlock B = g1_rot_block(nb, nblocks, gb0);
 #pragma unroll
   for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
@@ -229,15 +289,37 @@ __device__ __forceinline__ void g1_rot_store(const uint32_t (&w)[8], int nb, int
   if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
   const int k = max(-120, min(120, 10 - ex));
   const float sc = ldexpf(1.0f, k);
-  if (b < nb) {
+  if (B.act) {
     uint4* dst = reinterpret_cast<uint4*>(xs);
 #pragma unroll
     for (int c = 0; c < 2; ++c)
-      dst[g1_xs_chunk(b, 2 * q + c)] =
+      dst[g1_xs_chunk(B.gb, 2 * q + c)] =
           make_uint4(pack_half2(v[8 * c] * sc, v[8 * c + 1] * sc), pack_half2(v[8 * c + 2] * sc, v[8 * c + 3] * sc),
                      pack_half2(v[8 * c + 4] * sc, v[8 * c + 5] * sc), pack_half2(v[8 * c + 6] * sc, v[8 * c + 7] * sc));
-    if (q == 0) xinv[b] = ldexpf(1.0f, -k);
+    if (q == 0) xinv[B.gb] = ldexpf(1.0f, -k);
   }
+}
+
+__device__ __forceinline__ void g1_rot_store(const uint32_t (&w)[8], int nb, int nblocks, int gb0, uint16_t* xs,
+                                             float* xinv) {
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+  g1_rot_core(v, nb, nblocks, gb0, xs, xinv);
+}
+
+// fp32 source (the MoE intermediate h), loaded and rotated in one step.
+__device__ __forceinline__ void g1_rot_f32(const float* __restrict__ x, int64_t ld, int in, int nb, int nblocks,
+                                           int gb0, uint16_t* xs, float* xinv) {
+  const RotBlock B = g1_rot_block(nb, nblocks, gb0);
+  const float* row = x + B.vec * ld;
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = (B.act && B.i0 + e < in) ? row[B.i0 + e] : 0.0f;
+  g1_rot_core(v, nb, nblocks, gb0, xs, xinv);
 }
 
 template <int C, int S>
@@ -245,7 +327,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
 gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restrict__ norms,
              const float* __restrict__ codebook, int64_t O, int in, int nb, const uint16_t* __restrict__ x,
              void* __restrict__ Y, int out_bf16, int pass_rows, int xvec) {
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(16) uint8_t smem[];
   constexpr int L2C = 2 * C;   // lanes per row
   constexpr int G = 32 / L2C;  // rows of one half item
   constexpr int RG = 2 * G;    // rows per item
@@ -254,7 +336,6 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
   float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
   float* part = reinterpret_cast<float*>(smem + L.part_off);
-  uint16_t* c16 = reinterpret_cast<uint16_t*>(smem + L.c16_off);
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
 
   const int64_t ngroups = (O + RG - 1) / RG;
@@ -276,7 +357,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     fence_barrier_init();
   }
   __syncwarp();
-  load_codebook16(c16, codebook);  // read by all warps after the first CTA barrier
+  const uint32_t c16r = g1_codebook_lane(codebook);
   const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
   bool ok = true;
   uint32_t phase = 0;    // parity of the next completion, one bit per slot
@@ -321,17 +402,16 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     if (p0 == 0) {
       // set-up while the first boxes are in flight: the first round of x
       // loads is issued before the pair table is built, so its latency
-      // overlaps the table stores
+      // overlaps the table stores; the barrier below publishes both
       pdl_wait();  // x may be produced by the previous kernel on the stream
       uint32_t xw[8];
       const int rb0 = 4 * warp;
-      if (rb0 < nb) g1_rot_load(x, in, nb, xvec != 0, rb0, xw);
-      __syncthreads();  // c16
-      build_pair_table_warps(reinterpret_cast<uint32_t*>(smem), c16, 0, kG1Warps);
-      if (rb0 < nb) g1_rot_store(xw, nb, rb0, xs, xinv);
+      if (rb0 < nb) g1_rot_load(x, in, in, nb, nb, xvec != 0, rb0, xw);
+      g1_build_table(smem, c16r, 0, kG1Warps);
+      if (rb0 < nb) g1_rot_store(xw, nb, nb, rb0, xs, xinv);
       for (int b0 = rb0 + 4 * kG1Warps; b0 < nb; b0 += 4 * kG1Warps) {
-        g1_rot_load(x, in, nb, xvec != 0, b0, xw);
-        g1_rot_store(xw, nb, b0, xs, xinv);
+        g1_rot_load(x, in, in, nb, nb, xvec != 0, b0, xw);
+        g1_rot_store(xw, nb, nb, b0, xs, xinv);
       }
       __syncthreads();
       pdl_trigger();
@@ -347,7 +427,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
         if (k < nw) {
           const uint32_t nr = nraw[d];
           if (ok && ((pending >> d) & 1u)) {
-            ok = __all_sync(0xffffffffu, mbar_wait_sleep(bar + 8 * d, (phase >> d) & 1u, deadline));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
             if (ok) {
               phase ^= 1u << d;
               pending &= ~(1u << d);
@@ -402,7 +482,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       // a box never arrived: drain what is still in flight (bounded), then stop
       const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
       for (int d = 0; d < S; ++d)
-        if ((pending >> d) & 1u) mbar_wait_sleep(bar + 8 * d, (phase >> d) & 1u, dl);
+        if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
       if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
     }
     __syncthreads();
@@ -419,36 +499,36 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
   }
 }
 
-// Tensor map of the codes viewed as a 3-D byte tensor {80, NB, O}; one box is
-// one item {80, C, G}.  Encoding costs host time, so the last few maps are
-// kept (a map depends only on the pointer and the shape).
+// Tensor map of the codes viewed as a 3-D byte tensor {80, NB, O}.  Encoding
+// costs host time, so the last few maps are kept (a map depends only on the
+// pointer, the shape and the box).
 struct CodesMapEntry {
   const void* ptr;
   int64_t O;
-  int nb, C;
+  int nb, C, rows;
   CUtensorMap map;
 };
 
-inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, CUtensorMap* out) {
+// box = {80 bytes, C blocks, box_rows rows}
+inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, int box_rows, CUtensorMap* out) {
   static std::mutex mu;
   static CodesMapEntry cache[8];
   static int used = 0, next = 0;
   std::lock_guard<std::mutex> lock(mu);
   for (int k = 0; k < used; ++k) {
     const CodesMapEntry& e = cache[k];
-    if (e.ptr == packed && e.O == O && e.nb == nb && e.C == C) {
+    if (e.ptr == packed && e.O == O && e.nb == nb && e.C == C && e.rows == box_rows) {
       *out = e.map;
       return HLWQ_OK;
     }
   }
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
-  const int RG = 32 / C;  // rows per item
   const cuuint64_t dim[3] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb),
                              static_cast<cuuint64_t>(O)};
   const cuuint64_t stride[2] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nb) * kBlockBytes};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(C),
-                             static_cast<cuuint32_t>(RG)};
+                             static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUtensorMap m;
   if (encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dim, stride, box, estr,
@@ -460,6 +540,7 @@ inline int codes_map(const uint8_t* packed, int64_t O, int nb, int C, CUtensorMa
   e.O = O;
   e.nb = nb;
   e.C = C;
+  e.rows = box_rows;
   e.map = m;
   next = (next + 1) % 8;
   used = std::min(used + 1, 8);
@@ -514,7 +595,7 @@ int launch_gemv1_c(const uint8_t* packed, const uint16_t* norms, const float* co
   const int grid = static_cast<int>(std::min<int64_t>(sm_count(), ngroups));
   const int rows_cta = static_cast<int>(ceil_div(ngroups, grid) * RG);
   CUtensorMap map;
-  const int st = codes_map(packed, O, nb, C, &map);
+  const int st = codes_map(packed, O, nb, C, RG, &map);
   if (st != HLWQ_OK) return st;
   // deepest ring that fits beside the table and the rotated activation
   if (const int pr = g1_pass_rows(nb, C, 2, rows_cta))

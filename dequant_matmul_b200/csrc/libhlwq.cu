@@ -3,5 +3,6 @@
 #include "quantize.cuh"
 #include "gemv.cuh"
 #include "moe.cuh"
+#include "moe1.cuh"
 #include "gemm_tc.cuh"
 #include "api.cuh"

@@ -76,49 +76,87 @@ size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char
   return off;
 }
 
+// Top-k routing of one token by one warp: the k largest logits (ties: lower
+// expert id) and softmax weights over the k selected logits, accumulated in
+// selection order.  ids / wts get k entries; every lane of the warp must call
+// it.  Each logit (expert lane + 32 i, E <= 1024) is held as an unsigned key
+// whose order is the float order (-0 counted as +0; logits must not be NaN),
+// so one selection round is a warp max-reduction of the keys and a min-
+// reduction of the indices that hold the maximum (a real key is never 0: the
+// smallest, that of -NaN payloads aside, is the key of -inf, 0x007fffff).
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7fffffffu) == 0u) b = 0u;  // -0 == +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// NL keys per lane (E <= 32 NL); per-lane maxima and minima as pairwise trees.
+template <int NL>
+__device__ __forceinline__ void route_token_warp_n(const float* __restrict__ lg, int E, int topk, int* ids,
+                                                   float* wts) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NL];
+#pragma unroll
+  for (int i = 0; i < NL; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? logit_key(__ldg(lg + e)) : 0u;  // key 0: absent or taken (real keys are > 0)
+  }
+  float vmax = 0.0f, wsum = 0.0f;
+  for (int s = 0; s < topk; ++s) {
+    uint32_t t[NL];
+#pragma unroll
+    for (int i = 0; i < NL; ++i) t[i] = key[i];
+#pragma unroll
+    for (int w = NL / 2; w > 0; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) t[i] = max(t[i], t[i + w]);
+    const uint32_t gm = __reduce_max_sync(0xffffffffu, t[0]);
+#pragma unroll
+    for (int i = 0; i < NL; ++i) t[i] = key[i] == gm ? static_cast<uint32_t>(lane + 32 * i) : 0xffffffffu;
+#pragma unroll
+    for (int w = NL / 2; w > 0; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) t[i] = min(t[i], t[i + w]);
+    const int bi = static_cast<int>(__reduce_min_sync(0xffffffffu, t[0]));
+#pragma unroll
+    for (int i = 0; i < NL; ++i)
+      if (lane + 32 * i == bi) key[i] = 0u;
+    const float bv = key_logit(gm);
+    if (s == 0) vmax = bv;
+    const float ex = expf(bv - vmax);
+    wsum += ex;
+    if (lane == 0) {
+      ids[s] = bi;
+      wts[s] = ex;
+    }
+  }
+  __syncwarp();
+  if (lane < topk) wts[lane] = wts[lane] / wsum;
+  __syncwarp();
+}
+
+__device__ __forceinline__ void route_token_warp(const float* __restrict__ lg, int E, int topk, int* ids,
+                                                 float* wts) {
+  if (E <= 256) route_token_warp_n<8>(lg, E, topk, ids, wts);
+  else route_token_warp_n<32>(lg, E, topk, ids, wts);
+}
+
 __global__ void __launch_bounds__(kRouterThreads, 1)
 router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, int E, int H, int T, int topk,
               int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
   __shared__ int s_count[1025];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per_lane = (E + 31) / 32;
 
   // 1. top-k + softmax, one warp per token.
   for (int t = warp; t < T; t += kRouterThreads / 32) {
-    const float* lg = logits + static_cast<int64_t>(t) * E;
-    unsigned taken = 0u;  // bit i: element lane + 32 i selected
-    float vmax = 0.0f, wsum = 0.0f;
-    for (int s = 0; s < topk; ++s) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int i = 0; i < per_lane; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u)) {
-          const float v = lg[e];
-          if (v > bv || (v == bv && e < bi) || bi == 0x7fffffff) { bv = v; bi = e; }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (s == 0) vmax = bv;
-      const float ex = expf(bv - vmax);
-      wsum += ex;
-      if (lane == 0) {
-        ws.sel_id[t * topk + s] = bi;
-        ws.sel_w[t * topk + s] = ex;
-      }
-    }
-    __syncwarp();
+    route_token_warp(logits + static_cast<int64_t>(t) * E, E, topk, ws.sel_id + t * topk, ws.sel_w + t * topk);
     if (lane < topk) {
-      const float wv = ws.sel_w[t * topk + lane] / wsum;
-      ws.sel_w[t * topk + lane] = wv;
       if (ids_out) ids_out[t * topk + lane] = ws.sel_id[t * topk + lane];
-      if (w_out) w_out[t * topk + lane] = wv;
+      if (w_out) w_out[t * topk + lane] = ws.sel_w[t * topk + lane];
     }
   }
   __syncthreads();
