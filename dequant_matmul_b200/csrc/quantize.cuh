@@ -40,6 +40,7 @@ namespace hlwq {
 namespace {
 
 constexpr int kQThreads = 256;
+constexpr int kQCtasPerSm = 3;  // 85 registers per thread: the code group and the rotation stay in registers
 constexpr int kQBuckets = 385;           // clamped shifted value in [-3, 3] at 1/64 resolution
 constexpr float kQGuard = 2e-5f;
 constexpr float kQMagic = 12583104.0f;   // 1.5 * 2^23 + 192: fmaf(y, 64, kQMagic) -> round(64 y + 192) in the low bits
@@ -235,19 +236,23 @@ __device__ __forceinline__ float quad_sum_m(float x, unsigned mask) {
 
 // Replaces the 5-bit field of code e (0..31) in a lane's 160-bit group p[5].
 __device__ __forceinline__ void patch_code(uint32_t (&p)[5], int e, uint32_t code) {
-  const int bit = 5 * e, w = bit >> 5, sh = bit & 31;
+  // the field's bits are written into each word they overlap, with shift
+  // amounts computed at run time (a runtime index into p would put the whole
+  // group in local memory)
+  const int bit = 5 * e;
 #pragma unroll
   for (int q = 0; q < 5; ++q) {
-    if (q == w) p[q] = (p[q] & ~(31u << sh)) | (code << sh);
-    if (q == w + 1 && sh > 27) {
-      const int hb = sh - 27;
-      p[q] = (p[q] & ~((1u << hb) - 1u)) | (code >> (5 - hb));
+    const int rel = bit - 32 * q;  // field position relative to word q
+    if (rel > -5 && rel < 32) {
+      const uint64_t m64 = rel >= 0 ? (31ull << rel) : (31ull >> -rel);
+      const uint64_t c64 = rel >= 0 ? (static_cast<uint64_t>(code) << rel) : (static_cast<uint64_t>(code) >> -rel);
+      p[q] = (p[q] & ~static_cast<uint32_t>(m64)) | static_cast<uint32_t>(c64);
     }
   }
 }
 
 template <bool kBf16, bool kVec>
-__global__ void __launch_bounds__(kQThreads, 4)
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
 quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const float* __restrict__ codebook,
                 uint8_t* __restrict__ packed, uint16_t* __restrict__ norms) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -268,7 +273,10 @@ quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const 
     int len = 0;
     const char* wblk = static_cast<const char*>(W);
     if (active) {
-      const int64_t o = F / nb;
+      // (row, block) of F; 32-bit division whenever the block count allows it
+      int64_t o;
+      if (nblocks <= 0xffffffffll) o = static_cast<uint32_t>(F) / static_cast<uint32_t>(nb);
+      else o = F / nb;
       const int b = static_cast<int>(F - o * nb);
       len = min(kBlock, in - kBlock * b);
       wblk += (o * static_cast<int64_t>(in) + static_cast<int64_t>(kBlock) * b) * kEsz;
@@ -431,7 +439,8 @@ dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict
     uint32_t w[5] = {0u, 0u, 0u, 0u, 0u};
     float scale = 0.0f;
     if (active) {
-      o = F / nb;
+      if (nblocks <= 0xffffffffll) o = static_cast<uint32_t>(F) / static_cast<uint32_t>(nb);
+      else o = F / nb;
       b = static_cast<int>(F - o * nb);
       len = min(kBlock, in - kBlock * b);
       const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + F * kBlockBytes + 20 * q);
@@ -498,7 +507,7 @@ int launch_quantize(const void* W, bool bf16, int64_t rows, int in, const float*
   const int nb = static_cast<int>(ceil_div(in, kBlock));
   const int64_t nblocks = rows * nb;
   const int64_t warps_needed = ceil_div(nblocks, 8);
-  const int64_t max_ctas = static_cast<int64_t>(sm_count()) * 4;
+  const int64_t max_ctas = static_cast<int64_t>(sm_count()) * kQCtasPerSm;  // persistent: one wave
   const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(warps_needed, kQThreads / 32)));
   const bool vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) &&
                    ((static_cast<int64_t>(in) * (bf16 ? 2 : 4)) % 16 == 0);
