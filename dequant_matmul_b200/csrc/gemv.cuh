@@ -98,9 +98,9 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 // (deterministic).
 //
 // Launched with programmatic stream serialisation (HLWQ_FLAG_WEIGHTS_STATIC),
-// the set-up -- first code boxes, codebook, pair table -- runs before
-// griddepcontrol.wait, i.e. while the previous kernel on the stream is still
-// finishing; x is read and y written only after it.
+// the set-up -- first code boxes (issued first), codebook, pair table -- runs
+// before griddepcontrol.wait, i.e. while the previous kernel on the stream is
+// still finishing; x is read and y written only after it.
 constexpr int kG1Threads = 512;
 constexpr int kG1Warps = kG1Threads / 32;
 constexpr int kG1ItemBytes = 32 * kBlockBytes;  // 2G rows x C blocks = 32 blocks for every C
@@ -357,7 +357,6 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     fence_barrier_init();
   }
   __syncwarp();
-  const uint32_t c16r = g1_codebook_lane(codebook);
   const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
   bool ok = true;
   uint32_t phase = 0;    // parity of the next completion, one bit per slot
@@ -400,14 +399,16 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       if (d < nw) issue(d);
 
     if (p0 == 0) {
-      // set-up while the first boxes are in flight: the first round of x
-      // loads is issued before the pair table is built, so its latency
-      // overlaps the table stores; the barrier below publishes both
+      // set-up while the first boxes are in flight: the codebook and the pair
+      // table depend on nothing the previous kernel writes, so they are built
+      // before the dependency wait (overlapping that kernel's last CTAs); then
+      // x is loaded and rotated; the barrier below publishes table and x
+      const uint32_t c16r = g1_codebook_lane(codebook);
+      g1_build_table(smem, c16r, 0, kG1Warps);
       pdl_wait();  // x may be produced by the previous kernel on the stream
       uint32_t xw[8];
       const int rb0 = 4 * warp;
       if (rb0 < nb) g1_rot_load(x, in, in, nb, nb, xvec != 0, rb0, xw);
-      g1_build_table(smem, c16r, 0, kG1Warps);
       if (rb0 < nb) g1_rot_store(xw, nb, nb, rb0, xs, xinv);
       for (int b0 = rb0 + 4 * kG1Warps; b0 < nb; b0 += 4 * kG1Warps) {
         g1_rot_load(x, in, in, nb, nb, xvec != 0, b0, xw);
