@@ -70,15 +70,16 @@ __host__ __device__ inline Moe1Layout moe1_layout(int S, int nvec, int nb, int p
   return L;
 }
 
-// Routes every token into rid / rw: pair t * KP + s holds the expert id (E =
-// the shared expert) and weight.  Warps 0 .. min(T, 15) - 1 route the tokens
-// (t = warp, warp + that count, ...); the other warps return at once.
-__device__ __forceinline__ void moe1_route(const Moe1Params& P, int* rid, float* rw, bool write_out) {
+// Routes tokens t_lo .. t_hi into rid / rw: pair t * KP + s holds the expert
+// id (E = the shared expert) and weight.  Warps 0 .. min(count, 15) - 1 route
+// (t = t_lo + warp, + that count, ...); the other warps return at once.
+__device__ __forceinline__ void moe1_route(const Moe1Params& P, int* rid, float* rw, bool write_out, int t_lo,
+                                           int t_hi) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KP = P.topk + P.has_shared;
-  const int nroute = min(P.T, kG1Warps - 1);
+  const int nroute = min(t_hi - t_lo + 1, kG1Warps - 1);
   if (warp >= nroute) return;
-  for (int t = warp; t < P.T; t += nroute) {
+  for (int t = t_lo + warp; t <= t_hi; t += nroute) {
     route_token_warp(P.logits + static_cast<int64_t>(t) * P.E, P.E, P.topk, rid + t * KP, rw + t * KP);
     if (lane == 0 && P.has_shared) {
       rid[t * KP + P.topk] = P.E;
@@ -113,7 +114,7 @@ __device__ __forceinline__ void moe1_load_x(const uint16_t* xs, const float* xin
 template <int C, int S>
 __global__ void __launch_bounds__(kG1Threads, 1)
 moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__ CUtensorMap smap, Moe1Params P,
-               int part_rows) {
+               int part_rows, int tok_max) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int L2C = 2 * C, G = 32 / L2C;
   const int nb = (P.H + kBlock - 1) / kBlock, nch = (nb + C - 1) / C;
@@ -124,7 +125,10 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
   const int q0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * nq_all / gridDim.x);
   const int q1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * nq_all / gridDim.x);
   const int nq = q1 - q0;
-  const Moe1Layout L = moe1_layout(S, P.T, nb, part_rows * nch * 2, NP);
+  // the tokens this CTA's pairs belong to (its range is contiguous in pairs)
+  const int t_lo = nq > 0 ? (q0 / ngj) / KP : 0, t_hi = nq > 0 ? ((q1 - 1) / ngj) / KP : 0;
+  const int ntok = t_hi - t_lo + 1;
+  const Moe1Layout L = moe1_layout(S, tok_max, nb, part_rows * nch * 2, NP);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
   float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
   float* part = reinterpret_cast<float*>(smem + L.part_off);  // [nq * G][nch][2] (gate, up)
@@ -146,12 +150,13 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
   }
   // the tokens' activations are loaded now and rotated once the boxes are on
   // their way; the routing warps run while the other warps build the table
-  const int nblk = P.T * nb;
+  const int nblk = ntok * nb;
+  const uint16_t* Xc = P.X + static_cast<int64_t>(t_lo) * P.H;
   const bool xvec = (reinterpret_cast<uintptr_t>(P.X) % 16 == 0) && (P.H % 8 == 0);
   uint32_t xw[8];
-  if (4 * warp < nblk) g1_rot_load(P.X, P.H, P.H, nb, nblk, xvec, 4 * warp, xw);
-  const int nroute = min(P.T, kG1Warps - 1);
-  moe1_route(P, rid, rw, blockIdx.x == 0);
+  if (4 * warp < nblk) g1_rot_load(Xc, P.H, P.H, nb, nblk, xvec, 4 * warp, xw);
+  const int nroute = min(ntok, kG1Warps - 1);
+  moe1_route(P, rid, rw, true, t_lo, t_hi);  // CTAs sharing a token write the same ids / weights
   g1_build_table(smem, c16r, nroute, kG1Warps - nroute);
   __syncthreads();  // routing, table, barriers
 
@@ -190,7 +195,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
 
   if (4 * warp < nblk) g1_rot_store(xw, nb, nblk, 4 * warp, xs, xinv);
   for (int gb0 = 4 * warp + 4 * kG1Warps; gb0 < nblk; gb0 += 4 * kG1Warps) {
-    g1_rot_load(P.X, P.H, P.H, nb, nblk, xvec, gb0, xw);
+    g1_rot_load(Xc, P.H, P.H, nb, nblk, xvec, gb0, xw);
     g1_rot_store(xw, nb, nblk, gb0, xs, xinv);
   }
   __syncthreads();
@@ -229,7 +234,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
         if (key != xkey) {
           xkey = key;
           const int b = cch * C + s;
-          moe1_load_x(xs, xinv, t * nb + b, b < nb, hh, xr, xi);
+          moe1_load_x(xs, xinv, (t - t_lo) * nb + b, b < nb, hh, xr, xi);
         }
         const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
                          (half_bits_to_float(static_cast<uint16_t>(nr)) * xi);
@@ -265,10 +270,13 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
 }
 
 // -------------------------------------------------------------------- down
+// The pairs are taken in groups of at most pg_max whose rotated h fit in
+// shared memory; every pair's partial sums stay in shared memory until the
+// fixed-order combine at the end.
 template <int C, int S>
 __global__ void __launch_bounds__(kG1Threads, 1)
 moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__ CUtensorMap smap, Moe1Params P,
-               int rows_max) {
+               int rows_max, int pg_max) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int L2C = 2 * C, G = 32 / L2C, RG = 2 * G;
   const int H = P.H, F = P.F;
@@ -278,7 +286,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
   const int g0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * ngr_all / gridDim.x);
   const int g1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * ngr_all / gridDim.x);
   const int ngr = g1 - g0, row0 = g0 * RG, nr = min(g1 * RG, H) - row0;
-  const Moe1Layout L = moe1_layout(S, NP, nb, NP * rows_max * nch, NP);
+  const Moe1Layout L = moe1_layout(S, pg_max, nb, NP * rows_max * nch, NP);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
   float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
   float* part = reinterpret_cast<float*>(smem + L.part_off);  // [NP][rows_max][nch]
@@ -301,106 +309,112 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
     fence_barrier_init();
   }
   const int nroute = min(P.T, kG1Warps - 1);
-  moe1_route(P, rid, rw, false);
+  moe1_route(P, rid, rw, false, 0, P.T - 1);
   g1_build_table(smem, c16r, nroute, kG1Warps - nroute);
   __syncthreads();  // routing, table, barriers
 
   const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
   bool ok = true;
   uint32_t phase = 0, pending = 0;
-  const int nitems = NP * nch * ngr;  // item k = (pair, chunk, row group), row group fastest
-  const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
-  const int nw = it1 - it0;
-  int ilg = it0 % ngr, ich = (it0 / ngr) % nch, ip = it0 / (ngr * nch);
-  uint32_t nraw[S];
-  auto issue = [&](int d) {
-    const int e = rid[ip];
-    const bool sh = e == P.E;
-    const int64_t rbase = sh ? 0 : static_cast<int64_t>(e) * H;
-    const int lrow = (g0 + ilg) * RG;  // first output row of the item
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
-      tma_load_3d(ring + d * kG1ItemBytes, sh ? &smap : &dmap, 0, ich * C, static_cast<int>(rbase + lrow),
-                  bar + 8 * d);
-    }
-    const int b = ich * C + s;
-    const uint16_t* nm = (sh ? P.sh_dn_norms : P.dn_norms) + (rbase + lrow + r) * nb + b;
-    const uint32_t n0 = (b < nb && lrow + r < H) ? static_cast<uint32_t>(__ldg(nm)) : 0u;
-    const uint32_t n1 = (b < nb && lrow + r + G < H) ? static_cast<uint32_t>(__ldg(nm + G * nb)) : 0u;
-    nraw[d] = n0 | (n1 << 16);
-    pending |= 1u << d;
-    if (++ilg == ngr) {
-      ilg = 0;
-      if (++ich == nch) { ich = 0; ++ip; }
-    }
-  };
+  for (int pg0 = 0; pg0 < NP; pg0 += pg_max) {
+    const int npg = min(pg_max, NP - pg0);
+    const int nitems = npg * nch * ngr;  // item k = (pair, chunk, row group), row group fastest
+    const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
+    const int nw = it1 - it0;
+    int ilg = it0 % ngr, ich = (it0 / ngr) % nch, ip = pg0 + it0 / (ngr * nch);
+    uint32_t nraw[S];
+    auto issue = [&](int d) {
+      const int e = rid[ip];
+      const bool sh = e == P.E;
+      const int64_t rbase = sh ? 0 : static_cast<int64_t>(e) * H;
+      const int lrow = (g0 + ilg) * RG;  // first output row of the item
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
+        tma_load_3d(ring + d * kG1ItemBytes, sh ? &smap : &dmap, 0, ich * C, static_cast<int>(rbase + lrow),
+                    bar + 8 * d);
+      }
+      const int b = ich * C + s;
+      const uint16_t* nm = (sh ? P.sh_dn_norms : P.dn_norms) + (rbase + lrow + r) * nb + b;
+      const uint32_t n0 = (b < nb && lrow + r < H) ? static_cast<uint32_t>(__ldg(nm)) : 0u;
+      const uint32_t n1 = (b < nb && lrow + r + G < H) ? static_cast<uint32_t>(__ldg(nm + G * nb)) : 0u;
+      nraw[d] = n0 | (n1 << 16);
+      pending |= 1u << d;
+      if (++ilg == ngr) {
+        ilg = 0;
+        if (++ich == nch) { ich = 0; ++ip; }
+      }
+    };
+    if (lane == 0) fence_proxy_async();  // the previous group's reads of the slots precede the refills
 #pragma unroll
-  for (int d = 0; d < S; ++d)
-    if (d < nw) issue(d);
+    for (int d = 0; d < S; ++d)
+      if (ok && d < nw) issue(d);
 
-  pdl_wait();  // h is written by the gate_up kernel
-  const int nblk = NP * nb;
-  for (int gb0 = 4 * warp; gb0 < nblk; gb0 += 4 * kG1Warps) g1_rot_f32(P.h, F, F, nb, nblk, gb0, xs, xinv);
-  __syncthreads();
-  pdl_trigger();
+    if (pg0 == 0) pdl_wait();  // h is written by the gate_up kernel
+    const int nblk = npg * nb;
+    for (int gb0 = 4 * warp; gb0 < nblk; gb0 += 4 * kG1Warps)
+      g1_rot_f32(P.h + static_cast<int64_t>(pg0) * F, F, F, nb, nblk, gb0, xs, xinv);
+    __syncthreads();
+    if (pg0 == 0) pdl_trigger();
 
-  int clg = it0 % ngr, cch = (it0 / ngr) % nch, cp = it0 / (ngr * nch), xkey = -1;
-  uint32_t xr[32];
-  float xi = 0.0f;
-  for (int base = 0; base < nw; base += S) {
+    int clg = it0 % ngr, cch = (it0 / ngr) % nch, cp = pg0 + it0 / (ngr * nch), xkey = -1;
+    uint32_t xr[32];
+    float xi = 0.0f;
+    for (int base = 0; base < nw; base += S) {
 #pragma unroll
-    for (int d = 0; d < S; ++d) {
-      const int k = base + d;
-      if (k < nw) {
-        const uint32_t nr2 = nraw[d];
-        if (ok && ((pending >> d) & 1u)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
-          if (ok) {
-            phase ^= 1u << d;
-            pending &= ~(1u << d);
+      for (int d = 0; d < S; ++d) {
+        const int k = base + d;
+        if (k < nw) {
+          const uint32_t nr2 = nraw[d];
+          if (ok && ((pending >> d) & 1u)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
+            if (ok) {
+              phase ^= 1u << d;
+              pending &= ~(1u << d);
+            }
           }
-        }
-        uint2 cw0[5], cw1[5];
-        const uint2* src = reinterpret_cast<const uint2*>(my_codes + d * kG1ItemBytes);
+          uint2 cw0[5], cw1[5];
+          const uint2* src = reinterpret_cast<const uint2*>(my_codes + d * kG1ItemBytes);
 #pragma unroll
-        for (int q = 0; q < 5; ++q) {
-          cw0[q] = src[q];
-          cw1[q] = src[q + kG1ItemBytes / 16];
-        }
-        __syncwarp();
-        if (ok && k + S < nw) {
-          if (lane == 0) fence_proxy_async();
-          issue(d);
-        }
-        const int key = cp * nch + cch;
-        if (key != xkey) {
-          xkey = key;
-          const int b = cch * C + s;
-          moe1_load_x(xs, xinv, cp * nb + b, b < nb, hh, xr, xi);
-        }
-        const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                         (half_bits_to_float(static_cast<uint16_t>(nr2)) * xi);
-        const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                         (half_bits_to_float(static_cast<uint16_t>(nr2 >> 16)) * xi);
-        const bool hi = (u & C) != 0;
-        float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
+          for (int q = 0; q < 5; ++q) {
+            cw0[q] = src[q];
+            cw1[q] = src[q + kG1ItemBytes / 16];
+          }
+          __syncwarp();
+          if (ok && k + S < nw) {
+            if (lane == 0) fence_proxy_async();
+            issue(d);
+          }
+          const int key = cp * nch + cch;
+          if (key != xkey) {
+            xkey = key;
+            const int b = cch * C + s;
+            moe1_load_x(xs, xinv, (cp - pg0) * nb + b, b < nb, hh, xr, xi);
+          }
+          const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+                           (half_bits_to_float(static_cast<uint16_t>(nr2)) * xi);
+          const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+                           (half_bits_to_float(static_cast<uint16_t>(nr2 >> 16)) * xi);
+          const bool hi = (u & C) != 0;
+          float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
 #pragma unroll
-        for (int off = C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if ((u & (C - 1)) == 0) part[(cp * rows_max + clg * RG + r + (hi ? G : 0)) * nch + cch] = acc;
-        if (++clg == ngr) {
-          clg = 0;
-          if (++cch == nch) { cch = 0; ++cp; }
+          for (int off = C / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+          if ((u & (C - 1)) == 0) part[(cp * rows_max + clg * RG + r + (hi ? G : 0)) * nch + cch] = acc;
+          if (++clg == ngr) {
+            clg = 0;
+            if (++cch == nch) { cch = 0; ++cp; }
+          }
         }
       }
     }
+    if (!ok) {
+      const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
+      for (int d = 0; d < S; ++d)
+        if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
+      pending = 0;
+      if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
+    }
+    __syncthreads();  // the next group overwrites the rotated h
   }
-  if (!ok) {
-    const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
-    for (int d = 0; d < S; ++d)
-      if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
-    if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
-  }
-  __syncthreads();
   for (int idx = threadIdx.x; idx < P.T * nr; idx += kG1Threads) {
     const int t = idx / nr, i = idx - t * nr;
     float y = 0.0f;
@@ -426,19 +440,19 @@ bool moe1_attr(K kernel) {
 
 template <int C, int S>
 int moe1_launch_gu(const CUtensorMap& gm, const CUtensorMap& sm, const Moe1Params& P, int grid, int part_rows,
-                   int smem, cudaStream_t stream) {
+                   int tok_max, int smem, cudaStream_t stream) {
   static bool attr = false;
   if (!attr) {
     if (!moe1_attr(moe_gu1_kernel<C, S>)) return HLWQ_ECUDA;
     attr = true;
   }
-  moe_gu1_kernel<C, S><<<grid, kG1Threads, smem, stream>>>(gm, sm, P, part_rows);
+  moe_gu1_kernel<C, S><<<grid, kG1Threads, smem, stream>>>(gm, sm, P, part_rows, tok_max);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
 
 template <int C, int S>
 int moe1_launch_dn(const CUtensorMap& dm, const CUtensorMap& sm, const Moe1Params& P, int grid, int rows_max,
-                   int smem, cudaStream_t stream) {
+                   int pg_max, int smem, cudaStream_t stream) {
   static bool attr = false;
   if (!attr) {
     if (!moe1_attr(moe_dn1_kernel<C, S>)) return HLWQ_ECUDA;
@@ -454,21 +468,22 @@ int moe1_launch_dn(const CUtensorMap& dm, const CUtensorMap& sm, const Moe1Param
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_dn1_kernel<C, S>, dm, sm, P, rows_max) == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+  return cudaLaunchKernelEx(&cfg, moe_dn1_kernel<C, S>, dm, sm, P, rows_max, pg_max) == cudaSuccess ? HLWQ_OK
+                                                                                              : HLWQ_ECUDA;
 }
 
 template <int C>
 int moe1_gu_c(int S, const CUtensorMap& gm, const CUtensorMap& sm, const Moe1Params& P, int grid, int part_rows,
-              int smem, cudaStream_t stream) {
-  return S == 2 ? moe1_launch_gu<C, 2>(gm, sm, P, grid, part_rows, smem, stream)
-                : moe1_launch_gu<C, 1>(gm, sm, P, grid, part_rows, smem, stream);
+              int tok_max, int smem, cudaStream_t stream) {
+  return S == 2 ? moe1_launch_gu<C, 2>(gm, sm, P, grid, part_rows, tok_max, smem, stream)
+                : moe1_launch_gu<C, 1>(gm, sm, P, grid, part_rows, tok_max, smem, stream);
 }
 
 template <int C>
 int moe1_dn_c(int S, const CUtensorMap& dm, const CUtensorMap& sm, const Moe1Params& P, int grid, int rows_max,
-              int smem, cudaStream_t stream) {
-  return S == 2 ? moe1_launch_dn<C, 2>(dm, sm, P, grid, rows_max, smem, stream)
-                : moe1_launch_dn<C, 1>(dm, sm, P, grid, rows_max, smem, stream);
+              int pg_max, int smem, cudaStream_t stream) {
+  return S == 2 ? moe1_launch_dn<C, 2>(dm, sm, P, grid, rows_max, pg_max, smem, stream)
+                : moe1_launch_dn<C, 1>(dm, sm, P, grid, rows_max, pg_max, smem, stream);
 }
 
 }  // namespace
@@ -488,22 +503,33 @@ int launch_moe1(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_
   const int nchg = (nbh + cg - 1) / cg, nchd = (nbf + cd - 1) / cd;
   const int sms = sm_count();
   // gate_up: groups of Gg columns per pair
-  const int64_t nq_all = static_cast<int64_t>(NP) * ceil_div(F, Gg);
+  const int64_t ngj = ceil_div(F, Gg);
+  const int64_t nq_all = static_cast<int64_t>(NP) * ngj;
   const int grid_g = static_cast<int>(std::min<int64_t>(sms, nq_all));
-  const int part_rows = static_cast<int>(ceil_div(nq_all, grid_g)) * Gg;
+  const int64_t nq_max = ceil_div(nq_all, grid_g);
+  const int part_rows = static_cast<int>(nq_max) * Gg;
+  // tokens one CTA's contiguous range of pairs can touch
+  const int tok_max = static_cast<int>(std::min<int64_t>(T, (ceil_div(nq_max, ngj) + 1 + KP - 1) / KP + 1));
   int Sg = 0, smem_g = 0;
   for (int S : {2, 1}) {
-    const int t = moe1_layout(S, T, nbh, part_rows * nchg * 2, NP).total;
+    const int t = moe1_layout(S, tok_max, nbh, part_rows * nchg * 2, NP).total;
     if (t <= 227 * 1024) { Sg = S; smem_g = t; break; }
   }
   // down: groups of RGd output rows, all pairs
   const int64_t ngr_all = ceil_div(H, RGd);
   const int grid_d = static_cast<int>(std::min<int64_t>(sms, ngr_all));
   const int rows_max = static_cast<int>(ceil_div(ngr_all, grid_d)) * RGd;
-  int Sd = 0, smem_d = 0;
+  // pairs per group: as many rotated h as fit beside the ring and all partials
+  int Sd = 0, smem_d = 0, pg_max = 0;
   for (int S : {2, 1}) {
-    const int t = moe1_layout(S, NP, nbf, NP * rows_max * nchd, NP).total;
-    if (t <= 227 * 1024) { Sd = S; smem_d = t; break; }
+    int pg = NP;
+    while (pg > 0 && moe1_layout(S, pg, nbf, NP * rows_max * nchd, NP).total > 227 * 1024) pg = pg > 8 ? pg * 3 / 4 : pg - 1;
+    if (pg > 0 && (pg >= std::min(NP, KP) || S == 1)) {
+      Sd = S;
+      pg_max = pg;
+      smem_d = moe1_layout(S, pg, nbf, NP * rows_max * nchd, NP).total;
+      break;
+    }
   }
   if (!Sg || !Sd) return HLWQ_EUNSUPPORTED;
 
@@ -537,15 +563,15 @@ int launch_moe1(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_
   P.has_shared = shared ? 1 : 0;
   P.out_bf16 = out_bf16 ? 1 : 0;
   switch (cg) {
-    case 8: st = moe1_gu_c<8>(Sg, gm, gsm, P, grid_g, part_rows, smem_g, stream); break;
-    case 4: st = moe1_gu_c<4>(Sg, gm, gsm, P, grid_g, part_rows, smem_g, stream); break;
-    default: st = moe1_gu_c<2>(Sg, gm, gsm, P, grid_g, part_rows, smem_g, stream); break;
+    case 8: st = moe1_gu_c<8>(Sg, gm, gsm, P, grid_g, part_rows, tok_max, smem_g, stream); break;
+    case 4: st = moe1_gu_c<4>(Sg, gm, gsm, P, grid_g, part_rows, tok_max, smem_g, stream); break;
+    default: st = moe1_gu_c<2>(Sg, gm, gsm, P, grid_g, part_rows, tok_max, smem_g, stream); break;
   }
   if (st != HLWQ_OK) return st;
   switch (cd) {
-    case 8: return moe1_dn_c<8>(Sd, dm, dsm, P, grid_d, rows_max, smem_d, stream);
-    case 4: return moe1_dn_c<4>(Sd, dm, dsm, P, grid_d, rows_max, smem_d, stream);
-    default: return moe1_dn_c<2>(Sd, dm, dsm, P, grid_d, rows_max, smem_d, stream);
+    case 8: return moe1_dn_c<8>(Sd, dm, dsm, P, grid_d, rows_max, pg_max, smem_d, stream);
+    case 4: return moe1_dn_c<4>(Sd, dm, dsm, P, grid_d, rows_max, pg_max, smem_d, stream);
+    default: return moe1_dn_c<2>(Sd, dm, dsm, P, grid_d, rows_max, pg_max, smem_d, stream);
   }
 }
 
