@@ -105,7 +105,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n) {
 }
 
 // Shared address of the fp32 centroid of the code at bit POS of a half block
-// (10 words): the 5-bit field moved to bit 2 with one shift and masked.
+// (10 words): the 5-bit field moved to bit 2 with one shift, masked and or-ed
+// with the (1024-byte aligned) table address.
 // (pos is a compile-time constant after unrolling.)
 __device__ __forceinline__ uint32_t code_addr(const uint2 (&cw)[5], int pos, uint32_t tab) {
   const int wi = pos >> 5, sh = pos & 31;
@@ -118,7 +119,7 @@ __device__ __forceinline__ uint32_t code_addr(const uint2 (&cw)[5], int pos, uin
   } else {
     t = lo << (2 - sh);
   }
-  return (t & 0x7cu) + tab;
+  return (t & 0x7cu) | tab;  // tab is 1024-byte aligned: or == add, one and-or instruction
 }
 
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
