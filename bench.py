@@ -283,6 +283,34 @@ def bench_moe(hl, cb, peaks, stream, scrub):
         moe[f"T{T}"] = {"ms": round(ms, 4), "distinct_experts": distinct, "gbs": round(byts / ms / 1e6, 1),
                         "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
     out["moe_256x(1024x2048+2048x512)_top8_shared"] = moe
+    del gu, dn, sh
+    # MoE: the 128-expert layer, hidden 2816, intermediate 704 (tail block
+    # zero-padded), top-8, no shared expert, T = 1 and 16.
+    E5, H5, F5 = 128, 2816, 704
+    gu5 = hl.quantize(synth.student_t_device((E5, 2 * F5, H5), seed=90), cb, stream=stream)
+    dn5 = hl.quantize(synth.student_t_device((E5, H5, F5), seed=91), cb, stream=stream)
+    per_expert5 = (2 * F5 * 22 + H5 * 6) * 82
+    moe5 = {}
+    for T in (1, 16):
+        logits = torch.randn(T, E5, generator=torch.Generator(device="cuda").manual_seed(100 + T), device="cuda")
+        X = synth.activations_device(T, H5, seed=110 + T)
+        Y = torch.empty(T, H5, dtype=torch.float32, device="cuda")
+        ids = torch.empty(T, 8, dtype=torch.int32, device="cuda")
+        wts = torch.empty(T, 8, dtype=torch.float32, device="cuda")
+        ws = torch.empty(hl.workspace_bytes(hl.HLWQ_OP_MOE, H5, F5, T, E5, 8), dtype=torch.uint8, device="cuda")
+
+        def run_moe5():
+            flush_l2(scrub)
+            hl.moe_gemv(gu5, dn5, cb, logits, X, 8, Y=Y, ids=ids, weights=wts, workspace=ws, stream=stream)
+
+        ms_all, _ = time_graph(run_moe5, reps=20, warmup=3, stream=stream)
+        ms_flush, _ = time_graph(lambda: flush_l2(scrub), reps=20, warmup=3, stream=stream)
+        ms = max(ms_all - ms_flush, 1e-6)
+        distinct = int(torch.unique(ids).numel())
+        byts = distinct * per_expert5
+        moe5[f"T{T}"] = {"ms": round(ms, 4), "distinct_experts": distinct, "gbs": round(byts / ms / 1e6, 1),
+                         "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
+    out["moe_128x(1408x2816+2816x704)_top8"] = moe5
     return out
 
 

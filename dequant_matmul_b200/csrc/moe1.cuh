@@ -505,15 +505,20 @@ int launch_moe1(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_
   // gate_up: groups of Gg columns per pair
   const int64_t ngj = ceil_div(F, Gg);
   const int64_t nq_all = static_cast<int64_t>(NP) * ngj;
-  const int grid_g = static_cast<int>(std::min<int64_t>(sms, nq_all));
-  const int64_t nq_max = ceil_div(nq_all, grid_g);
-  const int part_rows = static_cast<int>(nq_max) * Gg;
-  // tokens one CTA's contiguous range of pairs can touch
-  const int tok_max = static_cast<int>(std::min<int64_t>(T, (ceil_div(nq_max, ngj) + 1 + KP - 1) / KP + 1));
-  int Sg = 0, smem_g = 0;
-  for (int S : {2, 1}) {
-    const int t = moe1_layout(S, tok_max, nbh, part_rows * nchg * 2, NP).total;
-    if (t <= 227 * 1024) { Sg = S; smem_g = t; break; }
+  // one CTA per SM when its partial sums fit; otherwise more CTAs (in waves),
+  // each with a shorter range of column groups
+  int grid_g = 0, part_rows = 0, tok_max = 0, Sg = 0, smem_g = 0;
+  for (int waves = 1; waves <= 4 && !Sg; ++waves) {
+    grid_g = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(sms) * waves, nq_all));
+    const int64_t nq_max = ceil_div(nq_all, grid_g);
+    part_rows = static_cast<int>(nq_max) * Gg;
+    // tokens one CTA's contiguous range of pairs can touch
+    tok_max = static_cast<int>(std::min<int64_t>(T, (ceil_div(nq_max, ngj) + 1 + KP - 1) / KP + 1));
+    for (int S : {2, 1}) {
+      const int t = moe1_layout(S, tok_max, nbh, part_rows * nchg * 2, NP).total;
+      if (t <= 227 * 1024) { Sg = S; smem_g = t; break; }
+    }
+    if (grid_g == nq_all) break;
   }
   // down: groups of RGd output rows, all pairs
   const int64_t ngr_all = ceil_div(H, RGd);

@@ -121,3 +121,33 @@ def test_moe_full_t64_sampled_tokens(hl, cb):
         want, _, _ = O.moe_forward(gu_o, dn_o, H, F, k, logits[t:t + 1], X[t:t + 1],
                                    (qsg["packed"], qsg["norms"]), (qsd["packed"], qsd["norms"]))
         assert rel_l2(Y[t].cpu().numpy(), want[0]) <= MATMUL_REL
+
+
+def test_moe_128_experts_full_t16_sampled_tokens(hl, cb):
+    """The 128-expert layer (hidden 2816, intermediate 704, no shared expert)
+    at T = 16: the gate_up kernel's partial sums need two waves of CTAs and the
+    down kernel takes the 128 pairs in groups.  The oracle encodes and
+    evaluates the experts of three sampled tokens itself."""
+    E, H, F, T, k = 128, 2816, 704, 16, 8
+    seed = 600
+    logits = synth.router_logits(T, E, seed=seed)
+    X = synth.activations(T, H, seed=seed + 1)
+    gu_w = torch.empty(E, 2 * F, H, dtype=torch.bfloat16, device="cuda")
+    dn_w = torch.empty(E, H, F, dtype=torch.bfloat16, device="cuda")
+    for e in range(E):
+        gu_w[e] = synth.student_t((2 * F, H), df4_seed=seed + 10 + 2 * e).cuda()
+        dn_w[e] = synth.student_t((H, F), df4_seed=seed + 11 + 2 * e).cuda()
+    gu = hl.quantize(gu_w, cb)
+    dn = hl.quantize(dn_w, cb)
+    for odt in (torch.float32, torch.bfloat16):
+        Y, ids, w = hl.moe_gemv(gu, dn, cb, logits.cuda(), X.cuda(), k, out_dtype=odt)
+        torch.cuda.synchronize()
+        ids_o, w_o = O.router_topk(logits, k)
+        assert np.array_equal(ids.cpu().numpy(), ids_o)
+        assert np.allclose(w.cpu().numpy(), w_o, rtol=1e-5, atol=1e-7)
+        for t in (0, 7, 15):
+            sel = ids_o[t]
+            gu_o = {int(e): (lambda q: (q["packed"], q["norms"]))(O.quantize(gu_w[int(e)].cpu())) for e in sel}
+            dn_o = {int(e): (lambda q: (q["packed"], q["norms"]))(O.quantize(dn_w[int(e)].cpu())) for e in sel}
+            want, _, _ = O.moe_forward(gu_o, dn_o, H, F, k, logits[t:t + 1], X[t:t + 1], None, None)
+            assert rel_l2(Y[t].double().cpu().numpy(), want[0]) <= MATMUL_REL, (odt, t)
