@@ -39,7 +39,7 @@ bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Threshold between the CUDA-core decode path and the tensor-core path.
-constexpr int64_t kTensorCoreMinM = 16;
+constexpr int64_t kTensorCoreMinM = 5;  // M = 2..4: the multi-token CUDA-core kernel; M >= 5: tcgen05
 
 }  // namespace
 

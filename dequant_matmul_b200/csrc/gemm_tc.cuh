@@ -1,7 +1,7 @@
 #pragma once
 // Small-M GEMM on the 5th-generation tensor cores (tcgen05 / TMEM / TMA), sm_100a.
 //
-// Y[m][o] = sum_i X[m][i] w_hat[o][i] for M >= 16 tokens, evaluated in the
+// Y[m][o] = sum_i X[m][i] w_hat[o][i] for M >= 5 tokens, evaluated in the
 // rotated domain ("Qwen3.6-35B-A3B -- HLWQ Q5", Method step [3]; H symmetric,
 // H H = 128 I):
 //     Y[m][o] = 2^e_o / (128 s_m) * sum_K A[o][K] B[m][K],

@@ -260,10 +260,10 @@ __device__ __forceinline__ void g1_rot_load(const uint16_t* __restrict__ x, int6
   }
 }
 
-__device__ __forceinline__ void g1_rot_core(float (&v)[16], int nb, int nblocks, int gb0, uint16_t* xs,
-                                            float* xinv) {
-  const int lane = threadIdx.x & 31, q = lane & 7;
-  const RotBlock B = g1_rot_block(nb, nblocks, gb0);
+// Butterflies of one block held 16 values per lane by 8 lanes; returns the
+// power-of-two exponent k with max |x_tilde| * 2^k in [2^9, 2^10).
+__device__ __forceinline__ int g1_rot_compute(float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
@@ -287,7 +287,14 @@ __device__ __forceinline__ void g1_rot_core(float (&v)[16], int nb, int nblocks,
   for (int lm = 1; lm < 8; lm <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lm));
   int ex = 0;
   if (mx > 0.0f && isfinite(mx)) frexpf(mx, &ex);
-  const int k = max(-120, min(120, 10 - ex));
+  return max(-120, min(120, 10 - ex));
+}
+
+__device__ __forceinline__ void g1_rot_core(float (&v)[16], int nb, int nblocks, int gb0, uint16_t* xs,
+                                            float* xinv) {
+  const int q = threadIdx.x & 7;
+  const RotBlock B = g1_rot_block(nb, nblocks, gb0);
+  const int k = g1_rot_compute(v);
   const float sc = ldexpf(1.0f, k);
   if (B.act) {
     uint4* dst = reinterpret_cast<uint4*>(xs);
@@ -686,10 +693,19 @@ int launch_dense_m1(const uint8_t* packed, const uint16_t* norms, const float* c
   }
 }
 
+int launch_gemvm(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                 const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
+
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
   if (M == 1) return launch_gemv1(packed, norms, codebook, O, in, X, Y, out_bf16, stream, 0u);
+  if (M <= 8) {
+    // few tokens: the TMA-fed multi-token kernel (falls through when its
+    // shared memory does not fit, e.g. very long rows)
+    const int st = launch_gemvm(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
+    if (st != HLWQ_EUNSUPPORTED) return st;
+  }
   int mt = M >= 3 ? 4 : M;
   while (mt > 1 && dense_smem_bytes(O, in, mt) > 227 * 1024) mt >>= 1;
   switch (pick_chunk(nb)) {

@@ -2,6 +2,7 @@
 // and are compiled together (no relocatable device code needed).
 #include "quantize.cuh"
 #include "gemv.cuh"
+#include "gemvm.cuh"
 #include "moe.cuh"
 #include "moe1.cuh"
 #include "gemm_tc.cuh"

@@ -140,7 +140,8 @@ int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const float* code
  *   X  device bf16 [M][ldx] (ldx >= in, ldx % 8 == 0)
  *   Y  device ydtype [M][ldy] (ldy >= out)
  *   workspace  device, ws_bytes >= hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
- * M < 16 runs on the CUDA-core decode path; M >= 16 on the tensor-core path.
+ * M = 1..4 runs on the CUDA-core decode path (one launch streams the weights for
+ * up to four tokens); M >= 5 on the tensor-core path (workspace needed).
  */
 int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook,
               int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx,

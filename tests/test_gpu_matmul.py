@@ -145,20 +145,27 @@ def test_gemm_small_m(hl, cb, M):
     assert rel_l2(Y.double().cpu().numpy(), want) <= MATMUL_REL
 
 
-def test_gemm_ragged_fp32_out_and_pitch(hl, cb):
+@pytest.mark.parametrize("M", [3, 6])
+def test_gemm_ragged_fp32_out_and_pitch(hl, cb, M):
+    """Row pitches larger than the rows (X: 720 > 704, Y: 208 > 200) on the
+    multi-token CUDA-core path (M = 3) and the tensor-core path (M = 6, with
+    the workspace hlwq_workspace_bytes reports); the pitch padding of Y stays
+    untouched."""
     W, q = _layer((200, 704), seed=5)
     p, n = oracle_to_dev(q)
-    X = synth.activations(6, 720, seed=6)[:, :704]        # row pitch 720 > in
+    X = synth.activations(M, 720, seed=6)[:, :704]        # row pitch 720 > in
     Xd = X.cuda()
-    Y = torch.full((6, 208), 7.0, device="cuda")          # row pitch 208 > out
-    hl.gemm(p, n, cb, Xd, Y=Y[:, :200].contiguous(), out_dtype=torch.float32)  # contiguous path
-    Y2 = torch.full((6, 208), 7.0, device="cuda")
-    hl.lib.hlwq_gemm(p.data_ptr(), n.data_ptr(), cb.data_ptr(), 200, 704, 6, Xd.data_ptr(), Xd.stride(0),
-                     Y2.data_ptr(), 208, hl.HLWQ_F32, None, 0, torch.cuda.current_stream().cuda_stream)
+    Y = torch.full((M, 208), 7.0, device="cuda")          # row pitch 208 > out
+    need = hl.workspace_bytes(hl.HLWQ_OP_GEMM, 200, 704, M)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    st = hl.lib.hlwq_gemm(p.data_ptr(), n.data_ptr(), cb.data_ptr(), 200, 704, M, Xd.data_ptr(), Xd.stride(0),
+                          Y.data_ptr(), 208, hl.HLWQ_F32, ws.data_ptr() if need else None, need,
+                          torch.cuda.current_stream().cuda_stream)
+    assert st == hl.HLWQ_OK
     torch.cuda.synchronize()
     want = O.matmul(q["packed"], q["norms"], 704, X)
-    assert rel_l2(Y2[:, :200].cpu().numpy(), want) <= MATMUL_REL
-    assert torch.all(Y2[:, 200:] == 7.0)
+    assert rel_l2(Y[:, :200].cpu().numpy(), want) <= MATMUL_REL
+    assert torch.all(Y[:, 200:] == 7.0)
 
 
 def test_gemm_m1_equals_gemv(hl, cb):
@@ -190,7 +197,7 @@ def test_gemv_full_27648x5120_sampled_rows(hl, cb):
 @pytest.mark.parametrize("O,I,M", [(200, 704, 16), (384, 1024, 17), (256, 5120, 256), (130, 256, 48),
                                    (1024, 5120, 200), (128, 128, 300)])
 def test_gemm_tensor_core_shapes(hl, cb, O, I, M):
-    """M >= 16 runs on the tcgen05 path: partial 128-row tile, ragged K (704 =
+    """M >= 5 runs on the tcgen05 path: partial 128-row tile, ragged K (704 =
     5.5 blocks), M not a multiple of 16, M = 256, and M > 256 (two token tiles)."""
     W, q = _layer((O, I), seed=O + I + M)
     p, n = oracle_to_dev(q)
