@@ -164,6 +164,24 @@ def frac(a, p):
     return round(a / p, 4) if (a is not None and p) else None
 
 
+# ---------------------------------------------------------------- ranks (N > 1: independent replicas)
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """The largest of the ranks' values (every rank gets it); the timed region
+    of a multi-GPU run is the slowest rank's."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: int, steps: int, ms_total_max: float) -> float:
+    """Whole-job throughput: the bytes all ranks processed / the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (ms_total_max * 1e6)
+
+
 # ---------------------------------------------------------------- components (N = 1)
 def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe")):
     import torch
@@ -441,13 +459,9 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(end)
-    t = torch.tensor([ms_total], device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
     ms_step = ms_total / args.steps
-    value = world * LAYERS * WEIGHT_BYTES * args.steps / (ms_total * 1e6)
+    value = whole_job_gbs(world, LAYERS * WEIGHT_BYTES, args.steps, ms_total)
     launch_ms = ms_step / LAYERS
     achieved = GEMV_ALGO_BYTES / launch_ms / 1e6
 
@@ -472,10 +486,7 @@ def main():
             e2e_step()
         e2.record(stream)
         e2.synchronize()
-    te = torch.tensor([s2.elapsed_time(e2)], device="cuda")
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_val = world * LAYERS * WEIGHT_BYTES * e2e_steps / (float(te.item()) * 1e6)
+    e2e_val = whole_job_gbs(world, LAYERS * WEIGHT_BYTES, e2e_steps, max_over_ranks(s2.elapsed_time(e2), world, "cuda"))
 
     comp = None
     if world == 1 and not args.no_components:
