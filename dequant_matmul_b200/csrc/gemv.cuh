@@ -98,9 +98,10 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 // (deterministic).
 //
 // Launched with programmatic stream serialisation (HLWQ_FLAG_WEIGHTS_STATIC),
-// the set-up -- first code boxes (issued first), codebook, pair table -- runs
-// before griddepcontrol.wait, i.e. while the previous kernel on the stream is
-// still finishing; x is read and y written only after it.
+// the first code boxes and their norms (issued first) and the codebook load do
+// not wait for the previous kernel on the stream (griddepcontrol.wait); x is
+// read and y written only after that wait, and the pair table is built while
+// the x loads are in flight.
 constexpr int kG1Threads = 512;
 constexpr int kG1Warps = kG1Threads / 32;
 constexpr int kG1ItemBytes = 32 * kBlockBytes;  // 2G rows x C blocks = 32 blocks for every C
@@ -189,29 +190,38 @@ __device__ __forceinline__ float g1_dot(const uint8_t* tab, const uint2 (&cw)[5]
   return g1_dot_n<4>(tab, cw, lane4, xr, seq);
 }
 
-// Lane l's centroid c[l] as binary16 (warp 0 also checks that the codebook is
-// strictly ascending and raises HLWQ_DEVERR_CODEBOOK otherwise).
-__device__ __forceinline__ uint32_t g1_codebook_lane(const float* __restrict__ codebook) {
+// Lane l's centroid c = c[l] as binary16 (a warp with `check` set, warp 0 in
+// g1_codebook_lane, also checks that the codebook is strictly ascending and
+// raises HLWQ_DEVERR_CODEBOOK otherwise).
+__device__ __forceinline__ uint32_t g1_codebook_half(float c, bool check) {
   const int lane = threadIdx.x & 31;
-  const float c = __ldg(codebook + lane);
-  if (threadIdx.x < 32) {
+  if (check) {
     const float next = __shfl_down_sync(0xffffffffu, c, 1);
     if (lane + 1 < kLevels && !(c < next)) raise_device_error(HLWQ_DEVERR_CODEBOOK);
   }
   return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(c)));
 }
 
+__device__ __forceinline__ uint32_t g1_codebook_lane(const float* __restrict__ codebook) {
+  return g1_codebook_half(__ldg(codebook + (threadIdx.x & 31)), threadIdx.x < 32);
+}
+
 // Warps [w0, w0 + nw) write the lane-replicated pair table, word (v * 32 +
 // lane) = half2(c[v & 31], c[v >> 5]), from the centroids in their lanes (no
 // shared copy of the codebook, so no CTA barrier before the table is built).
+// One 16-byte store per lane covers four entries (lane l: entry 4m + l / 8,
+// words 4 (l & 7) .. + 3), so the low halves c[4 (m & 7) + l / 8] repeat with
+// period 8 in m and are shuffled once when the warp count is a multiple of 8.
 __device__ __forceinline__ void g1_build_table(uint8_t* smem, uint32_t c16r, int w0, int nw) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp < w0 || warp >= w0 + nw) return;
   uint4* t4 = reinterpret_cast<uint4*>(smem);
-  for (int q = (warp - w0) * 32 + lane; q < 1024 * 8; q += nw * 32) {  // same trip count on every lane
-    const int v = q >> 3;
-    const uint32_t e = __shfl_sync(0xffffffffu, c16r, v & 31) | (__shfl_sync(0xffffffffu, c16r, v >> 5) << 16);
-    t4[q] = make_uint4(e, e, e, e);
+  const int k = warp - w0;
+  uint32_t lo = __shfl_sync(0xffffffffu, c16r, 4 * (k & 7) + (lane >> 3));
+  for (int m = k; m < 256; m += nw) {
+    if (nw & 7) lo = __shfl_sync(0xffffffffu, c16r, 4 * (m & 7) + (lane >> 3));
+    const uint32_t e = lo | (__shfl_sync(0xffffffffu, c16r, m >> 3) << 16);
+    t4[m * 32 + lane] = make_uint4(e, e, e, e);
   }
 }
 
@@ -381,7 +391,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     // points at the norm of (row ig * RG + r, block ich * C + s)
     int ich = it0 / ngr, ig = it0 - (it0 / ngr) * ngr;
     const uint16_t* nptr = norms + (prow0 + ig * RG + r) * nb + ich * C + s;
-    uint32_t nraw[S];
+    uint32_t nlo[S], nhi[S];  // the two rows' norms, kept apart so that no instruction waits on them before use
     auto issue = [&](int d) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
@@ -389,9 +399,12 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       }
       const int v = ig * RG + r;
       const bool bok = ich * C + s < nb;
-      const uint32_t n0 = (bok && v < prow) ? static_cast<uint32_t>(__ldg(nptr)) : 0u;
-      const uint32_t n1 = (bok && v + G < prow) ? static_cast<uint32_t>(__ldg(nptr + G * nb)) : 0u;
-      nraw[d] = n0 | (n1 << 16);
+      uint32_t n0 = 0u;
+      if (bok && v < prow) n0 = __ldg(nptr);
+      uint32_t n1 = 0u;
+      if (bok && v + G < prow) n1 = __ldg(nptr + G * nb);
+      nlo[d] = n0;
+      nhi[d] = n1;
       pending |= 1u << d;
       if (++ig == ngr) {
         ig = 0;
@@ -406,16 +419,18 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       if (d < nw) issue(d);
 
     if (p0 == 0) {
-      // set-up while the first boxes are in flight: the codebook and the pair
-      // table depend on nothing the previous kernel writes, so they are built
-      // before the dependency wait (overlapping that kernel's last CTAs); then
-      // x is loaded and rotated; the barrier below publishes table and x
-      const uint32_t c16r = g1_codebook_lane(codebook);
-      g1_build_table(smem, c16r, 0, kG1Warps);
-      pdl_wait();  // x may be produced by the previous kernel on the stream
+      // set-up while the first boxes are in flight.  x may be produced by the
+      // previous kernel on the stream, so the dependency wait comes first and
+      // every thread passes it before it touches x or y; the x loads are then
+      // in flight while the pair table is built (the codebook load was issued
+      // before the wait), and the rotation consumes them.  The barrier below
+      // publishes table and x.
+      const float cl = __ldg(codebook + lane);
+      pdl_wait();
       uint32_t xw[8];
       const int rb0 = 4 * warp;
       if (rb0 < nb) g1_rot_load(x, in, in, nb, nb, xvec != 0, rb0, xw);
+      g1_build_table(smem, g1_codebook_half(cl, warp == 0), 0, kG1Warps);
       if (rb0 < nb) g1_rot_store(xw, nb, nb, rb0, xs, xinv);
       for (int b0 = rb0 + 4 * kG1Warps; b0 < nb; b0 += 4 * kG1Warps) {
         g1_rot_load(x, in, in, nb, nb, xvec != 0, b0, xw);
@@ -433,7 +448,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       for (int d = 0; d < S; ++d) {
         const int k = base + d;
         if (k < nw) {
-          const uint32_t nr = nraw[d];
+          const uint32_t nr0 = nlo[d], nr1 = nhi[d];
           if (ok && ((pending >> d) & 1u)) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
             if (ok) {
@@ -471,9 +486,9 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
             }
           }
           const float a0 = g1_dot(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                           (half_bits_to_float(static_cast<uint16_t>(nr)) * xi);
+                           (half_bits_to_float(static_cast<uint16_t>(nr0)) * xi);
           const float a1 = g1_dot(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                           (half_bits_to_float(static_cast<uint16_t>(nr >> 16)) * xi);
+                           (half_bits_to_float(static_cast<uint16_t>(nr1)) * xi);
           // reduce both rows over the 2C lanes: the first exchange leaves row
           // r's partial on lanes with bit C clear and row r + G's on the others
           const bool hi = (u & C) != 0;

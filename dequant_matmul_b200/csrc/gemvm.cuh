@@ -165,7 +165,7 @@ gemvm_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
 
     int ich = it0 / ngr, ig = it0 - (it0 / ngr) * ngr;
     const uint16_t* nptr = norms + (prow0 + ig * RG + r) * nb + ich * C + s;
-    uint32_t nraw[S];
+    uint32_t nlo[S], nhi[S];  // the two rows' norms, kept apart so that no instruction waits on them before use
     auto issue = [&](int d) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
@@ -173,9 +173,12 @@ gemvm_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       }
       const int v = ig * RG + r;
       const bool bok = ich * C + s < nb;
-      const uint32_t n0 = (bok && v < prow) ? static_cast<uint32_t>(__ldg(nptr)) : 0u;
-      const uint32_t n1 = (bok && v + G < prow) ? static_cast<uint32_t>(__ldg(nptr + G * nb)) : 0u;
-      nraw[d] = n0 | (n1 << 16);
+      uint32_t n0 = 0u;
+      if (bok && v < prow) n0 = __ldg(nptr);
+      uint32_t n1 = 0u;
+      if (bok && v + G < prow) n1 = __ldg(nptr + G * nb);
+      nlo[d] = n0;
+      nhi[d] = n1;
       pending |= 1u << d;
       if (++ig == ngr) {
         ig = 0;
@@ -215,7 +218,7 @@ gemvm_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
       for (int d = 0; d < S; ++d) {
         const int k = base + d;
         if (k < nw) {
-          const uint32_t nr = nraw[d];
+          const uint32_t nr0 = nlo[d], nr1 = nhi[d];
           if (ok && ((pending >> d) & 1u)) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
             if (ok) {
@@ -245,8 +248,8 @@ gemvm_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
           }
           float a0[MT], a1[MT];
           gm_dot<MT>(smem, cw0, cw1, lane4, xrow, a0, a1, std::make_integer_sequence<int, 32>{});
-          const float n0f = half_bits_to_float(static_cast<uint16_t>(nr));
-          const float n1f = half_bits_to_float(static_cast<uint16_t>(nr >> 16));
+          const float n0f = half_bits_to_float(static_cast<uint16_t>(nr0));
+          const float n1f = half_bits_to_float(static_cast<uint16_t>(nr1));
           const bool hi = (u & C) != 0;
           const int v = cg * RG + r + (hi ? G : 0);
 #pragma unroll

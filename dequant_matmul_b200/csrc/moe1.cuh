@@ -167,7 +167,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
   const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
   const int nw = it1 - it0;
   int ich = nq ? it0 / nq : 0, iq = it0 - ich * nq;
-  uint32_t nraw[S];
+  uint32_t nlo[S], nhi[S];  // the two rows' norms, kept apart so that no instruction waits on them before use
   auto issue = [&](int d) {
     const int q = q0 + iq, p = q / ngj, j0 = (q - p * ngj) * G;
     const int e = rid[p];
@@ -183,9 +183,12 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
     const int j = j0 + r, b = ich * C + s;
     const uint16_t* nm = sh ? P.sh_gu_norms : P.gu_norms;
     const bool v = j < F && b < nb;
-    const uint32_t n0 = v ? static_cast<uint32_t>(__ldg(nm + (rbase + j) * nb + b)) : 0u;
-    const uint32_t n1 = v ? static_cast<uint32_t>(__ldg(nm + (rbase + F + j) * nb + b)) : 0u;
-    nraw[d] = n0 | (n1 << 16);
+    uint32_t n0 = 0u;
+    if (v) n0 = __ldg(nm + (rbase + j) * nb + b);
+    uint32_t n1 = 0u;
+    if (v) n1 = __ldg(nm + (rbase + F + j) * nb + b);
+    nlo[d] = n0;
+    nhi[d] = n1;
     pending |= 1u << d;
     if (++iq == nq) { iq = 0; ++ich; }
   };
@@ -209,7 +212,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
     for (int d = 0; d < S; ++d) {
       const int k = base + d;
       if (k < nw) {
-        const uint32_t nr = nraw[d];
+        const uint32_t nr0 = nlo[d], nr1 = nhi[d];
         if (ok && ((pending >> d) & 1u)) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
           if (ok) {
@@ -237,9 +240,9 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
           moe1_load_x(xs, xinv, (t - t_lo) * nb + b, b < nb, hh, xr, xi);
         }
         const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                         (half_bits_to_float(static_cast<uint16_t>(nr)) * xi);
+                         (half_bits_to_float(static_cast<uint16_t>(nr0)) * xi);
         const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                         (half_bits_to_float(static_cast<uint16_t>(nr >> 16)) * xi);
+                         (half_bits_to_float(static_cast<uint16_t>(nr1)) * xi);
         const bool hi = (u & C) != 0;
         float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
 #pragma unroll
@@ -322,7 +325,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
     const int it0 = warp * nitems / kG1Warps, it1 = (warp + 1) * nitems / kG1Warps;
     const int nw = it1 - it0;
     int ilg = it0 % ngr, ich = (it0 / ngr) % nch, ip = pg0 + it0 / (ngr * nch);
-    uint32_t nraw[S];
+    uint32_t nlo[S], nhi[S];  // the two rows' norms, kept apart so that no instruction waits on them before use
     auto issue = [&](int d) {
       const int e = rid[ip];
       const bool sh = e == P.E;
@@ -335,9 +338,12 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
       }
       const int b = ich * C + s;
       const uint16_t* nm = (sh ? P.sh_dn_norms : P.dn_norms) + (rbase + lrow + r) * nb + b;
-      const uint32_t n0 = (b < nb && lrow + r < H) ? static_cast<uint32_t>(__ldg(nm)) : 0u;
-      const uint32_t n1 = (b < nb && lrow + r + G < H) ? static_cast<uint32_t>(__ldg(nm + G * nb)) : 0u;
-      nraw[d] = n0 | (n1 << 16);
+      uint32_t n0 = 0u;
+      if (b < nb && lrow + r < H) n0 = __ldg(nm);
+      uint32_t n1 = 0u;
+      if (b < nb && lrow + r + G < H) n1 = __ldg(nm + G * nb);
+      nlo[d] = n0;
+      nhi[d] = n1;
       pending |= 1u << d;
       if (++ilg == ngr) {
         ilg = 0;
@@ -364,7 +370,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
       for (int d = 0; d < S; ++d) {
         const int k = base + d;
         if (k < nw) {
-          const uint32_t nr2 = nraw[d];
+          const uint32_t nq0 = nlo[d], nq1 = nhi[d];
           if (ok && ((pending >> d) & 1u)) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar + 8 * d, (phase >> d) & 1u, deadline));
             if (ok) {
@@ -391,9 +397,9 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
             moe1_load_x(xs, xinv, (cp - pg0) * nb + b, b < nb, hh, xr, xi);
           }
           const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                           (half_bits_to_float(static_cast<uint16_t>(nr2)) * xi);
+                           (half_bits_to_float(static_cast<uint16_t>(nq0)) * xi);
           const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
-                           (half_bits_to_float(static_cast<uint16_t>(nr2 >> 16)) * xi);
+                           (half_bits_to_float(static_cast<uint16_t>(nq1)) * xi);
           const bool hi = (u & C) != 0;
           float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
 #pragma unroll
