@@ -26,7 +26,8 @@
 //              (no multicast);
 //   warp 25    allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
 //              N = tokens, K = 16) into an fp32 accumulator in TMEM;
-//   warps 0-3  epilogue: tcgen05.ld of the accumulator, scaling, bf16/fp32 store.
+//   warps 0-23 epilogue (six per TMEM lane quarter, split by columns):
+//              tcgen05.ld of the accumulator, scaling, bf16/fp32 store.
 // Stages are handed over with mbarriers; every wait is bounded (2 s), after
 // which the kernel raises HLWQ_DEVERR_TIMEOUT, drains and frees TMEM.
 
@@ -272,21 +273,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  __syncthreads();
-  uint16_t* nrm_s = reinterpret_cast<uint16_t*>(gbase + (nst - base));
-  if (warp < kTcDecWarps) {
-    // the tile's norms, row-major [128][nb], coalesced
-    for (int q = threadIdx.x; q < kTcTileRows * nb; q += 32 * kTcDecWarps) {
-      const int rr = q / nb;
-      nrm_s[q] = (o0 + rr < O) ? __ldg(norms + (o0 + rr) * nb + (q - rr * nb)) : static_cast<uint16_t>(0);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc_g[0];
+  uint16_t* nrm_s = reinterpret_cast<uint16_t*>(gbase + (nst - base));
 
   if (warp < kTcDecWarps) {
+    // The tile's norms [128][nb] are one contiguous run of the norm array
+    // (rows past O read as zero); they are staged while the producers start
+    // on the first code and B boxes, then a barrier of the decode warps only.
+    const int64_t nvalid = std::min<int64_t>(kTcTileRows, O - o0) * nb;
+    const uint16_t* nsrc = norms + o0 * nb;
+    const int ntot = kTcTileRows * nb;  // a multiple of 8
+    if ((reinterpret_cast<uintptr_t>(nsrc) & 15u) == 0) {
+      for (int q = threadIdx.x; q < ntot / 8; q += 32 * kTcDecWarps) {
+        if (8 * q + 8 <= nvalid) {
+          reinterpret_cast<uint4*>(nrm_s)[q] = __ldg(reinterpret_cast<const uint4*>(nsrc) + q);
+        } else {
+          for (int k = 8 * q; k < 8 * q + 8; ++k) nrm_s[k] = k < nvalid ? __ldg(nsrc + k) : static_cast<uint16_t>(0);
+        }
+      }
+    } else {
+      for (int q = threadIdx.x; q < ntot; q += 32 * kTcDecWarps)
+        nrm_s[q] = q < nvalid ? __ldg(nsrc + q) : static_cast<uint16_t>(0);
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcDecWarps) : "memory");
+
     // ---------------------------------------------------------- decode
     // two groups of 8 warps take alternate blocks; in a group, warp (q4, hh)
     // decodes half block hh of rows 32 q4 + lane
@@ -340,8 +353,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
       raise_device_error(HLWQ_DEVERR_TIMEOUT);
     }
 
-    // ---------------------------------------------------------- epilogue (warps 0-3)
-    if (warp < 4) {
+    // ---------------------------------------------------------- epilogue
+    // every decode warp: warp w reads TMEM lanes 32 (w mod 4) .. + 31 (its own
+    // rows) and columns 16 (w / 4) + 96 j, so six warps share a lane quarter
+    {
       const bool done = mbar_wait(accum, 0, deadline);
       tc_fence_after();
       if (!done) {
@@ -350,7 +365,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
       }
       const float rscale = ldexpf(1.0f, erow) * (1.0f / 128.0f);
       const bool store = done && misc_g[1] == 0u && row_ok;
-      for (int c0 = 0; c0 < n_box; c0 += 16) {
+      for (int c0 = 16 * (warp >> 2); c0 < n_box; c0 += 16 * (kTcDecWarps / 4)) {
         uint32_t acc[16];
         tc_ld16(tm_row + c0, acc);
         tc_wait_ld();
