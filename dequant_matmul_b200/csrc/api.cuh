@@ -21,6 +21,7 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
                    const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
                    size_t ws_bytes, cudaStream_t stream);
 size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M);
+size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M);
 size_t moe_workspace_bytes(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk);
 int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
                const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
@@ -97,7 +98,9 @@ extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const flo
   if (!aligned16(packed) || !aligned2(norms) || !aligned2(X) || !aligned2(Y) ||
       (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(Y) & 3u)))
     return HLWQ_EALIGN;
-  const size_t need = hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0);
+  // the tensor-core path accepts its smallest workspace (no K split of the
+  // last wave) up to the size hlwq_workspace_bytes reports
+  const size_t need = M >= kTensorCoreMinM ? hlwq::gemm_tc_workspace_min_bytes(out, in, M) : 0;
   if (need && (!workspace || ws_bytes < need)) return HLWQ_EWORKSPACE;
   if (need && !aligned16(workspace)) return HLWQ_EALIGN;
   if (M >= kTensorCoreMinM)

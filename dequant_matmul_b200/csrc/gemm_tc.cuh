@@ -84,6 +84,13 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -141,13 +148,16 @@ __device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
 // ---------------------------------------------------------------- rotation
 constexpr int kRotThreads = 256;
 
-// One CTA per token: B[m][:] = binary16(x_tilde[m][:] * s_m), inv_s[m] = 1 / s_m.
+// One CTA per token: B[m][:] = binary16(x_tilde[m][:] * s_m), inv_s[m] = 1 / s_m;
+// CTA 0 also clears the GEMM's K-split counters.
 __global__ void __launch_bounds__(kRotThreads)
 rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, uint16_t* __restrict__ B,
-                float* __restrict__ inv_s) {
+                float* __restrict__ inv_s, unsigned* __restrict__ part_cnt, int nsplit) {
   extern __shared__ __align__(16) float buf[];  // [nb * 128]
   __shared__ float red[kRotThreads / 32];
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (m == 0)  // the K-split counters of the GEMM that follows start at zero
+    for (int i = threadIdx.x; i < nsplit; i += kRotThreads) part_cnt[i] = 0u;
   const uint16_t* x = X + static_cast<int64_t>(m) * ldx;
   float mx = 0.0f;
   for (int b = warp; b < nb; b += kRotThreads / 32) {
@@ -224,7 +234,8 @@ __host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
                const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
-               const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box) {
+               const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box,
+               int row_tiles, int nfull, float* __restrict__ part, unsigned* __restrict__ part_cnt) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -236,7 +247,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   const uint32_t nst = cst + CS * kTcCodeBytes;          // tile norms [128][nb] (binary16)
   const uint32_t bars = base + 4 * kLevels;              // after the table, inside the first 1 KiB
   // barrier block: full[S] empty[S] c_full[CS] c_empty[CS] accum, then misc
-  // (TMEM base, abort flag): at most 128 + 8 (2 S + 2 CS + 1) + 8 = 288 bytes
+  // (TMEM base, abort flag, split count): at most 128 + 8 (2 S + 2 CS + 1) + 16 = 296 bytes
   const uint32_t full0 = bars, empty0 = full0 + 8 * S, c_full0 = empty0 + 8 * S, c_empty0 = c_full0 + 8 * CS,
                  accum = c_empty0 + 8 * CS;
   const uint32_t misc = accum + 8;
@@ -245,8 +256,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   const uint8_t* codes_g = gbase + (cst - base);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t o0 = static_cast<int64_t>(blockIdx.x) * kTcTileRows;
-  const int n0 = blockIdx.y * n_box;
+  // CTA -> tile and K range: CTAs [0, nfull) take whole tiles; the rest take
+  // the two K halves of the tiles after them (tile nfull + j / 2, half j % 2)
+  int tt = blockIdx.x, half = -1, kb0 = 0, kb1 = nb;
+  if (tt >= nfull) {
+    const int j = tt - nfull;
+    tt = nfull + (j >> 1);
+    half = j & 1;
+    kb0 = half ? nb / 2 : 0;
+    kb1 = half ? nb : nb / 2;
+  }
+  const int64_t o0 = static_cast<int64_t>(tt % row_tiles) * kTcTileRows;
+  const int n0 = (tt / row_tiles) * n_box;
   const uint64_t deadline = globaltimer_ns() + kTcTimeoutNs;
 
   // ---- set-up: codebook, barriers, TMEM
@@ -305,8 +326,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // decodes half block hh of rows 32 q4 + lane
     const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod kTcGroups
     const int r = 32 * q4 + lane;
-    const int64_t o = o0 + r;
-    const bool row_ok = o < O;
     const uint16_t* rown = nrm_s + r * nb;
     float nmax = 0.0f;
     for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, half_bits_to_float(rown[b]));
@@ -315,11 +334,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     const float rs = ldexpf(1.0f, -erow);
     const uint32_t tm_row = tmem + (static_cast<uint32_t>(32 * q4) << 16);
     bool ok = true;
-    for (int b = dg; b < nb && dg < G; b += G) {
-      const int cs = tc_code_stage(b, G), as = tc_ab_stage(b, G);
+    for (int b = kb0 + dg; b < kb1 && dg < G; b += G) {
+      const int lb = b - kb0;
+      const int cs = tc_code_stage(lb, G), as = tc_ab_stage(lb, G);
       const float nsc = half_bits_to_float(rown[b]) * rs;
       uint2 cw[5];
-      if (ok) ok = mbar_wait(c_full0 + 8 * cs, tc_code_parity(b, G), deadline);
+      if (ok) ok = mbar_wait(c_full0 + 8 * cs, tc_code_parity(lb, G), deadline);
       const uint2* src = reinterpret_cast<const uint2*>(codes_g + cs * kTcCodeBytes + r * kBlockBytes + 40 * hh);
 #pragma unroll
       for (int k = 0; k < 5; ++k) cw[k] = src[k];
@@ -334,7 +354,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const float2 a = fmul2(c, sc2);
         v[p] = cvt_half2(a.x, a.y);
       }
-      if (ok) ok = mbar_wait(empty0 + 8 * as, tc_ab_parity(b, G) ^ 1u, deadline);
+      if (ok) ok = mbar_wait(empty0 + 8 * as, tc_ab_parity(lb, G) ^ 1u, deadline);
       if (ok && misc_g[1] == 0u) {
         const uint32_t ta = tm_row + kTcAccCols + 64 * as + 32 * hh;
         uint32_t v0[16], v1[16];
@@ -364,20 +384,89 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
       const float rscale = ldexpf(1.0f, erow) * (1.0f / 128.0f);
-      const bool store = done && misc_g[1] == 0u && row_ok;
-      for (int c0 = 16 * (warp >> 2); c0 < n_box; c0 += 16 * (kTcDecWarps / 4)) {
-        uint32_t acc[16];
-        tc_ld16(tm_row + c0, acc);
-        tc_wait_ld();
-        if (store) {
+      constexpr int kCStep = 16 * (kTcDecWarps / 4);
+      bool write_tile = true;
+      const float* p0 = nullptr;
+      const float* p1 = nullptr;
+      if (half >= 0) {
+        // K-split tile: both halves write their fp32 partial ([column][row],
+        // so a warp's stores are contiguous), then count themselves in; the
+        // half that arrives second adds the two partials in the fixed order
+        // (K half 0) + (K half 1), so the result does not depend on which
+        // half finished first.  No CTA waits for another.
+        const int slot = tt - nfull;
+        float* q0 = part + static_cast<int64_t>(2 * slot) * n_box * kTcTileRows;
+        float* mine = q0 + (half ? static_cast<int64_t>(n_box) * kTcTileRows : 0);
+        p0 = q0;
+        p1 = q0 + static_cast<int64_t>(n_box) * kTcTileRows;
+        for (int c0 = 16 * (warp >> 2); c0 < n_box; c0 += kCStep) {
+          uint32_t acc[16];
+          tc_ld16(tm_row + c0, acc);
+          tc_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = n0 + c0 + j;
-            if (m < M) {
-              const float yv = __uint_as_float(acc[j]) * rscale * __ldg(inv_s + m);
-              const int64_t off = static_cast<int64_t>(m) * ldy + o;
-              if (out_bf16) static_cast<uint16_t*>(Y)[off] = static_cast<uint16_t>(float_to_bf16_bits(yv));
-              else static_cast<float*>(Y)[off] = yv;
+          for (int j = 0; j < 16; ++j) mine[(c0 + j) * kTcTileRows + r] = __uint_as_float(acc[j]);
+        }
+        __threadfence();
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * kTcDecWarps) : "memory");
+        if (threadIdx.x == 0) misc_g[2] = atomicAdd(part_cnt + slot, 1u);
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * kTcDecWarps) : "memory");
+        write_tile = misc_g[2] == 1u;
+        if (write_tile) __threadfence();
+      }
+      if (write_tile) {
+        // The scaled tile is staged in shared memory as [token][row] (the B
+        // stages are free once the accumulator is complete: n_box x 128 x 4
+        // bytes at most, within S >= 2 stages of n_box x 256), then written
+        // out as contiguous runs of every token's 128 outputs.
+        const int es = out_bf16 ? 2 : 4;
+        uint8_t* stage = gbase + (bst - base);
+        for (int c0 = 16 * (warp >> 2); c0 < n_box; c0 += kCStep) {
+#pragma unroll
+          for (int h8 = 0; h8 < 16; h8 += 8) {  // eight columns at a time (register budget)
+            float v[8];
+            if (half < 0) {
+              uint32_t acc[8];
+              tc_ld8(tm_row + c0 + h8, acc);
+              tc_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(acc[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int idx = (c0 + h8 + j) * kTcTileRows + r;
+                v[j] = __ldcg(p0 + idx) + __ldcg(p1 + idx);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int m = n0 + c0 + h8 + j;
+              const float yv = m < M ? v[j] * rscale * __ldg(inv_s + m) : 0.0f;
+              const int si = (c0 + h8 + j) * kTcTileRows + r;
+              if (out_bf16) reinterpret_cast<uint16_t*>(stage)[si] = static_cast<uint16_t>(float_to_bf16_bits(yv));
+              else reinterpret_cast<float*>(stage)[si] = yv;
+            }
+          }
+        }
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * kTcDecWarps) : "memory");
+        if (done && misc_g[1] == 0u) {
+          const int ncols = static_cast<int>(std::min<int64_t>(kTcTileRows, O - o0));  // outputs of the tile
+          const int mrows = std::min(n_box, M - n0);                                   // tokens of the tile
+          char* yb = static_cast<char*>(Y);
+          if (ncols == kTcTileRows && ((ldy * es) & 15) == 0) {
+            const int sh = out_bf16 ? 4 : 5;  // 16-byte pieces per token: 128 x es / 16
+            const int64_t pitch = ldy * es;
+            char* yt = yb + (static_cast<int64_t>(n0) * ldy + o0) * es;
+            for (int q = threadIdx.x; q < (mrows << sh); q += 32 * kTcDecWarps) {
+              const int ml = q >> sh, pc = q & ((1 << sh) - 1);
+              *reinterpret_cast<uint4*>(yt + ml * pitch + 16 * pc) = reinterpret_cast<const uint4*>(stage)[q];
+            }
+          } else {
+            for (int q = threadIdx.x; q < mrows * kTcTileRows; q += 32 * kTcDecWarps) {
+              const int ml = q >> 7, oc = q & (kTcTileRows - 1);
+              if (oc >= ncols) continue;
+              const int64_t off = (n0 + ml) * ldy + o0 + oc;
+              if (out_bf16) reinterpret_cast<uint16_t*>(yb)[off] = reinterpret_cast<const uint16_t*>(stage)[q];
+              else reinterpret_cast<float*>(yb)[off] = reinterpret_cast<const float*>(stage)[q];
             }
           }
         }
@@ -387,9 +476,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // ---------------------------------------------------------- TMA producer: code tiles
     if (lane == 0) {
       bool ok = true;
-      for (int b = 0; b < nb; ++b) {
-        const int cs = tc_code_stage(b, G);
-        ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b, G) ^ 1u, deadline) && misc_g[1] == 0u;
+      for (int b = kb0; b < kb1; ++b) {
+        const int cs = tc_code_stage(b - kb0, G);
+        ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
         mbar_arrive_expect_tx(c_full0 + 8 * cs, kTcCodeBytes);
         tma_load_2d(cst + cs * kTcCodeBytes, &cmap, kBlockBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
@@ -404,9 +493,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     if (lane == 0) {
       const uint32_t half_bytes = static_cast<uint32_t>(n_box) * 128u;
       bool ok = true;
-      for (int b = 0; b < nb; ++b) {
-        const int st = tc_ab_stage(b, G);
-        ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b, G) ^ 1u, deadline) && misc_g[1] == 0u;
+      for (int b = kb0; b < kb1; ++b) {
+        const int st = tc_ab_stage(b - kb0, G);
+        ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
         mbar_arrive_expect_tx(full0 + 8 * st, 2 * half_bytes);
         const uint32_t dst = bst + st * n_box * 256;
@@ -423,9 +512,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(n_box);
       bool ok = true;
-      for (int b = 0; b < nb; ++b) {
-        const int st = tc_ab_stage(b, G);
-        ok = mbar_wait(full0 + 8 * st, tc_ab_parity(b, G), deadline) && misc_g[1] == 0u;
+      for (int b = kb0; b < kb1; ++b) {
+        const int st = tc_ab_stage(b - kb0, G);
+        ok = mbar_wait(full0 + 8 * st, tc_ab_parity(b - kb0, G), deadline) && misc_g[1] == 0u;
         if (!ok) break;
         tc_fence_after();
         const uint32_t bstage = bst + st * n_box * 256;
@@ -435,7 +524,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < kTcKChunk / 16; ++kk)
             tc_mma_f16(tmem, tmem + kTcAccCols + 64 * st + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk),
-                       idesc, (b > 0 || h > 0 || kk > 0) ? 1u : 0u);
+                       idesc, (b > kb0 || h > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(empty0 + 8 * st);  // frees both the A stage (TMEM) and the B stage (shared memory)
       }
@@ -457,12 +546,44 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 
 }  // namespace
 
-size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
-  (void)O;
-  const int64_t nb = ceil_div(in, kBlock);
-  const size_t b_bytes = static_cast<size_t>(M) * nb * kBlock * 2;
-  return ((b_bytes + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(M) * 4 + 256;
+// Launch plan for a shape on the current device.  Tiles are 128 rows x n_box
+// tokens.  When the tiles fill the SMs once and leave a partial second wave
+// of at most half the SMs, those last tiles are split into two K halves (two
+// CTAs each), so the second wave takes half a tile's time on up to all SMs.
+// Workspace: B (binary16 rotated activations) | 1/s_m | split counters |
+// split partials (fp32, two per split tile).  A workspace of base_bytes
+// runs without the split.
+struct TcPlan {
+  int nb, n_box, row_tiles, n_tiles, nsplit;
+  size_t inv_off, cnt_off, part_off, base_bytes, split_bytes;
+};
+
+inline TcPlan tc_plan(int64_t O, int64_t in, int64_t M) {
+  auto r256 = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  TcPlan P;
+  P.nb = static_cast<int>(ceil_div(in, kBlock));
+  int n_box = static_cast<int>(std::min<int64_t>(256, (std::min<int64_t>(M, 256) + 15) / 16 * 16));
+  while (n_box > 16 && tc_smem_bytes(n_box, P.nb) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
+  P.n_box = n_box;
+  P.row_tiles = static_cast<int>(ceil_div(O, kTcTileRows));
+  P.n_tiles = static_cast<int>(ceil_div(M, n_box));
+  const int64_t tiles = static_cast<int64_t>(P.row_tiles) * P.n_tiles;
+  const int64_t sms = sm_count();
+  P.nsplit = (P.nb >= 2 && tiles > sms && 2 * (tiles - sms) <= sms) ? static_cast<int>(tiles - sms) : 0;
+  P.inv_off = r256(static_cast<size_t>(M) * P.nb * kBlock * 2);
+  P.base_bytes = P.inv_off + static_cast<size_t>(M) * 4 + 256;
+  P.cnt_off = r256(P.inv_off + static_cast<size_t>(M) * 4);
+  P.part_off = r256(P.cnt_off + static_cast<size_t>(P.nsplit) * 4);
+  P.split_bytes = P.part_off + static_cast<size_t>(P.nsplit) * 2 * kTcTileRows * n_box * 4;
+  return P;
 }
+
+size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
+  const TcPlan P = tc_plan(O, in, M);
+  return P.nsplit ? std::max(P.split_bytes, P.base_bytes) : P.base_bytes;
+}
+
+size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) { return tc_plan(O, in, M).base_bytes; }
 
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
@@ -473,10 +594,14 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
   const int nb = static_cast<int>(ceil_div(in, kBlock));
   // Rows longer than kTcMaxNb blocks do not fit the tile-norm staging: CUDA-core path.
   if (nb > kTcMaxNb) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
-  if (ws_bytes < gemm_tc_workspace_bytes(O, in, M)) return HLWQ_EWORKSPACE;
-  uint16_t* B = static_cast<uint16_t*>(workspace);
-  const size_t b_bytes = static_cast<size_t>(M) * nb * kBlock * 2;
-  float* inv_s = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((b_bytes + 255) & ~static_cast<size_t>(255)));
+  const TcPlan P = tc_plan(O, in, M);
+  if (ws_bytes < P.base_bytes) return HLWQ_EWORKSPACE;
+  const int nsplit = ws_bytes >= P.split_bytes ? P.nsplit : 0;
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* B = reinterpret_cast<uint16_t*>(ws);
+  float* inv_s = reinterpret_cast<float*>(ws + P.inv_off);
+  unsigned* part_cnt = reinterpret_cast<unsigned*>(ws + P.cnt_off);
+  float* part = nsplit ? reinterpret_cast<float*>(ws + P.part_off) : nullptr;
   const int rot_smem = nb * kBlock * 4;
   if (rot_smem > 200 * 1024) return HLWQ_EUNSUPPORTED;
   static bool rot_attr = false;
@@ -485,11 +610,10 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
       return HLWQ_ECUDA;
     rot_attr = true;
   }
-  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s);
+  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s, part_cnt, nsplit);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
 
-  int n_box = static_cast<int>(std::min<int64_t>(256, (std::min<int64_t>(M, 256) + 15) / 16 * 16));
-  while (n_box > 16 && tc_smem_bytes(n_box, nb) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
+  const int n_box = P.n_box;
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
   CUtensorMap map;
@@ -518,9 +642,10 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
     attr = true;
   }
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
-  dim3 grid(static_cast<unsigned>(ceil_div(O, kTcTileRows)), static_cast<unsigned>(ceil_div(M, n_box)));
-  gemm_tc_kernel<<<grid, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y, ldy,
-                                                     out_bf16 ? 1 : 0, n_box);
+  const int nfull = P.row_tiles * P.n_tiles - nsplit;
+  gemm_tc_kernel<<<nfull + 2 * nsplit, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
+                                                                   ldy, out_bf16 ? 1 : 0, n_box, P.row_tiles, nfull,
+                                                                   part, part_cnt);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
 

@@ -24,7 +24,7 @@
 #include "hlwq.h"
 
 namespace hlwq {
-size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M);
+size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M);
 }  // namespace hlwq
 
 namespace {
@@ -61,7 +61,10 @@ extern "C" int hlwq_gemm_noalloc(const uint8_t* packed, const uint16_t* norms, c
                                  int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy,
                                  int ydtype, void* stream) {
   if (!packed || !norms || !codebook || !X || !Y || out <= 0 || in <= 0 || M <= 0) return HLWQ_EINVAL;
-  const size_t need = hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0);
+  // the tensor-core path runs with its smallest workspace here; it uses the
+  // K split of its last tiles only when the scratch also holds the partials
+  const size_t need = hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
+                          ? hlwq::gemm_tc_workspace_min_bytes(out, in, M) : 0;
   if (need > kNoallocScratchBytes) return HLWQ_ESCRATCH;
   void* scratch = nullptr;
   if (need > 0) {

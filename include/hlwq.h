@@ -56,7 +56,7 @@ typedef enum {
   HLWQ_EALIGN = -2,       /* a pointer or leading dimension breaks the alignment rule */
   HLWQ_EUNSUPPORTED = -3, /* a size or dtype combination this build does not handle */
   HLWQ_ECUDA = -4,        /* a CUDA runtime call (launch, attribute) failed */
-  HLWQ_EWORKSPACE = -5,   /* workspace is NULL or smaller than hlwq_workspace_bytes() */
+  HLWQ_EWORKSPACE = -5,   /* workspace is NULL or below the call's minimum (hlwq_workspace_bytes; hlwq_gemm) */
   HLWQ_ESCRATCH = -6      /* request needs more than the static scratch of hlwq_gemm_noalloc */
 } hlwq_status;
 
@@ -142,6 +142,11 @@ int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const float* code
  *   workspace  device, ws_bytes >= hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
  * M = 1..4 runs on the CUDA-core decode path (one launch streams the weights for
  * up to four tokens); M >= 5 on the tensor-core path (workspace needed).
+ * On the tensor-core path the reported size includes fp32 partials for
+ * splitting the K range of the tiles of a partial last wave over two CTAs
+ * each (added in a fixed order, so results do not depend on timing).  Any
+ * workspace of at least 2 * M * 128 * ceil(in / 128) + 4 * M + 512 bytes is
+ * accepted; below the reported size the call runs without that split.
  */
 int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook,
               int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx,
@@ -188,9 +193,9 @@ size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, 
  * it is the same computation as hlwq_gemm, taking its scratch from a static
  * device array of HLWQ_NOALLOC_SCRATCH_BYTES instead of a caller workspace.
  *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
- *   - Requests needing more than HLWQ_NOALLOC_SCRATCH_BYTES of scratch
- *     (hlwq_workspace_bytes(HLWQ_OP_GEMM, ...)) return HLWQ_ESCRATCH; for the
- *     tensor-core path that is about M * ceil(in / 128) * 256 bytes.
+ *   - Requests whose smallest tensor-core workspace (about
+ *     M * ceil(in / 128) * 256 bytes, see hlwq_gemm) exceeds
+ *     HLWQ_NOALLOC_SCRATCH_BYTES return HLWQ_ESCRATCH.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
  *     stream capture.

@@ -237,3 +237,39 @@ def test_gemm_long_rows_m256(hl, cb):
         torch.cuda.synchronize()
         want = O_.matmul(q["packed"], q["norms"], I, X)
         assert rel_l2(Y.double().cpu().numpy(), want) <= MATMUL_REL, I
+
+
+def test_gemm_k_split_of_the_last_wave(hl, cb):
+    """168 row tiles on a 148-SM part: the 20 tiles after the first wave run as
+    two K halves each (fp32 partials, added in a fixed order by the half that
+    finishes second).  Rows sampled in whole and split tiles against the
+    oracle; repeated calls are bit-identical; the same call with the smallest
+    accepted workspace (no split) agrees within the tolerance."""
+    Od = 168 * 128
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(5)
+    for I, M in ((1024, 16), (704, 80)):
+        W = synth.student_t_device((Od, I), seed=I + M)
+        p, n = hl.quantize(W, cb)
+        rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(sms * 128 - 8, sms * 128 + 8),
+                                         np.arange(Od - 16, Od), rng.choice(Od, 64, replace=False)]))
+        q = O_.quantize(W[torch.as_tensor(rows, device=W.device)].cpu())
+        del W
+        X = synth.activations(M, I, seed=M + 2)
+        Xc = X.cuda()
+        full = hl.workspace_bytes(hl.HLWQ_OP_GEMM, Od, I, M)
+        small = 2 * M * 128 * ((I + 127) // 128) + 4 * M + 512
+        if sms == 148:
+            assert full > small  # the split's partials are part of the reported size
+        ws = torch.empty(full, dtype=torch.uint8, device="cuda")
+        Y1 = hl.gemm(p, n, cb, Xc, out_dtype=torch.float32, workspace=ws)
+        Y2 = hl.gemm(p, n, cb, Xc, out_dtype=torch.float32, workspace=ws)
+        Y3 = hl.gemm(p, n, cb, Xc, out_dtype=torch.float32,
+                     workspace=torch.empty(small, dtype=torch.uint8, device="cuda"))
+        torch.cuda.synchronize()
+        assert torch.equal(Y1, Y2)
+        want = O_.matmul(q["packed"], q["norms"], I, X)
+        for Y in (Y1, Y3):
+            assert rel_l2(Y.double().cpu().numpy()[:, rows], want) <= MATMUL_REL, (I, M)
+        assert (Y1 - Y3).abs().max().item() <= 1e-3 * Y3.abs().max().item()
+    assert hl.device_error() == 0
