@@ -14,9 +14,12 @@
 // bucket of width 1/64 by one FFMA whose rounding leaves the bucket index in the
 // low mantissa bits; each bucket holds at most one decision midpoint, stored as
 // an fp32 threshold whose low 5 bits carry the code of the bucket's lower edge,
-// so one compare finishes the search.  The table is replicated once per lane
-// (lane l reads bank l), so lookups never conflict.  A grid shift sigma keeps
-// every midpoint at least 4e-5 from a bucket edge.
+// so one compare finishes the search.  y is clamped to the table's range
+// [-3, 3] first; values beyond it land in the edge buckets, which send them to
+// the exact path below when a midpoint lies beyond the table on their side
+// (never for the Lloyd-Max codebook).  The table is replicated once per lane
+// (lane l reads bank l), so lookups never conflict.  A grid shift sigma keeps every midpoint at least 4e-5 from a
+// bucket edge.
 //
 // Exactness.  The fp32 rotation differs from the exact value by at most ~7.5e-6
 // (seven rounded additions of terms whose magnitudes sum to <= sqrt(128), plus
@@ -103,8 +106,12 @@ __device__ void build_quant_tables(const QuantShared& s, const float* __restrict
       else if (m <= hi) { ++inside; inside_k = k; }
       if (!shifted && (fabs(m - lo) < 4e-5 || fabs(m - hi) < 4e-5)) risky = true;
     }
+    // values beyond the table's range land in the edge buckets: those take
+    // the exact path when a midpoint (ascending) lies beyond the range on
+    // their side
+    const bool beyond = (i == 0 && s.mid[0] + sig < lo) || (i == kQBuckets - 1 && s.mid[kLevels - 2] + sig > hi);
     uint32_t thr;
-    if (inside >= 2 || risky) thr = 0x7fc00000u;                      // NaN: always the exact path
+    if (inside >= 2 || risky || beyond) thr = 0x7fc00000u;            // NaN: always the exact path
     else if (inside == 1) thr = __float_as_uint(static_cast<float>(s.mid[inside_k] + sig));
     else thr = __float_as_uint(3.0e38f);
     const uint32_t e = (thr & ~31u) | static_cast<uint32_t>(below);
@@ -356,8 +363,8 @@ quantize_kernel(const void* __restrict__ W, int64_t rows, int in, int nb, const 
           const uint32_t code = (ent & 31u) + (ys > thr ? 1u : 0u);
           if (!(fabsf(ys - thr) >= kQGuard)) fm |= 1u << e;
           const int bit = 5 * e, w = bit >> 5, sh = bit & 31;
-          p[w] |= code << sh;
-          if (sh > 27) p[w + 1] |= code >> (32 - sh);
+          p[w] += code << sh;  // fields are disjoint: + lets shift and add be one instruction
+          if (sh > 27) p[w + 1] += code >> (32 - sh);
         }
       }
     }

@@ -106,3 +106,28 @@ def test_dequantize(hl, cb, shape, odt):
     else:
         # bf16 output: exactly the bf16 rounding of the fp32 result (within one bf16 ulp of fp64)
         assert rel_l2(g, want) <= 4e-3
+
+
+def test_quantize_codebook_with_midpoints_beyond_the_table(hl, cb):
+    """A strictly ascending codebook whose outer decision midpoints lie beyond
+    +-3 (the Lloyd-Max centroids times 1.6, outermost midpoint ~4): rotated
+    values beyond the quantizer's bucket table go to its exact path, so the
+    codes still equal brute-force nearest-centroid codes of the oracle's
+    rotated values (decisions within 1e-5 of a midpoint excepted)."""
+    wide = (cb * 1.6).contiguous()
+    c = wide.cpu().double().numpy()
+    mids = 0.5 * (c[1:] + c[:-1])
+    assert mids.max() > 3.5 and mids.min() < -3.5
+    W = synth.gaussian_with_outliers(256, 1024, seed=7)
+    p, n = hl.quantize(W.cuda(), wide)
+    torch.cuda.synchronize()
+    assert hl.device_error() == 0
+    q = O.quantize(W, return_rotated=True)
+    y = q["y"]
+    assert (np.abs(y) > 3.5).sum() > 50  # the case is exercised
+    want = O.nearest_centroid(y, c)
+    got = O.unpack_codes(p.cpu().numpy()).reshape(want.shape)
+    bad = got != want
+    if bad.any():
+        near = np.min(np.abs(y[bad][:, None] - mids[None, :]), axis=1)
+        assert np.all(near < 1e-5), (int(bad.sum()), float(near.max()))
