@@ -15,6 +15,8 @@ int launch_quantize(const void* W, bool bf16, int64_t rows, int in, const float*
                     uint16_t* norms, cudaStream_t stream);
 int launch_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows, int in,
                       void* out, bool bf16, cudaStream_t stream);
+int launch_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows,
+                           int in, uint8_t* q4, uint16_t* scale, uint16_t* zero, cudaStream_t stream);
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
 int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
@@ -63,6 +65,18 @@ extern "C" int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, con
     return HLWQ_EALIGN;
   return hlwq::launch_dequantize(packed, norms, codebook, rows, static_cast<int>(in), W_out, odtype == HLWQ_BF16,
                                  as_stream(stream));
+}
+
+extern "C" int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+                                    int64_t rows, int64_t in, uint8_t* q4, uint16_t* scale, uint16_t* zero,
+                                    void* stream) {
+  if (!packed || !norms || !codebook || !q4 || !scale || !zero || rows <= 0 || in <= 0 || in > kMaxIn)
+    return HLWQ_EINVAL;
+  if (in % hlwq::kBlock) return HLWQ_EUNSUPPORTED;  // non-aligned rows stay in the Q5 / dequantized form
+  if (!aligned16(packed) || !aligned16(q4) || !aligned2(norms) || !aligned2(scale) || !aligned2(zero))
+    return HLWQ_EALIGN;
+  return hlwq::launch_requantize_int4(packed, norms, codebook, rows, static_cast<int>(in), q4, scale, zero,
+                                      as_stream(stream));
 }
 
 extern "C" int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,

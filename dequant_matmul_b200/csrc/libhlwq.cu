@@ -6,4 +6,5 @@
 #include "moe.cuh"
 #include "moe1.cuh"
 #include "gemm_tc.cuh"
+#include "int4.cuh"
 #include "api.cuh"

@@ -30,6 +30,7 @@ SIGNATURES = {
     "hlwq_lloyd_codebook": (_I, [_I, _P, _P, _P]),
     "hlwq_quantize": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
+    "hlwq_requantize_int4": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_gemv": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
     "hlwq_gemv_ex": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, ctypes.c_uint, _P]),
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
@@ -148,6 +149,24 @@ def dequantize(packed, norms, cb, in_features: int, out_dtype=torch.float32, out
     _check(lib.hlwq_dequantize(_ptr(packed), _ptr(norms), _ptr(cb), rows, in_features, _ptr(out),
                                _dtype_code(out.dtype), _stream(stream)), "hlwq_dequantize")
     return out
+
+
+def requantize_int4(packed, norms, cb, in_features: int, q4=None, scale=None, zero=None, stream=None):
+    """Q5 -> INT4 (groups of 128): returns (q4 uint8 [..., NB, 64], scale and
+    zero as bfloat16 bit patterns, uint16 [..., NB])."""
+    _cuda(packed, "packed")
+    nb = packed.shape[-2]
+    lead = tuple(packed.shape[:-2])
+    rows = packed.numel() // (nb * BLOCK_BYTES)
+    if q4 is None:
+        q4 = torch.empty(lead + (nb, 64), dtype=torch.uint8, device=packed.device)
+    if scale is None:
+        scale = torch.empty(lead + (nb,), dtype=torch.uint16, device=packed.device)
+    if zero is None:
+        zero = torch.empty(lead + (nb,), dtype=torch.uint16, device=packed.device)
+    _check(lib.hlwq_requantize_int4(_ptr(packed), _ptr(norms), _ptr(cb), rows, in_features, _ptr(q4), _ptr(scale),
+                                    _ptr(zero), _stream(stream)), "hlwq_requantize_int4")
+    return q4, scale, zero
 
 
 def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None, flags: int = 0):

@@ -111,6 +111,26 @@ int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, const float* c
                     int64_t rows, int64_t in, void* W_out, int odtype, void* stream);
 
 /*
+ * Q5 -> INT4 re-encoding ("Qwopus3.6-27B-v2 . HLWQ Q5", Pipeline: dequantize
+ * per Linear, then INT4 weight-only with groups of 128 on 128-aligned Linears).
+ * Per row and group b of 128 inputs (= the Q5 block), with w the dequantized
+ * weights (as hlwq_dequantize, evaluated exactly in fp64):
+ *   s = bf16((max w - min w) / 15),  z = bf16(min w)   (round to nearest even
+ *       from the fp64 value; magnitudes below 2^-126 give a signed zero; a
+ *       zero minimum is stored as +0)
+ *   q_i = clamp(rint((w_i - z) / s), 0, 15) in fp64 (q = 0 when s = 0)
+ *   q4     device uint8 [rows][in/128][64]: element 2k in bits 0-3 of byte k,
+ *          element 2k+1 in bits 4-7 (16-byte aligned)
+ *   scale  device uint16 [rows][in/128]: bfloat16 bits of s
+ *   zero   device uint16 [rows][in/128]: bfloat16 bits of z
+ * The INT4 weights are z + q * s.  in must be a multiple of 128 (non-aligned
+ * rows stay in the Q5 form): otherwise HLWQ_EUNSUPPORTED.
+ * Errors: HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_ECUDA.
+ */
+int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook,
+                         int64_t rows, int64_t in, uint8_t* q4, uint16_t* scale, uint16_t* zero, void* stream);
+
+/*
  * Decode GEMV: y[o] = sum_i x[i] * w_hat[o][i], fp32 accumulation, without
  * materialising w_hat (the activation is rotated once per 128-block and dotted
  * with centroid values in the rotated domain).

@@ -11,7 +11,7 @@ rotated-and-cleaned weights are re-encoded to INT4):
   1. w_hat = the HLWQ dequantization of the row (hlwq_oracle.dequantize);
   2. per row and group g of 128 consecutive inputs (the HLWQ block b = g):
        lo = min w_hat, hi = max w_hat over the group,
-       s  = bf16(( hi - lo ) / 15),  z = bf16(lo),
+       s  = bf16(( hi - lo ) / 15),  z = bf16(lo + 0),
        q  = clamp(rint((w_hat - z) / s), 0, 15)   (q = 0 everywhere if s = 0),
      dequantized as z + q * s;
   3. store q two per byte, element 2k in the low nibble of byte k (64 bytes per
@@ -23,7 +23,9 @@ Readings where the pages are silent (each pinned in tests/test_oracle_int4.py):
       of the library the pages name is not reproduced.
   I2  Scale and zero are stored as bfloat16, rounded to nearest even directly
       from the fp64 value; values below the bfloat16 normal range round to a
-      signed zero.  The codes are chosen against the stored (rounded) s and z.
+      signed zero.  A zero minimum is stored as +0 (z = bf16(min + 0.0): the
+      minimum of a zero block may be -0 or +0).  The codes are chosen against
+      the stored (rounded) s and z.
   I3  Every step is evaluated in fp64.  w_hat is exact in fp64 (sums of 128
       fp32 centroids times +-1, times an fp16 norm / 128), so the decisions are
       reproducible bit for bit by any implementation that evaluates the same
@@ -97,7 +99,7 @@ def int4_encode_groups(w) -> dict:
     lo = w.min(axis=-1)
     hi = w.max(axis=-1)
     s_bits = bf16_rne_bits((hi - lo) / 15.0)
-    z_bits = bf16_rne_bits(lo)
+    z_bits = bf16_rne_bits(lo + 0.0)  # -0 -> +0 (reading I2)
     s = bf16_bits_to_f64(s_bits)[..., None]
     z = bf16_bits_to_f64(z_bits)[..., None]
     with np.errstate(divide="ignore", invalid="ignore"):

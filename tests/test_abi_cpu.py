@@ -60,6 +60,9 @@ def test_validation_before_launch(hl):
     assert L.hlwq_quantize(p, hl.HLWQ_BF16, 4, 128, p, odd, p, None) == hl.HLWQ_EALIGN
     assert L.hlwq_dequantize(p, p, p, 4, -1, p, hl.HLWQ_F32, None) == hl.HLWQ_EINVAL
     assert L.hlwq_gemv(p, p, p, 4, 128, p, p, 7, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_requantize_int4(p, p, p, 4, 128, None, p, p, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_requantize_int4(p, p, p, 4, 704, p, p, p, None) == hl.HLWQ_EUNSUPPORTED  # not 128-aligned
+    assert L.hlwq_requantize_int4(p, p, p, 4, 128, ctypes.c_void_p(264), p, p, None) == hl.HLWQ_EALIGN
     assert L.hlwq_gemm(p, p, p, 4, 128, 2, p, 64, p, 4, hl.HLWQ_BF16, None, 0, None) == hl.HLWQ_EINVAL  # ldx < in
     ws = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 8, 256, 8)
     assert ws > 0

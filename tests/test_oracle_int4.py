@@ -115,6 +115,8 @@ def test_int4_constant_group_and_zero_block():
     r = O.requantize_int4(q["packed"], q["norms"], 256)
     back = O.dequantize_int4(r["q4"], r["scale"], r["zero"])
     assert np.all(back[0] == 0.0) and np.all(back[1, :128] == 0.0)
+    # the zero block's minimum is a signed zero: stored as +0 (reading I2)
+    assert np.all(r["zero"][0] == 0x0000) and np.all(r["scale"][0] == 0x0000)
 
 
 def test_int4_only_for_aligned_rows():
