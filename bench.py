@@ -9,7 +9,8 @@ weight bytes (packed codes + fp16 norms) of all ranks / device time (max over
 ranks).  At N = 1 the same run also measures the other parts of the metric
 ("components"): quantizer Gweights/s on the 128-expert layer (128 x (1408 x 2816
 + 2816 x 704) weights), GEMM TFLOP/s on 27648 x 5120 at M = 16/64/256, MoE GB/s
-on the 256(+1)-expert layer at T = 1/8/64 and the dequantizer.
+on the 256(+1)-expert layer at T = 1/8/64 and the 128-expert layer at T = 1/16,
+and the Q5 -> INT4 re-encoder on 27648 x 5120.
 
 ``--impl reference`` times the CPU oracle (oracle/, fp64 numpy) on the host
 cores on a bounded sample of the same GEMV workload and prints the same line.
@@ -183,7 +184,7 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, steps: int, ms_total_max
 
 
 # ---------------------------------------------------------------- components (N = 1)
-def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe")):
+def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4")):
     import torch
     from dequant_matmul_b200 import synth
     out = {}
@@ -196,6 +197,8 @@ def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe")):
         out.update(bench_gemm(hl, cb, peaks, stream))
     if "moe" in parts:
         out.update(bench_moe(hl, cb, peaks, stream, scrub))
+    if "int4" in parts:
+        out.update(bench_int4(hl, cb, peaks, stream))
     return out
 
 
@@ -264,6 +267,35 @@ def bench_gemm(hl, cb, peaks, stream):
     out["gemm_27648x5120"] = gemm
     del copies
     return out
+
+
+def bench_int4(hl, cb, peaks, stream):
+    import torch
+    from dequant_matmul_b200 import synth
+    # Q5 -> INT4 re-encoding of the 27648 x 5120 layer; two copies alternate (> L2).
+    O3, I3 = 27648, 5120
+    nb = I3 // 128
+    copies = []
+    for c in range(2):
+        w = synth.student_t_device((O3, I3), seed=90 + c)
+        copies.append(hl.quantize(w, cb, stream=stream))
+        del w
+    q4 = torch.empty(O3, nb, 64, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(O3, nb, dtype=torch.uint16, device="cuda")
+    zr = torch.empty(O3, nb, dtype=torch.uint16, device="cuda")
+
+    def run():
+        for p, n in copies:
+            hl.requantize_int4(p, n, cb, I3, q4, sc, zr, stream=stream)
+
+    ms, _ = time_graph(run, reps=10, warmup=3, stream=stream)
+    ms /= len(copies)
+    byts = O3 * nb * (80 + 2 + 64 + 2 + 2)   # Q5 codes + norm in, INT4 codes + scale + zero out
+    gbs = byts / ms / 1e6
+    del copies, q4, sc, zr
+    return {"requantize_int4_27648x5120": {"ms": round(ms, 4), "gweights_per_s": round(O3 * I3 / ms / 1e6, 2),
+                                           "gbs": round(gbs, 1), "hbm_frac": frac(gbs, peaks["hbm_gbs"]),
+                                           "algo_bytes": byts}}
 
 
 def bench_moe(hl, cb, peaks, stream, scrub):
@@ -376,7 +408,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe"], default=None,
+    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4"], default=None,
                     help="run only the component measurements (used for profiling captures)")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
@@ -415,7 +447,7 @@ def main():
     stream = torch.cuda.Stream()
     cb = hl.codebook("cuda")
     if args.only is not None:
-        parts = ("quantize", "gemm", "moe") if args.only == "components" else (args.only,)
+        parts = ("quantize", "gemm", "moe", "int4") if args.only == "components" else (args.only,)
         print(json.dumps({"components": components(hl, cb, peaks, stream, parts)}), flush=True)
         return
     # 64 distinct layers (quantized on the device from seeded synthetic weights)
