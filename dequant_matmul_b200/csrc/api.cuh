@@ -17,6 +17,12 @@ int launch_dequantize(const uint8_t* packed, const uint16_t* norms, const float*
                       void* out, bool bf16, cudaStream_t stream);
 int launch_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows,
                            int in, uint8_t* q4, uint16_t* scale, uint16_t* zero, cudaStream_t stream);
+int launch_kv_quantize(const uint16_t* X, int64_t n, int64_t ldx, const float* codebook, uint8_t* packed,
+                       uint16_t* norms, cudaStream_t stream);
+int launch_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t n, void* out,
+                         bool bf16, cudaStream_t stream);
+int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
+                     const float* codebook, int64_t n, float* S, int64_t lds, cudaStream_t stream);
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
 int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
@@ -77,6 +83,34 @@ extern "C" int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms
     return HLWQ_EALIGN;
   return hlwq::launch_requantize_int4(packed, norms, codebook, rows, static_cast<int>(in), q4, scale, zero,
                                       as_stream(stream));
+}
+
+extern "C" int hlwq_kv_quantize(const uint16_t* x, int64_t n, int64_t ldx, const float* codebook8, uint8_t* packed,
+                                uint16_t* norms, void* stream) {
+  if (!x || !codebook8 || !packed || !norms || n <= 0 || n > (int64_t(1) << 40) || ldx < 256) return HLWQ_EINVAL;
+  if (!aligned2(x) || (reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms)) return HLWQ_EALIGN;
+  return hlwq::launch_kv_quantize(x, n, ldx, codebook8, packed, norms, as_stream(stream));
+}
+
+extern "C" int hlwq_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook8, int64_t n,
+                                  void* out, int odtype, void* stream) {
+  if (!packed || !norms || !codebook8 || !out || n <= 0 || n > (int64_t(1) << 40)) return HLWQ_EINVAL;
+  if (odtype != HLWQ_F32 && odtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms) || !aligned16(out)) return HLWQ_EALIGN;
+  return hlwq::launch_kv_dequantize(packed, norms, codebook8, n, out, odtype == HLWQ_BF16, as_stream(stream));
+}
+
+extern "C" int hlwq_kv_scores(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* packed,
+                              const uint16_t* norms, const float* codebook8, int64_t n, float* scores, int64_t lds,
+                              void* stream) {
+  if (!q || !packed || !norms || !codebook8 || !scores || m <= 0 || n <= 0 || n > (int64_t(1) << 40) ||
+      ldq < 256 || lds < n)
+    return HLWQ_EINVAL;
+  if (m > 64) return HLWQ_EUNSUPPORTED;
+  if (!aligned2(q) || (reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms) ||
+      (reinterpret_cast<uintptr_t>(scores) & 3u))
+    return HLWQ_EALIGN;
+  return hlwq::launch_kv_scores(q, m, ldq, packed, norms, codebook8, n, scores, lds, as_stream(stream));
 }
 
 extern "C" int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,

@@ -7,4 +7,5 @@
 #include "moe1.cuh"
 #include "gemm_tc.cuh"
 #include "int4.cuh"
+#include "kv.cuh"
 #include "api.cuh"

@@ -31,6 +31,9 @@ SIGNATURES = {
     "hlwq_quantize": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
     "hlwq_requantize_int4": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P]),
+    "hlwq_kv_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "hlwq_kv_dequantize": (_I, [_P, _P, _P, _I64, _P, _I, _P]),
+    "hlwq_kv_scores": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _I64, _P]),
     "hlwq_gemv": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
     "hlwq_gemv_ex": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, ctypes.c_uint, _P]),
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
@@ -91,6 +94,14 @@ def _cuda(t: torch.Tensor, name: str):
         raise HLWQError(f"{name} must be contiguous")
 
 
+def _cuda_rows(t: torch.Tensor, name: str):
+    """A CUDA matrix whose rows are contiguous (any row pitch)."""
+    if not t.is_cuda:
+        raise HLWQError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise HLWQError(f"{name} must be a matrix with contiguous rows")
+
+
 def n_blocks(in_features: int) -> int:
     return (in_features + BLOCK - 1) // BLOCK
 
@@ -109,6 +120,11 @@ def lloyd_codebook(levels: int = LEVELS):
 
 def codebook(device="cuda") -> torch.Tensor:
     return lloyd_codebook(LEVELS)[0].to(device)
+
+
+def kv_codebook(device="cuda") -> torch.Tensor:
+    """The 8 Lloyd-Max centroids of the Q3 KV-cache encoding."""
+    return lloyd_codebook(8)[0].to(device)
 
 
 def workspace_bytes(op: int, a: int, b: int, c: int, E: int = 1, topk: int = 0) -> int:
@@ -167,6 +183,39 @@ def requantize_int4(packed, norms, cb, in_features: int, q4=None, scale=None, ze
     _check(lib.hlwq_requantize_int4(_ptr(packed), _ptr(norms), _ptr(cb), rows, in_features, _ptr(q4), _ptr(scale),
                                     _ptr(zero), _stream(stream)), "hlwq_requantize_int4")
     return q4, scale, zero
+
+
+def kv_quantize(X: torch.Tensor, cb8, packed=None, norms=None, stream=None):
+    """X bf16 [N][256] (row pitch X.stride(0)) -> (packed uint8 [N][96], norms fp16 bits uint16 [N])."""
+    _cuda_rows(X, "X")
+    N = X.shape[0]
+    if packed is None:
+        packed = torch.empty(N, 96, dtype=torch.uint8, device=X.device)
+    if norms is None:
+        norms = torch.empty(N, dtype=torch.uint16, device=X.device)
+    _check(lib.hlwq_kv_quantize(_ptr(X), N, X.stride(0), _ptr(cb8), _ptr(packed), _ptr(norms), _stream(stream)),
+           "hlwq_kv_quantize")
+    return packed, norms
+
+
+def kv_dequantize(packed, norms, cb8, out_dtype=torch.float32, out=None, stream=None):
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty(N, 256, dtype=out_dtype, device=packed.device)
+    _check(lib.hlwq_kv_dequantize(_ptr(packed), _ptr(norms), _ptr(cb8), N, _ptr(out), _dtype_code(out.dtype),
+                                  _stream(stream)), "hlwq_kv_dequantize")
+    return out
+
+
+def kv_scores(Q: torch.Tensor, packed, norms, cb8, S=None, stream=None):
+    """Q bf16 [M][256] (M <= 64, row pitch Q.stride(0)) against N encoded vectors -> S fp32 [M][N]."""
+    _cuda_rows(Q, "Q")
+    M, N = Q.shape[0], packed.shape[0]
+    if S is None:
+        S = torch.empty(M, N, dtype=torch.float32, device=Q.device)
+    _check(lib.hlwq_kv_scores(_ptr(Q), M, Q.stride(0), _ptr(packed), _ptr(norms), _ptr(cb8), N, _ptr(S), S.stride(0),
+                              _stream(stream)), "hlwq_kv_scores")
+    return S
 
 
 def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None, flags: int = 0):

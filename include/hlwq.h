@@ -131,6 +131,32 @@ int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const flo
                          int64_t rows, int64_t in, uint8_t* q4, uint16_t* scale, uint16_t* zero, void* stream);
 
 /*
+ * Q3 KV-cache encoding ("Qwopus3.6-27B-v2 . HLWQ Q5", Methodology notes,
+ * KV-cache bullet: per-head Hadamard 256x256, 8-centroid Lloyd-Max, 3 bits per
+ * value; head_dim = 256).  One vector = one (token, head) key or value.
+ *   codebook8  device float32 [8], strictly ascending (hlwq_lloyd_codebook(8))
+ *   packed     [N][96]: code j of a vector at bits [3j, 3j+3), LSB first
+ *   norms      [N]: binary16 bits of ||x||_2 (round to nearest even from fp64)
+ * hlwq_kv_quantize: x bf16 [N][ldx] (ldx >= 256) -> packed, norms; code_j =
+ *   number of midpoints of the codebook below y_j = (x @ H256)_j / ||x||, all
+ *   in fp64 (ties to the lower index; a zero vector gets code 3).
+ * hlwq_kv_dequantize: -> out [N][256] (HLWQ_F32 or HLWQ_BF16, 16-byte
+ *   aligned) = n16 * (c[code] @ H256) / 256.
+ * hlwq_kv_scores: S[m][i] = q_m . x_hat_i for M <= 64 bf16 queries [M][ldq]
+ *   (fp32, row pitch lds >= N); evaluated with each query rotated once.
+ * The 128 most recent tokens (the residual buffer) are the caller's: they stay
+ * in bf16 and are encoded as they leave that window.
+ * Errors: HLWQ_EINVAL, HLWQ_EALIGN (packed 4-byte, norms / x / q 2-byte
+ * alignment), HLWQ_EUNSUPPORTED (dtype; M > 64), HLWQ_ECUDA.
+ */
+int hlwq_kv_quantize(const uint16_t* x, int64_t n, int64_t ldx, const float* codebook8, uint8_t* packed,
+                     uint16_t* norms, void* stream);
+int hlwq_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook8, int64_t n,
+                       void* out, int odtype, void* stream);
+int hlwq_kv_scores(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
+                   const float* codebook8, int64_t n, float* scores, int64_t lds, void* stream);
+
+/*
  * Decode GEMV: y[o] = sum_i x[i] * w_hat[o][i], fp32 accumulation, without
  * materialising w_hat (the activation is rotated once per 128-block and dotted
  * with centroid values in the rotated domain).

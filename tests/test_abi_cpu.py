@@ -63,6 +63,10 @@ def test_validation_before_launch(hl):
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, None, p, p, None) == hl.HLWQ_EINVAL
     assert L.hlwq_requantize_int4(p, p, p, 4, 704, p, p, p, None) == hl.HLWQ_EUNSUPPORTED  # not 128-aligned
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, ctypes.c_void_p(264), p, p, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_kv_quantize(p, 4, 128, p, p, p, None) == hl.HLWQ_EINVAL             # ldx < 256
+    assert L.hlwq_kv_dequantize(p, p, p, 4, p, hl.HLWQ_F16, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_kv_scores(p, 65, 256, p, p, p, 4, p, 4, None) == hl.HLWQ_EUNSUPPORTED  # > 64 queries
+    assert L.hlwq_kv_scores(p, 2, 256, odd, p, p, 4, p, 4, None) == hl.HLWQ_EALIGN
     assert L.hlwq_gemm(p, p, p, 4, 128, 2, p, 64, p, 4, hl.HLWQ_BF16, None, 0, None) == hl.HLWQ_EINVAL  # ldx < in
     ws = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 8, 256, 8)
     assert ws > 0
