@@ -10,7 +10,8 @@ ranks).  At N = 1 the same run also measures the other parts of the metric
 ("components"): quantizer Gweights/s on the 128-expert layer (128 x (1408 x 2816
 + 2816 x 704) weights), GEMM TFLOP/s on 27648 x 5120 at M = 16/64/256, MoE GB/s
 on the 256(+1)-expert layer at T = 1/8/64 and the 128-expert layer at T = 1/16,
-and the Q5 -> INT4 re-encoder on 27648 x 5120.
+the Q5 -> INT4 re-encoder on 27648 x 5120 and the Q3 KV-cache encoding (131072
+vectors of 256: quantize, decode, scores for 6 queries).
 
 ``--impl reference`` times the CPU oracle (oracle/, fp64 numpy) on the host
 cores on a bounded sample of the same GEMV workload and prints the same line.
@@ -184,7 +185,7 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, steps: int, ms_total_max
 
 
 # ---------------------------------------------------------------- components (N = 1)
-def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4")):
+def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", "kv")):
     import torch
     from dequant_matmul_b200 import synth
     out = {}
@@ -199,6 +200,8 @@ def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4"))
         out.update(bench_moe(hl, cb, peaks, stream, scrub))
     if "int4" in parts:
         out.update(bench_int4(hl, cb, peaks, stream))
+    if "kv" in parts:
+        out.update(bench_kv(hl, peaks, stream))
     return out
 
 
@@ -296,6 +299,39 @@ def bench_int4(hl, cb, peaks, stream):
     return {"requantize_int4_27648x5120": {"ms": round(ms, 4), "gweights_per_s": round(O3 * I3 / ms / 1e6, 2),
                                            "gbs": round(gbs, 1), "hbm_frac": frac(gbs, peaks["hbm_gbs"]),
                                            "algo_bytes": byts}}
+
+
+def bench_kv(hl, peaks, stream):
+    import torch
+    from dequant_matmul_b200 import synth
+    # Q3 KV cache: 4 KV heads x 32768 tokens = 131072 vectors of 256 (a long
+    # context of the head_dim-256 GQA model); scores for one GQA group of 6
+    # query heads against one head's 32768 keys, and against all 131072.
+    N = 4 * 32768
+    cb8 = hl.kv_codebook("cuda")
+    X = synth.activations_device(N, 256, seed=95)
+    packed = torch.empty(N, 96, dtype=torch.uint8, device="cuda")
+    norms = torch.empty(N, dtype=torch.uint16, device="cuda")
+    out16 = torch.empty(N, 256, dtype=torch.bfloat16, device="cuda")
+    Q = synth.activations_device(6, 256, seed=96)
+    S = torch.empty(6, N, dtype=torch.float32, device="cuda")
+    res = {}
+    ms, _ = time_graph(lambda: hl.kv_quantize(X, cb8, packed, norms, stream=stream), reps=10, warmup=3, stream=stream)
+    b = N * (512 + 96 + 2)
+    res["quantize"] = {"ms": round(ms, 4), "vectors_per_s_M": round(N / ms / 1e3, 2), "gbs": round(b / ms / 1e6, 1),
+                       "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
+    ms, _ = time_graph(lambda: hl.kv_dequantize(packed, norms, cb8, out=out16, stream=stream), reps=10, warmup=3,
+                       stream=stream)
+    b = N * (96 + 2 + 512)
+    res["dequantize_bf16"] = {"ms": round(ms, 4), "gbs": round(b / ms / 1e6, 1),
+                              "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
+    ms, _ = time_graph(lambda: hl.kv_scores(Q, packed, norms, cb8, S=S, stream=stream), reps=10, warmup=3,
+                       stream=stream)
+    b = N * (96 + 2 + 6 * 4)
+    res["scores_6q"] = {"ms": round(ms, 4), "keys_per_s_G": round(N / ms / 1e6, 2), "gbs": round(b / ms / 1e6, 1),
+                        "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
+    del X, packed, norms, out16, Q, S
+    return {"kv_q3_131072x256": res}
 
 
 def bench_moe(hl, cb, peaks, stream, scrub):
@@ -408,7 +444,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4"], default=None,
+    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv"], default=None,
                     help="run only the component measurements (used for profiling captures)")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
@@ -447,7 +483,7 @@ def main():
     stream = torch.cuda.Stream()
     cb = hl.codebook("cuda")
     if args.only is not None:
-        parts = ("quantize", "gemm", "moe", "int4") if args.only == "components" else (args.only,)
+        parts = ("quantize", "gemm", "moe", "int4", "kv") if args.only == "components" else (args.only,)
         print(json.dumps({"components": components(hl, cb, peaks, stream, parts)}), flush=True)
         return
     # 64 distinct layers (quantized on the device from seeded synthetic weights)

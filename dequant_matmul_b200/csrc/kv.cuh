@@ -212,15 +212,17 @@ kv_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restr
   }
 }
 
-// Rotated queries in shared memory: value p of query m at m * 264 + p + p / 32,
-// so the eight lanes of a key (positions 32 l8 + j) read eight banks.
-__host__ __device__ inline int kv_qpos(int m, int p) { return m * (kKvDim + 8) + p + (p >> 5); }
+// Rotated queries in shared memory: value p of query m at m * 288 + p + 4 (p / 32),
+// so a lane's 32 values are eight aligned 16-byte chunks and the eight lanes of
+// a key (positions 32 l8 + j) read disjoint banks with 16-byte loads.
+constexpr int kKvQRow = kKvDim + 32;
+__host__ __device__ inline int kv_qpos(int m, int p) { return m * kKvQRow + p + 4 * (p >> 5); }
 
 __global__ void __launch_bounds__(kKvThreads)
 kv_scores_kernel(const uint16_t* __restrict__ Q, int m_count, int64_t ldq, const uint8_t* __restrict__ packed,
                  const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t n,
                  float* __restrict__ S, int64_t lds) {
-  extern __shared__ __align__(16) float qs[];  // [m_count][264]
+  extern __shared__ __align__(16) float qs[];  // [m_count][288]
   __shared__ float cb[kKvLevels];
   kv_check_codebook(codebook);
   if (threadIdx.x < kKvLevels) cb[threadIdx.x] = __ldg(codebook + threadIdx.x);
@@ -259,10 +261,16 @@ kv_scores_kernel(const uint16_t* __restrict__ Q, int m_count, int64_t ldq, const
 #pragma unroll
     for (int e = 0; e < 32; ++e) c[e] = cb[kv_code(w, e)];
     for (int m = 0; m < m_count; ++m) {
-      const float* qm = qs + kv_qpos(m, 32 * l8);
+      const float4* qm = reinterpret_cast<const float4*>(qs + kv_qpos(m, 32 * l8));
       float acc = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) acc = fmaf(c[e], qm[e], acc);
+      for (int i = 0; i < 8; ++i) {
+        const float4 t = qm[i];
+        acc = fmaf(c[4 * i], t.x, acc);
+        acc = fmaf(c[4 * i + 1], t.y, acc);
+        acc = fmaf(c[4 * i + 2], t.z, acc);
+        acc = fmaf(c[4 * i + 3], t.w, acc);
+      }
       acc = oct_sum(acc);
       if (active && l8 == 0) S[static_cast<int64_t>(m) * lds + r] = acc * sc;
     }
@@ -291,11 +299,11 @@ int launch_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const flo
 
 int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
                      const float* codebook, int64_t n, float* S, int64_t lds, cudaStream_t stream) {
-  const int smem = static_cast<int>(m) * (kKvDim + 8) * 4;
+  const int smem = static_cast<int>(m) * kKvQRow * 4;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kv_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kKvMaxQueries * (kKvDim + 8) * 4) != cudaSuccess)
+                             kKvMaxQueries * kKvQRow * 4) != cudaSuccess)
       return HLWQ_ECUDA;
     attr = true;
   }
