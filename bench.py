@@ -185,7 +185,7 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, steps: int, ms_total_max
 
 
 # ---------------------------------------------------------------- components (N = 1)
-def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", "kv")):
+def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", "kv", "codes")):
     import torch
     from dequant_matmul_b200 import synth
     out = {}
@@ -202,6 +202,8 @@ def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", 
         out.update(bench_int4(hl, cb, peaks, stream))
     if "kv" in parts:
         out.update(bench_kv(hl, peaks, stream))
+    if "codes" in parts:
+        out.update(bench_codes(hl, cb, peaks, stream))
     return out
 
 
@@ -299,6 +301,29 @@ def bench_int4(hl, cb, peaks, stream):
     return {"requantize_int4_27648x5120": {"ms": round(ms, 4), "gweights_per_s": round(O3 * I3 / ms / 1e6, 2),
                                            "gbs": round(gbs, 1), "hbm_frac": frac(gbs, peaks["hbm_gbs"]),
                                            "algo_bytes": byts}}
+
+
+def bench_codes(hl, cb, peaks, stream):
+    import torch
+    from dequant_matmul_b200 import synth
+    # One-code-per-byte layout of the 27648 x 5120 layer, both directions.
+    O3, I3 = 27648, 5120
+    nb = I3 // 128
+    w = synth.student_t_device((O3, I3), seed=97)
+    packed, _ = hl.quantize(w, cb, stream=stream)
+    del w
+    codes = torch.empty(O3, nb, 128, dtype=torch.uint8, device="cuda")
+    back = torch.empty_like(packed)
+    res = {}
+    byts = O3 * nb * (80 + 128)
+    ms, _ = time_graph(lambda: hl.codes_unpack(packed, codes, stream=stream), reps=10, warmup=3, stream=stream)
+    res["unpack"] = {"ms": round(ms, 4), "gbs": round(byts / ms / 1e6, 1), "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
+    ms, _ = time_graph(lambda: hl.codes_pack(codes, back, stream=stream), reps=10, warmup=3, stream=stream)
+    res["pack"] = {"ms": round(ms, 4), "gbs": round(byts / ms / 1e6, 1), "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
+    torch.cuda.synchronize()
+    res["round_trip_equal"] = bool(torch.equal(back, packed))
+    del packed, codes, back
+    return {"codes_int8_27648x5120": res}
 
 
 def bench_kv(hl, peaks, stream):
@@ -444,7 +469,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv"], default=None,
+    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv", "codes"], default=None,
                     help="run only the component measurements (used for profiling captures)")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
@@ -483,7 +508,7 @@ def main():
     stream = torch.cuda.Stream()
     cb = hl.codebook("cuda")
     if args.only is not None:
-        parts = ("quantize", "gemm", "moe", "int4", "kv") if args.only == "components" else (args.only,)
+        parts = ("quantize", "gemm", "moe", "int4", "kv", "codes") if args.only == "components" else (args.only,)
         print(json.dumps({"components": components(hl, cb, peaks, stream, parts)}), flush=True)
         return
     # 64 distinct layers (quantized on the device from seeded synthetic weights)

@@ -15,6 +15,8 @@ int launch_quantize(const void* W, bool bf16, int64_t rows, int in, const float*
                     uint16_t* norms, cudaStream_t stream);
 int launch_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows, int in,
                       void* out, bool bf16, cudaStream_t stream);
+int launch_codes_unpack(const uint8_t* packed, int64_t nblocks, uint8_t* codes, cudaStream_t stream);
+int launch_codes_pack(const uint8_t* codes, int64_t nblocks, uint8_t* packed, cudaStream_t stream);
 int launch_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows,
                            int in, uint8_t* q4, uint16_t* scale, uint16_t* zero, cudaStream_t stream);
 int launch_kv_quantize(const uint16_t* X, int64_t n, int64_t ldx, const float* codebook, uint8_t* packed,
@@ -71,6 +73,18 @@ extern "C" int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, con
     return HLWQ_EALIGN;
   return hlwq::launch_dequantize(packed, norms, codebook, rows, static_cast<int>(in), W_out, odtype == HLWQ_BF16,
                                  as_stream(stream));
+}
+
+extern "C" int hlwq_codes_unpack(const uint8_t* packed, int64_t nblocks, uint8_t* codes, void* stream) {
+  if (!packed || !codes || nblocks <= 0 || nblocks > (int64_t(1) << 40)) return HLWQ_EINVAL;
+  if (!aligned16(packed) || !aligned16(codes)) return HLWQ_EALIGN;
+  return hlwq::launch_codes_unpack(packed, nblocks, codes, as_stream(stream));
+}
+
+extern "C" int hlwq_codes_pack(const uint8_t* codes, int64_t nblocks, uint8_t* packed, void* stream) {
+  if (!packed || !codes || nblocks <= 0 || nblocks > (int64_t(1) << 40)) return HLWQ_EINVAL;
+  if (!aligned16(packed) || !aligned16(codes)) return HLWQ_EALIGN;
+  return hlwq::launch_codes_pack(codes, nblocks, packed, as_stream(stream));
 }
 
 extern "C" int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook,

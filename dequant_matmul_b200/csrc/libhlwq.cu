@@ -8,4 +8,5 @@
 #include "gemm_tc.cuh"
 #include "int4.cuh"
 #include "kv.cuh"
+#include "codes.cuh"
 #include "api.cuh"

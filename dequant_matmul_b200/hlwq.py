@@ -22,6 +22,7 @@ NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 + 64 * 1024
 HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
 HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
 HLWQ_FLAG_WEIGHTS_STATIC = 1
+DEVERR_CODEBOOK, DEVERR_TIMEOUT, DEVERR_CODE_RANGE = 0x1, 0x2, 0x4
 BLOCK, BLOCK_BYTES, LEVELS = 128, 80, 32
 
 # (name, restype, argtypes) for every symbol include/hlwq.h declares.
@@ -30,6 +31,8 @@ SIGNATURES = {
     "hlwq_lloyd_codebook": (_I, [_I, _P, _P, _P]),
     "hlwq_quantize": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
+    "hlwq_codes_unpack": (_I, [_P, _I64, _P, _P]),
+    "hlwq_codes_pack": (_I, [_P, _I64, _P, _P]),
     "hlwq_requantize_int4": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_dequantize": (_I, [_P, _P, _P, _I64, _P, _I, _P]),
@@ -165,6 +168,30 @@ def dequantize(packed, norms, cb, in_features: int, out_dtype=torch.float32, out
     _check(lib.hlwq_dequantize(_ptr(packed), _ptr(norms), _ptr(cb), rows, in_features, _ptr(out),
                                _dtype_code(out.dtype), _stream(stream)), "hlwq_dequantize")
     return out
+
+
+def codes_unpack(packed, codes=None, stream=None):
+    """packed uint8 [..., NB, 80] -> codes uint8 [..., NB, 128], one code per byte."""
+    _cuda(packed, "packed")
+    if packed.shape[-1] != BLOCK_BYTES:
+        raise HLWQError("packed must end in 80-byte blocks")
+    nblocks = packed.numel() // BLOCK_BYTES
+    if codes is None:
+        codes = torch.empty(tuple(packed.shape[:-1]) + (BLOCK,), dtype=torch.uint8, device=packed.device)
+    _check(lib.hlwq_codes_unpack(_ptr(packed), nblocks, _ptr(codes), _stream(stream)), "hlwq_codes_unpack")
+    return codes
+
+
+def codes_pack(codes, packed=None, stream=None):
+    """codes uint8 [..., NB, 128] (0..31) -> packed uint8 [..., NB, 80]."""
+    _cuda(codes, "codes")
+    if codes.shape[-1] != BLOCK:
+        raise HLWQError("codes must end in blocks of 128")
+    nblocks = codes.numel() // BLOCK
+    if packed is None:
+        packed = torch.empty(tuple(codes.shape[:-1]) + (BLOCK_BYTES,), dtype=torch.uint8, device=codes.device)
+    _check(lib.hlwq_codes_pack(_ptr(codes), nblocks, _ptr(packed), _stream(stream)), "hlwq_codes_pack")
+    return packed
 
 
 def requantize_int4(packed, norms, cb, in_features: int, q4=None, scale=None, zero=None, stream=None):

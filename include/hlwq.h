@@ -71,6 +71,7 @@ typedef enum { HLWQ_FLAG_WEIGHTS_STATIC = 1 } hlwq_flags;
 /* Device error bits (hlwq_device_error). */
 #define HLWQ_DEVERR_CODEBOOK 0x1u  /* codebook not strictly ascending or not finite */
 #define HLWQ_DEVERR_TIMEOUT  0x2u  /* a bounded in-kernel wait gave up */
+#define HLWQ_DEVERR_CODE_RANGE 0x4u  /* hlwq_codes_pack met a code above 31 */
 
 /*
  * Lloyd-Max codebook for N(0,1) (Method step [4]: "Lloyd-Max 5-bit quantization
@@ -109,6 +110,20 @@ int hlwq_quantize(const void* W, int wdtype, int64_t rows, int64_t in,
  */
 int hlwq_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook,
                     int64_t rows, int64_t in, void* W_out, int odtype, void* stream);
+
+/*
+ * One-code-per-byte layout ("Gemma-4-26B-A4B-it-HLWQ-Q5", Technical Details:
+ * codes stored as int8, one per byte) <-> the packed 5-bit stream (Method
+ * step [5]).  nblocks = rows * NB blocks of 128 codes.
+ *   codes   device uint8 [nblocks][128], values 0..31 (16-byte aligned)
+ *   packed  device uint8 [nblocks][80] (16-byte aligned)
+ * hlwq_codes_unpack writes codes from packed; hlwq_codes_pack writes packed
+ * from codes, storing the low five bits of a code above 31 and setting
+ * HLWQ_DEVERR_CODE_RANGE.  The norms are the same array in both layouts.
+ * Errors: HLWQ_EINVAL (NULL, nblocks <= 0 or above 2^40), HLWQ_EALIGN, HLWQ_ECUDA.
+ */
+int hlwq_codes_unpack(const uint8_t* packed, int64_t nblocks, uint8_t* codes, void* stream);
+int hlwq_codes_pack(const uint8_t* codes, int64_t nblocks, uint8_t* packed, void* stream);
 
 /*
  * Q5 -> INT4 re-encoding ("Qwopus3.6-27B-v2 . HLWQ Q5", Pipeline: dequantize

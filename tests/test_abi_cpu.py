@@ -63,6 +63,10 @@ def test_validation_before_launch(hl):
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, None, p, p, None) == hl.HLWQ_EINVAL
     assert L.hlwq_requantize_int4(p, p, p, 4, 704, p, p, p, None) == hl.HLWQ_EUNSUPPORTED  # not 128-aligned
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, ctypes.c_void_p(264), p, p, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_codes_unpack(p, 0, p, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_codes_pack(None, 4, p, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_codes_pack(p, 4, ctypes.c_void_p(264), None) == hl.HLWQ_EALIGN
+    assert L.hlwq_codes_unpack(ctypes.c_void_p(260), 4, p, None) == hl.HLWQ_EALIGN
     assert L.hlwq_kv_quantize(p, 4, 128, p, p, p, None) == hl.HLWQ_EINVAL             # ldx < 256
     assert L.hlwq_kv_dequantize(p, p, p, 4, p, hl.HLWQ_F16, None) == hl.HLWQ_EUNSUPPORTED
     assert L.hlwq_kv_scores(p, 65, 256, p, p, p, 4, p, 4, None) == hl.HLWQ_EUNSUPPORTED  # > 64 queries
