@@ -14,6 +14,9 @@ Distributions (the pages quantize BF16 checkpoints of these models):
     chi2_4 = -2 ln(u1 u2); fp32 or rounded to bf16.
   * ``activations``: N(0, 1) rounded to bf16.
   * ``router_logits``: N(0, 1) fp32.
+  * ``sign_vectors``: the two +-1 vectors of length 128 of the TQ3 rotation,
+    fair coin flips (the producer's own generator for its seed is not known;
+    these stand in for it).
 """
 
 from __future__ import annotations
@@ -66,6 +69,12 @@ def activations(rows: int, cols: int, seed: int = 1, dtype=torch.bfloat16) -> to
 def router_logits(tokens: int, experts: int, seed: int = 2) -> torch.Tensor:
     rng = _rng(seed)
     return torch.from_numpy(rng.standard_normal((tokens, experts), dtype=np.float32))
+
+
+def sign_vectors(seed: int = 42) -> torch.Tensor:
+    """int8 [2][128] of +-1: row 0 is applied before the FWHT, row 1 after it."""
+    bits = _rng(seed).integers(0, 2, size=(2, 128))
+    return torch.from_numpy((1 - 2 * bits).astype(np.int8))
 
 
 def uniform(shape, lo: float, hi: float, seed: int) -> np.ndarray:

@@ -6,3 +6,5 @@ from .int4_oracle import *  # noqa: F401,F403,E402
 from . import int4_oracle  # noqa: F401,E402
 from .kv_oracle import *  # noqa: F401,F403,E402
 from . import kv_oracle  # noqa: F401,E402
+from .tq3_oracle import *  # noqa: F401,F403,E402
+from . import tq3_oracle  # noqa: F401,E402
