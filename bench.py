@@ -185,7 +185,7 @@ def whole_job_gbs(world: int, bytes_per_rank_step: int, steps: int, ms_total_max
 
 
 # ---------------------------------------------------------------- components (N = 1)
-def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", "kv", "codes")):
+def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", "kv", "codes", "tq3")):
     import torch
     from dequant_matmul_b200 import synth
     out = {}
@@ -204,6 +204,8 @@ def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", 
         out.update(bench_kv(hl, peaks, stream))
     if "codes" in parts:
         out.update(bench_codes(hl, cb, peaks, stream))
+    if "tq3" in parts:
+        out.update(bench_tq3(hl, peaks, stream))
     return out
 
 
@@ -324,6 +326,64 @@ def bench_codes(hl, cb, peaks, stream):
     res["round_trip_equal"] = bool(torch.equal(back, packed))
     del packed, codes, back
     return {"codes_int8_27648x5120": res}
+
+
+def bench_tq3(hl, peaks, stream):
+    import torch
+    from dequant_matmul_b200 import synth
+    # TQ3 (3-bit HIGGS) weights: quantize the 27648 x 5120 layer; decode GEMV at
+    # 5120 x 5120 and 27648 x 5120 over enough weight copies to exceed L2.
+    cb8 = hl.kv_codebook("cuda")
+    signs = synth.sign_vectors(42).cuda()
+    res = {}
+    O3, I3 = 27648, 5120
+    nb = I3 // 128
+    w = synth.student_t_device((O3, I3), seed=98)
+    packed = torch.empty(O3, nb, 48, dtype=torch.uint8, device="cuda")
+    norms = torch.empty(O3, nb, dtype=torch.float32, device="cuda")
+    ms, _ = time_graph(lambda: hl.tq3_quantize(w, signs, cb8, packed, norms, stream=stream), reps=5, warmup=3,
+                       stream=stream)
+    b = O3 * I3 * 2 + O3 * nb * (48 + 4)
+    res["quantize_27648x5120"] = {"ms": round(ms, 4), "gweights_per_s": round(O3 * I3 / ms / 1e6, 2),
+                                  "gbs": round(b / ms / 1e6, 1), "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
+    out16 = torch.empty(O3, I3, dtype=torch.bfloat16, device="cuda")
+    ms, _ = time_graph(lambda: hl.tq3_dequantize(packed, norms, signs, cb8, I3, out=out16, stream=stream), reps=5,
+                       warmup=3, stream=stream)
+    b = O3 * nb * (48 + 4) + O3 * I3 * 2
+    res["dequantize_bf16_27648x5120"] = {"ms": round(ms, 4), "gbs": round(b / ms / 1e6, 1),
+                                         "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
+    del out16
+    for (Og, Ig) in ((5120, 5120), (27648, 5120)):
+        nbg = Ig // 128
+        wbytes = Og * nbg * (48 + 4)
+        ncopy = max(2, -(-(320 << 20) // wbytes))
+        copies = []
+        for c in range(ncopy):
+            if Og == O3 and c == 0:
+                copies.append((packed, norms))
+                continue
+            wc = synth.student_t_device((Og, Ig), seed=100 + c) if c < 2 else None
+            if wc is not None:
+                copies.append(hl.tq3_quantize(wc, signs, cb8, stream=stream))
+                del wc
+            else:  # further copies: same codes at other addresses
+                copies.append((copies[c % 2][0].clone(), copies[c % 2][1].clone()))
+        x = synth.activations_device(1, Ig, seed=101)[0]
+        y = torch.empty(Og, dtype=torch.float32, device="cuda")
+
+        def run():
+            for p, n in copies:
+                hl.tq3_gemv(p, n, signs, cb8, x, y=y, stream=stream)
+
+        ms, _ = time_graph(run, reps=20, warmup=3, stream=stream)
+        ms /= len(copies)
+        b = wbytes + Ig * 2 + Og * 4
+        res[f"gemv_{Og}x{Ig}"] = {"ms": round(ms, 5), "us": round(ms * 1e3, 2), "gbs": round(b / ms / 1e6, 1),
+                                  "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"]), "copies": len(copies),
+                                  "algo_bytes": b}
+        del copies
+    del w, packed, norms
+    return {"tq3": res}
 
 
 def bench_kv(hl, peaks, stream):
@@ -469,7 +529,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv", "codes"], default=None,
+    ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv", "codes", "tq3"], default=None,
                     help="run only the component measurements (used for profiling captures)")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
@@ -508,7 +568,7 @@ def main():
     stream = torch.cuda.Stream()
     cb = hl.codebook("cuda")
     if args.only is not None:
-        parts = ("quantize", "gemm", "moe", "int4", "kv", "codes") if args.only == "components" else (args.only,)
+        parts = ("quantize", "gemm", "moe", "int4", "kv", "codes", "tq3") if args.only == "components" else (args.only,)
         print(json.dumps({"components": components(hl, cb, peaks, stream, parts)}), flush=True)
         return
     # 64 distinct layers (quantized on the device from seeded synthetic weights)

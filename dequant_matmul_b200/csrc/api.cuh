@@ -17,6 +17,12 @@ int launch_dequantize(const uint8_t* packed, const uint16_t* norms, const float*
                       void* out, bool bf16, cudaStream_t stream);
 int launch_codes_unpack(const uint8_t* packed, int64_t nblocks, uint8_t* codes, cudaStream_t stream);
 int launch_codes_pack(const uint8_t* codes, int64_t nblocks, uint8_t* packed, cudaStream_t stream);
+int launch_tq3_quantize(const uint16_t* W, int64_t rows, int in, const int8_t* signs, const float* codebook,
+                        uint8_t* packed, float* norms, cudaStream_t stream);
+int launch_tq3_dequantize(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook,
+                          int64_t rows, int in, void* out, bool bf16, cudaStream_t stream);
+int launch_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook,
+                    int64_t O, int in, const uint16_t* x, void* y, bool out_bf16, cudaStream_t stream);
 int launch_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t rows,
                            int in, uint8_t* q4, uint16_t* scale, uint16_t* zero, cudaStream_t stream);
 int launch_kv_quantize(const uint16_t* X, int64_t n, int64_t ldx, const float* codebook, uint8_t* packed,
@@ -85,6 +91,40 @@ extern "C" int hlwq_codes_pack(const uint8_t* codes, int64_t nblocks, uint8_t* p
   if (!packed || !codes || nblocks <= 0 || nblocks > (int64_t(1) << 40)) return HLWQ_EINVAL;
   if (!aligned16(packed) || !aligned16(codes)) return HLWQ_EALIGN;
   return hlwq::launch_codes_pack(codes, nblocks, packed, as_stream(stream));
+}
+
+extern "C" int hlwq_tq3_quantize(const uint16_t* W, int64_t rows, int64_t in, const int8_t* signs,
+                                 const float* codebook8, uint8_t* packed, float* norms, void* stream) {
+  if (!W || !signs || !codebook8 || !packed || !norms || rows <= 0 || in <= 0 || in > kMaxIn) return HLWQ_EINVAL;
+  if (!aligned2(W) || (reinterpret_cast<uintptr_t>(packed) & 3u) || (reinterpret_cast<uintptr_t>(norms) & 3u))
+    return HLWQ_EALIGN;
+  return hlwq::launch_tq3_quantize(W, rows, static_cast<int>(in), signs, codebook8, packed, norms, as_stream(stream));
+}
+
+extern "C" int hlwq_tq3_dequantize(const uint8_t* packed, const float* norms, const int8_t* signs,
+                                   const float* codebook8, int64_t rows, int64_t in, void* W_out, int odtype,
+                                   void* stream) {
+  if (!packed || !norms || !signs || !codebook8 || !W_out || rows <= 0 || in <= 0 || in > kMaxIn)
+    return HLWQ_EINVAL;
+  if (odtype != HLWQ_F32 && odtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(packed) & 3u) || (reinterpret_cast<uintptr_t>(norms) & 3u) || !aligned2(W_out) ||
+      (odtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(W_out) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_tq3_dequantize(packed, norms, signs, codebook8, rows, static_cast<int>(in), W_out,
+                                     odtype == HLWQ_BF16, as_stream(stream));
+}
+
+extern "C" int hlwq_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook8,
+                             int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype, void* stream) {
+  if (!packed || !norms || !signs || !codebook8 || !x || !y || out <= 0 || in <= 0 || in > kMaxIn ||
+      out > (int64_t(1) << 40))
+    return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(packed) & 3u) || (reinterpret_cast<uintptr_t>(norms) & 3u) || !aligned2(x) ||
+      !aligned2(y) || (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(y) & 3u)))
+    return HLWQ_EALIGN;
+  return hlwq::launch_tq3_gemv(packed, norms, signs, codebook8, out, static_cast<int>(in), x, y, ydtype == HLWQ_BF16,
+                               as_stream(stream));
 }
 
 extern "C" int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const float* codebook,

@@ -9,4 +9,5 @@
 #include "int4.cuh"
 #include "kv.cuh"
 #include "codes.cuh"
+#include "tq3.cuh"
 #include "api.cuh"

@@ -33,6 +33,9 @@ SIGNATURES = {
     "hlwq_dequantize": (_I, [_P, _P, _P, _I64, _I64, _P, _I, _P]),
     "hlwq_codes_unpack": (_I, [_P, _I64, _P, _P]),
     "hlwq_codes_pack": (_I, [_P, _I64, _P, _P]),
+    "hlwq_tq3_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "hlwq_tq3_dequantize": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _I, _P]),
+    "hlwq_tq3_gemv": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
     "hlwq_requantize_int4": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_dequantize": (_I, [_P, _P, _P, _I64, _P, _I, _P]),
@@ -192,6 +195,51 @@ def codes_pack(codes, packed=None, stream=None):
         packed = torch.empty(tuple(codes.shape[:-1]) + (BLOCK_BYTES,), dtype=torch.uint8, device=codes.device)
     _check(lib.hlwq_codes_pack(_ptr(codes), nblocks, _ptr(packed), _stream(stream)), "hlwq_codes_pack")
     return packed
+
+
+def tq3_quantize(W: torch.Tensor, signs: torch.Tensor, cb8, packed=None, norms=None, stream=None):
+    """W bf16 [..., in] (leading dims are stacked rows), signs int8 [2][128]
+    (+-1; row 0 before the FWHT, row 1 after) -> (packed uint8 [..., NB, 48],
+    norms float32 [..., NB]: the shape-gain norms)."""
+    _cuda(W, "W")
+    _cuda(signs, "signs")
+    if W.dtype != torch.bfloat16 or signs.dtype != torch.int8 or signs.numel() != 2 * BLOCK:
+        raise HLWQError("tq3_quantize takes bf16 weights and int8 signs [2][128]")
+    in_f = W.shape[-1]
+    rows = W.numel() // in_f
+    nb = n_blocks(in_f)
+    lead = tuple(W.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (nb, 48), dtype=torch.uint8, device=W.device)
+    if norms is None:
+        norms = torch.empty(lead + (nb,), dtype=torch.float32, device=W.device)
+    _check(lib.hlwq_tq3_quantize(_ptr(W), rows, in_f, _ptr(signs), _ptr(cb8), _ptr(packed), _ptr(norms),
+                                 _stream(stream)), "hlwq_tq3_quantize")
+    return packed, norms
+
+
+def tq3_dequantize(packed, norms, signs, cb8, in_features: int, out_dtype=torch.float32, out=None, stream=None):
+    """-> W_hat [..., in] (the pad dropped)."""
+    _cuda(packed, "packed")
+    nb = packed.shape[-2]
+    lead = tuple(packed.shape[:-2])
+    rows = packed.numel() // (nb * 48)
+    if out is None:
+        out = torch.empty(lead + (in_features,), dtype=out_dtype, device=packed.device)
+    _check(lib.hlwq_tq3_dequantize(_ptr(packed), _ptr(norms), _ptr(signs), _ptr(cb8), rows, in_features, _ptr(out),
+                                   _dtype_code(out.dtype), _stream(stream)), "hlwq_tq3_dequantize")
+    return out
+
+
+def tq3_gemv(packed, norms, signs, cb8, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None):
+    """x bf16 [in] -> y [out] = W_hat @ x (fp32 accumulation)."""
+    _cuda(x, "x")
+    out_f = packed.shape[0]
+    if y is None:
+        y = torch.empty(out_f, dtype=out_dtype, device=x.device)
+    _check(lib.hlwq_tq3_gemv(_ptr(packed), _ptr(norms), _ptr(signs), _ptr(cb8), out_f, x.shape[-1], _ptr(x), _ptr(y),
+                             _dtype_code(y.dtype), _stream(stream)), "hlwq_tq3_gemv")
+    return y
 
 
 def requantize_int4(packed, norms, cb, in_features: int, q4=None, scale=None, zero=None, stream=None):

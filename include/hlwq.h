@@ -172,6 +172,37 @@ int hlwq_kv_scores(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* pac
                    const float* codebook8, int64_t n, float* scores, int64_t lds, void* stream);
 
 /*
+ * TQ3 weights, the scalar case of HIGGS ("Qwen3.6-35B-A3B-TQ3-native", "What
+ * TQ3 actually does" and "Files").  Per row and group g of 128 inputs (the
+ * tail zero-padded), with one pair of sign vectors for every group:
+ *   y      = s2 * (H128 (s1 * g)) / ||g||       (H128 the +-1 Sylvester matrix)
+ *   code_j = nearest of the 8 Lloyd-Max centroids (ties to the lower index),
+ *            decided in fp64
+ *   gamma  = ||g|| / sqrt(||c[code]||^2 / 128)   (shape-gain norm; 0 for a zero
+ *            group; ||c[code]||^2 = sum over levels l = 0..7 of
+ *            count_l * c_l^2 in fp64, in that order), rounded to fp32
+ *   w_hat  = gamma * s1 * (H128 (s2 * c[code])) / 128
+ *   signs     device int8 [2][128]: row 0 = s1, row 1 = s2; a negative byte
+ *             is -1, any other value +1
+ *   codebook8 device float32 [8] (hlwq_lloyd_codebook(8))
+ *   packed    [rows][NB][48]: code j of a group at bits [3j, 3j+3), LSB first
+ *   norms     float32 [rows][NB] (gamma)
+ * hlwq_tq3_quantize: W bf16 [rows][in] (row pitch in) -> packed, norms.
+ * hlwq_tq3_dequantize: -> W_out [rows][in] (HLWQ_F32 or HLWQ_BF16).
+ * hlwq_tq3_gemv: y[o] = sum_i x[i] w_hat[o][i] for one bf16 activation
+ *   x [in], fp32 accumulation, evaluated in the rotated domain (x rotated
+ *   once); one launch of thread-block clusters, no workspace.
+ * Errors: HLWQ_EINVAL, HLWQ_EALIGN (packed / norms 4-byte, W / x / y 2-byte,
+ * f32 outputs 4-byte alignment), HLWQ_EUNSUPPORTED (dtype), HLWQ_ECUDA.
+ */
+int hlwq_tq3_quantize(const uint16_t* W, int64_t rows, int64_t in, const int8_t* signs, const float* codebook8,
+                      uint8_t* packed, float* norms, void* stream);
+int hlwq_tq3_dequantize(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook8,
+                        int64_t rows, int64_t in, void* W_out, int odtype, void* stream);
+int hlwq_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook8,
+                  int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype, void* stream);
+
+/*
  * Decode GEMV: y[o] = sum_i x[i] * w_hat[o][i], fp32 accumulation, without
  * materialising w_hat (the activation is rotated once per 128-block and dotted
  * with centroid values in the rotated domain).
