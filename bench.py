@@ -353,7 +353,7 @@ def bench_tq3(hl, peaks, stream):
     res["dequantize_bf16_27648x5120"] = {"ms": round(ms, 4), "gbs": round(b / ms / 1e6, 1),
                                          "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
     del out16
-    for (Og, Ig) in ((5120, 5120), (27648, 5120)):
+    for (Og, Ig) in ((27648, 5120), (5120, 5120)):
         nbg = Ig // 128
         wbytes = Og * nbg * (48 + 4)
         ncopy = max(2, -(-(320 << 20) // wbytes))

@@ -36,6 +36,8 @@
 // cluster barrier, every CTA adds up a part of the rows over the cluster's
 // CTAs in rank order through distributed shared memory and writes y.
 
+#include <utility>
+
 #include "hlwq_common.cuh"
 
 namespace hlwq {
@@ -167,12 +169,11 @@ tq3_dequantize_kernel(const uint8_t* __restrict__ packed, const float* __restric
                       const int8_t* __restrict__ signs, const float* __restrict__ codebook, int64_t rows, int in,
                       int nb, void* __restrict__ out) {
   __shared__ float cb[kT3Levels];
-  __shared__ float sg[2 * kBlock];
   t3_check_codebook(codebook);
   if (threadIdx.x < kT3Levels) cb[threadIdx.x] = __ldg(codebook + threadIdx.x);
-  if (threadIdx.x < 2 * kBlock) sg[threadIdx.x] = __ldg(signs + threadIdx.x) < 0 ? -1.0f : 1.0f;
   __syncthreads();
   const int lane = threadIdx.x & 31, q = lane & 3;
+  const uint32_t m1 = t3_sign_mask(signs, 32 * q), m2 = t3_sign_mask(signs, kBlock + 32 * q);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kT3QThreads + threadIdx.x) >> 5;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kT3QThreads / 32);
   const int64_t ngroups = rows * nb;
@@ -194,12 +195,15 @@ tq3_dequantize_kernel(const uint8_t* __restrict__ packed, const float* __restric
     }
     float v[32];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] = cb[kv_code(w, e)] * sg[kBlock + 32 * q + e];
+    for (int e = 0; e < 32; ++e) {
+      const float t = cb[kv_code(w, e)];
+      v[e] = (m2 >> e) & 1u ? -t : t;
+    }
     fwht_4lanes(v, lane);
     const int qlen = active ? max(0, min(32, in - kBlock * b - 32 * q)) : 0;
     if (qlen == 0) continue;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] *= sg[32 * q + e] * scale;
+    for (int e = 0; e < 32; ++e) v[e] *= (m1 >> e) & 1u ? -scale : scale;
     const int64_t off = o * static_cast<int64_t>(in) + static_cast<int64_t>(kBlock) * b + 32 * q;
     if constexpr (!kOutBf16) {
       float* dst = static_cast<float*>(out) + off;
@@ -241,7 +245,7 @@ constexpr int kT3SliceGroups = 8;                                // groups per s
 constexpr int kT3Slice = kT3SliceGroups * kBlock;                // 1024 inputs
 constexpr int kT3TableBytes = 16 * 64 * 32 * 4;                  // [pair][a + 8b][lane] fp32
 constexpr int kT3ChunkRows = 4096;                               // slice sums kept per pass
-constexpr int kT3SmemBytes = kT3TableBytes + kT3Slice * 4 + kT3ChunkRows * 4;
+constexpr int kT3SmemBytes = 8192 + kT3TableBytes + kT3Slice * 4 + kT3ChunkRows * 4;  // + alignment slack
 constexpr int kT3MaxCluster = 8;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -270,22 +274,59 @@ __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t ran
   return v;
 }
 
-// Byte offset, within the table block of pair p, of the entry for the code
-// pair in bits [6p, 6p + 6) of a lane's 96-bit string (w0, w1, w2): the
-// 6-bit index times 128 bytes, or'ed with the lane's 4-byte column.
-__device__ __forceinline__ uint32_t t3_pair_off(int p, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t lane4) {
-  const int bit = 6 * p, k = bit >> 5, sh = bit & 31;
-  uint32_t src;
-  int s;
-  if (sh <= 26) {
-    src = k == 0 ? w0 : (k == 1 ? w1 : w2);
-    s = sh;
+// Table lookup of pair P of a lane's 96-bit code string (w0, w1, w2): the
+// 6-bit field at bits [6P, 6P + 6) moved to bit 7 (index times 128 bytes) and
+// or'ed into `lb` (the 8 KiB-aligned table address with the lane's 4-byte
+// column) -- one shift and one lop3 -- then read at the immediate offset
+// P * 8192 of the pair's table block.
+template <int P>
+__device__ __forceinline__ float t3_lookup(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t lb) {
+  constexpr int bit = 6 * P, k = bit >> 5, sh = bit & 31;
+  const uint32_t lo = k == 0 ? w0 : (k == 1 ? w1 : w2);
+  float t;
+  if constexpr (sh > 26) {
+    // the field crosses into the next word: funnel shift it to bit 7
+    const uint32_t hi = k == 0 ? w1 : w2;
+    asm volatile(
+        "{ .reg .b32 a;\n\t"
+        "shf.r.clamp.b32 a, %1, %2, %3;\n\t"
+        "lop3.b32 a, a, 0x1f80, %4, 0xea;\n\t"
+        "ld.shared.f32 %0, [a+%5]; }"
+        : "=f"(t)
+        : "r"(lo), "r"(hi), "n"(sh - 7), "r"(lb), "n"(P * 8192));
+  } else if constexpr (sh >= 7) {
+    asm volatile(
+        "{ .reg .b32 a;\n\t"
+        "shr.b32 a, %1, %2;\n\t"
+        "lop3.b32 a, a, 0x1f80, %3, 0xea;\n\t"
+        "ld.shared.f32 %0, [a+%4]; }"
+        : "=f"(t)
+        : "r"(lo), "n"(sh - 7), "r"(lb), "n"(P * 8192));
   } else {
-    src = __funnelshift_r(k == 0 ? w0 : w1, k == 0 ? w1 : w2, sh);
-    s = 0;
+    asm volatile(
+        "{ .reg .b32 a;\n\t"
+        "shl.b32 a, %1, %2;\n\t"
+        "lop3.b32 a, a, 0x1f80, %3, 0xea;\n\t"
+        "ld.shared.f32 %0, [a+%4]; }"
+        : "=f"(t)
+        : "r"(lo), "n"(7 - sh), "r"(lb), "n"(P * 8192));
   }
-  const uint32_t f = s >= 7 ? (src >> (s - 7)) : (src << (7 - s));
-  return (f & 0x1f80u) | lane4;
+  return t;
+}
+
+template <int... P>
+__device__ __forceinline__ float t3_row_sum(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t lb,
+                                            std::integer_sequence<int, P...>) {
+  float t[sizeof...(P)] = {t3_lookup<P>(w0, w1, w2, lb)...};
+  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < static_cast<int>(sizeof...(P)); i += 4) {
+    a0 += t[i];
+    a1 += t[i + 1];
+    a2 += t[i + 2];
+    a3 += t[i + 3];
+  }
+  return (a0 + a1) + (a2 + a3);
 }
 
 // Eight values per lane -> the sum over the warp of value i, held by the lanes
@@ -308,18 +349,69 @@ __device__ __forceinline__ float t3_reduce8(float (&v)[8], int lane) {
   return r + __shfl_xor_sync(0xffffffffu, r, 2);
 }
 
+// Codes and norms of the eight rows c0 + 8g .. c0 + 8g + 7 for the lane's
+// group gb (zeros where a row or the group does not exist).
+__device__ __forceinline__ void t3_load_rows(const uint8_t* __restrict__ packed, const float* __restrict__ norms,
+                                             int64_t c0, int g, int nrows, int nb, int gb, bool gvalid, int q,
+                                             uint32_t (&w)[8][3], float (&gm)[8]) {
+  const int64_t first = c0 + 8 * g;
+  const uint8_t* pc = packed + (first * nb + gb) * kT3GroupBytes + 12 * q;
+  const float* pn = norms + first * nb + gb;
+  const int64_t rs = static_cast<int64_t>(nb) * kT3GroupBytes;
+  if (gvalid && 8 * g + 8 <= nrows) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(pc + i * rs);
+      w[i][0] = __ldg(src);
+      w[i][1] = __ldg(src + 1);
+      w[i][2] = __ldg(src + 2);
+      gm[i] = __ldg(pn + static_cast<int64_t>(i) * nb);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[i][0] = w[i][1] = w[i][2] = 0u;
+      gm[i] = 0.0f;
+      if (gvalid && 8 * g + i < nrows) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(pc + i * rs);
+        w[i][0] = __ldg(src);
+        w[i][1] = __ldg(src + 1);
+        w[i][2] = __ldg(src + 2);
+        gm[i] = __ldg(pn + static_cast<int64_t>(i) * nb);
+      }
+    }
+  }
+}
+
+// Sums of eight rows' shares (rows i0 .. i0 + 7 of the pass) into acc.
+__device__ __forceinline__ void t3_rows_step(const uint32_t (&w)[8][3], const float (&gm)[8], uint32_t lb, int lane,
+                                             int q, int i0, int nrows, float* acc) {
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    v[i] = t3_row_sum(w[i][0], w[i][1], w[i][2], lb, std::make_integer_sequence<int, 16>{}) * gm[i];
+  const float r = t3_reduce8(v, lane);
+  const int i = i0 + (lane >> 2);
+  if (q == 0 && i < nrows) acc[i] += r;
+}
+
 __global__ void __launch_bounds__(kT3GThreads, 1)
 tq3_gemv_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ norms,
                 const int8_t* __restrict__ signs, const float* __restrict__ codebook, int64_t O, int in, int nb,
                 int nslices, int64_t rows_per_cluster, const uint16_t* __restrict__ x, void* __restrict__ y,
                 int out_bf16, int xvec) {
   extern __shared__ __align__(16) unsigned char t3s[];
-  float* xr = reinterpret_cast<float*>(t3s + kT3TableBytes);
+  // the table starts on an 8 KiB boundary, so a lookup address is the
+  // table's address or'ed with the lane column and the code-pair index
+  const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(t3s));
+  const uint32_t pad = (8192u - (raw & 8191u)) & 8191u;
+  unsigned char* tbl = t3s + pad;
+  float* xr = reinterpret_cast<float*>(tbl + kT3TableBytes);
   float* acc = xr + kT3Slice;
   const uint32_t C = cluster_size(), rank = cluster_rank();
   const int64_t cid = blockIdx.x / C;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, q = lane & 3;
-  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+  const uint32_t lb = (raw + pad) | (static_cast<uint32_t>(lane) * 4u);
   t3_check_codebook(codebook);
   float c[kT3Levels];
 #pragma unroll
@@ -330,9 +422,13 @@ tq3_gemv_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ no
     const int nrows = static_cast<int>(min(static_cast<int64_t>(kT3ChunkRows), r1 - c0));
     for (int i = threadIdx.x; i < nrows; i += kT3GThreads) acc[i] = 0.0f;
     for (int s = static_cast<int>(rank); s < nslices; s += static_cast<int>(C)) {
-      __syncthreads();  // readers of the previous table are done; acc is zeroed
       const int gb = s * kT3SliceGroups + (lane >> 2);
       const bool gvalid = gb < nb;
+      // the first rows' codes are requested before the table is built
+      uint32_t wc[8][3];
+      float gc[8];
+      t3_load_rows(packed, norms, c0, warp, nrows, nb, gb, gvalid, q, wc, gc);
+      __syncthreads();  // readers of the previous table are done; acc is zeroed
       if (warp == 0) {
         // xt for the slice: lane holds positions 32 lane .. 32 lane + 31
         float v[32];
@@ -373,7 +469,7 @@ tq3_gemv_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ no
       {
         // table block of pair p = warp: entry [a + 8b][lane] = c[a] xt[2p] + c[b] xt[2p + 1]
         const float2 xx = *reinterpret_cast<const float2*>(xr + 32 * lane + 2 * warp);
-        float* tb = reinterpret_cast<float*>(t3s + warp * 8192) + lane;
+        float* tb = reinterpret_cast<float*>(tbl + warp * 8192) + lane;
 #pragma unroll
         for (int b = 0; b < kT3Levels; ++b) {
           const float hb = c[b] * xx.y;
@@ -382,39 +478,16 @@ tq3_gemv_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ no
         }
       }
       __syncthreads();
-      for (int g = warp; 8 * g < nrows; g += kT3GWarps) {
-        uint32_t w[8][3];
-        float gm[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          w[i][0] = w[i][1] = w[i][2] = 0u;
-          gm[i] = 0.0f;
-          if (gvalid && 8 * g + i < nrows) {
-            const int64_t row = c0 + 8 * g + i;
-            const int64_t G = row * nb + gb;
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + G * kT3GroupBytes + 12 * q);
-            w[i][0] = __ldg(src);
-            w[i][1] = __ldg(src + 1);
-            w[i][2] = __ldg(src + 2);
-            gm[i] = __ldg(norms + G);
-          }
-        }
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const uint32_t off = t3_pair_off(p, w[i][0], w[i][1], w[i][2], lane4);
-            const float t = *reinterpret_cast<const float*>(t3s + p * 8192 + off);
-            if (p & 1) a1 += t;
-            else a0 += t;
-          }
-          v[i] = (a0 + a1) * gm[i];
-        }
-        const float r = t3_reduce8(v, lane);
-        const int i = 8 * g + (lane >> 2);
-        if (q == 0 && i < nrows) acc[i] += r;
+      // two register sets in turn: the next group's codes are in flight while
+      // the current group is summed
+      uint32_t wn[8][3];
+      float gn[8];
+      for (int g = warp; 8 * g < nrows; g += 2 * kT3GWarps) {
+        t3_load_rows(packed, norms, c0, g + kT3GWarps, nrows, nb, gb, gvalid, q, wn, gn);
+        t3_rows_step(wc, gc, lb, lane, q, 8 * g, nrows, acc);
+        if (8 * (g + kT3GWarps) >= nrows) break;
+        t3_load_rows(packed, norms, c0, g + 2 * kT3GWarps, nrows, nb, gb, gvalid, q, wc, gc);
+        t3_rows_step(wn, gn, lb, lane, q, 8 * (g + kT3GWarps), nrows, acc);
       }
     }
     cluster_sync_all();  // every CTA of the cluster has its slice sums of the chunk
