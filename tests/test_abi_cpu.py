@@ -63,6 +63,13 @@ def test_validation_before_launch(hl):
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, None, p, p, None) == hl.HLWQ_EINVAL
     assert L.hlwq_requantize_int4(p, p, p, 4, 704, p, p, p, None) == hl.HLWQ_EUNSUPPORTED  # not 128-aligned
     assert L.hlwq_requantize_int4(p, p, p, 4, 128, ctypes.c_void_p(264), p, p, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_tq3_quantize(p, 4, 128, None, p, p, p, None) == hl.HLWQ_EINVAL      # no signs
+    assert L.hlwq_tq3_quantize(p, 4, 128, p, p, ctypes.c_void_p(258), p, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_tq3_dequantize(p, p, p, p, 4, 128, p, hl.HLWQ_F16, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_tq3_dequantize(p, p, p, p, 0, 128, p, hl.HLWQ_F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_tq3_gemv(p, p, p, p, 4, 128, odd, p, hl.HLWQ_F32, None) == hl.HLWQ_EALIGN
+    assert L.hlwq_tq3_gemv(p, p, p, p, 4, 0, p, p, hl.HLWQ_F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_tq3_gemv(p, p, p, p, 4, 128, p, p, 9, None) == hl.HLWQ_EUNSUPPORTED
     assert L.hlwq_codes_unpack(p, 0, p, None) == hl.HLWQ_EINVAL
     assert L.hlwq_codes_pack(None, 4, p, None) == hl.HLWQ_EINVAL
     assert L.hlwq_codes_pack(p, 4, ctypes.c_void_p(264), None) == hl.HLWQ_EALIGN
