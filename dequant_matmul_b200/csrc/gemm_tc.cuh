@@ -604,11 +604,11 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
   float* part = nsplit ? reinterpret_cast<float*>(ws + P.part_off) : nullptr;
   const int rot_smem = nb * kBlock * 4;
   if (rot_smem > 200 * 1024) return HLWQ_EUNSUPPORTED;
-  static bool rot_attr = false;
-  if (!rot_attr) {
+  static PerDeviceFlag rot_attr;
+  if (!rot_attr()) {
     if (cudaFuncSetAttribute(rotate_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
       return HLWQ_ECUDA;
-    rot_attr = true;
+    rot_attr() = true;
   }
   rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s, part_cnt, nsplit);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
@@ -635,11 +635,11 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
   const int smem = tc_smem_bytes(n_box, nb);
-  static bool attr = false;
-  if (!attr) {
+  static PerDeviceFlag attr;
+  if (!attr()) {
     if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return HLWQ_ECUDA;
-    attr = true;
+    attr() = true;
   }
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const int nfull = P.row_tiles * P.n_tiles - nsplit;

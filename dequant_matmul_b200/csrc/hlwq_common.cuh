@@ -84,15 +84,27 @@ __device__ __forceinline__ uint32_t bits5(uint32_t lo, uint32_t hi) {
   }
 }
 
-inline int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+// A flag per device, for host-side work done once per device (kernel
+// attributes belong to the device that was current when they were set).
+struct PerDeviceFlag {
+  bool done[64] = {};
+  bool& operator()() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return done[d & 63];
   }
-  return n;
+};
+
+inline int sm_count() {
+  static int n[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& v = n[dev & 63];
+  if (v == 0) {
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (v <= 0) v = 148;
+  }
+  return v;
 }
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -397,13 +397,13 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
   const int smem_d = engine_layout(kMoePass, nbf, kHT, (nbf + cd - 1) / cd).total;
   if (smem_g > 227 * 1024 || smem_d > 227 * 1024) return HLWQ_EUNSUPPORTED;
   const int grid = sm_count();
-  static bool attrs = false;
-  if (!attrs) {
+  static PerDeviceFlag attrs;
+  if (!attrs()) {
     bool ok = set_smem_attr(gate_up_kernel<8>) && set_smem_attr(gate_up_kernel<4>) &&
               set_smem_attr(gate_up_kernel<2>) && set_smem_attr(down_kernel<8>) &&
               set_smem_attr(down_kernel<4>) && set_smem_attr(down_kernel<2>);
     if (!ok) return HLWQ_ECUDA;
-    attrs = true;
+    attrs() = true;
   }
   switch (cg) {
     case 8: gate_up_kernel<8><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
