@@ -190,9 +190,11 @@ extern "C" int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const 
                             as_stream(stream), flags);
 }
 
-extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
-                         int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy, int ydtype,
-                         void* workspace, size_t ws_bytes, void* stream) {
+namespace hlwq {
+// Host checks of hlwq_gemm's arguments other than the workspace (shared with
+// hlwq_gemm_noalloc, which runs them before it sizes its scratch).
+int gemm_check_args(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out, int64_t in,
+                    int64_t M, const uint16_t* X, int64_t ldx, const void* Y, int64_t ldy, int ydtype) {
   if (!packed || !norms || !codebook || !X || !Y || out <= 0 || in <= 0 || in > kMaxIn || M <= 0 || M > (1 << 20))
     return HLWQ_EINVAL;
   if (ldx < in || ldy < out) return HLWQ_EINVAL;
@@ -200,6 +202,14 @@ extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const flo
   if (!aligned16(packed) || !aligned2(norms) || !aligned2(X) || !aligned2(Y) ||
       (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(Y) & 3u)))
     return HLWQ_EALIGN;
+  return HLWQ_OK;
+}
+}  // namespace hlwq
+
+extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
+                         int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy, int ydtype,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  if (const int st = hlwq::gemm_check_args(packed, norms, codebook, out, in, M, X, ldx, Y, ldy, ydtype)) return st;
   // the tensor-core path accepts its smallest workspace (no K split of the
   // last wave) up to the size hlwq_workspace_bytes reports
   const size_t need = M >= kTensorCoreMinM ? hlwq::gemm_tc_workspace_min_bytes(out, in, M) : 0;

@@ -578,12 +578,19 @@ inline TcPlan tc_plan(int64_t O, int64_t in, int64_t M) {
   return P;
 }
 
+// Rows longer than kTcMaxNb blocks do not fit the tile-norm staging and run
+// on the CUDA-core path, which needs no workspace.
+inline bool gemm_tc_takes(int64_t in) { return ceil_div(in, kBlock) <= kTcMaxNb; }
+
 size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
+  if (!gemm_tc_takes(in)) return 0;
   const TcPlan P = tc_plan(O, in, M);
   return P.nsplit ? std::max(P.split_bytes, P.base_bytes) : P.base_bytes;
 }
 
-size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) { return tc_plan(O, in, M).base_bytes; }
+size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
+  return gemm_tc_takes(in) ? tc_plan(O, in, M).base_bytes : 0;
+}
 
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
@@ -592,8 +599,7 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
                    const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
                    size_t ws_bytes, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
-  // Rows longer than kTcMaxNb blocks do not fit the tile-norm staging: CUDA-core path.
-  if (nb > kTcMaxNb) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
+  if (!gemm_tc_takes(in)) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
   const TcPlan P = tc_plan(O, in, M);
   if (ws_bytes < P.base_bytes) return HLWQ_EWORKSPACE;
   const int nsplit = ws_bytes >= P.split_bytes ? P.nsplit : 0;
@@ -604,12 +610,12 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
   float* part = nsplit ? reinterpret_cast<float*>(ws + P.part_off) : nullptr;
   const int rot_smem = nb * kBlock * 4;
   if (rot_smem > 200 * 1024) return HLWQ_EUNSUPPORTED;
-  static PerDeviceFlag rot_attr;
-  if (!rot_attr()) {
-    if (cudaFuncSetAttribute(rotate_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
-      return HLWQ_ECUDA;
-    rot_attr() = true;
-  }
+  static PerDeviceOnce rot_attr;
+  if (const int st = rot_attr([&] {
+        return cudaFuncSetAttribute(rotate_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    200 * 1024) == cudaSuccess;
+      }))
+    return st;
   rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s, part_cnt, nsplit);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
 
@@ -635,12 +641,12 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
   const int smem = tc_smem_bytes(n_box, nb);
-  static PerDeviceFlag attr;
-  if (!attr()) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-      return HLWQ_ECUDA;
-    attr() = true;
-  }
+  static PerDeviceOnce attr;
+  if (const int st = attr([&] {
+        return cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024) == cudaSuccess;
+      }))
+    return st;
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const int nfull = P.row_tiles * P.n_tiles - nsplit;
   gemm_tc_kernel<<<nfull + 2 * nsplit, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,

@@ -584,13 +584,12 @@ int launch_gemv1_cs(const CUtensorMap& map, const uint16_t* norms, const float* 
                     int nb, const uint16_t* x, void* Y, bool out_bf16, unsigned flags, int grid, int pass_rows,
                     cudaStream_t stream) {
   const G1Layout L = g1_layout(nb, pass_rows, (nb + C - 1) / C, S);
-  static PerDeviceFlag attr_set;
-  if (!attr_set()) {
-    if (cudaFuncSetAttribute(gemv1_kernel<C, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
-      return HLWQ_ECUDA;
-    attr_set() = true;
-  }
+  static PerDeviceOnce attr_set;
+  if (const int st = attr_set([&] {
+        return cudaFuncSetAttribute(gemv1_kernel<C, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024) == cudaSuccess;
+      }))
+    return st;
   const int xvec = (reinterpret_cast<uintptr_t>(x) % 16 == 0 && in % 8 == 0) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -662,13 +661,12 @@ int launch_dense_t(const uint8_t* packed, const uint16_t* norms, const float* co
   const int nch = (nb + C - 1) / C;
   const EngineLayout L = engine_layout(MT, nb, max_rows, nch);
   if (L.total > 227 * 1024) return HLWQ_EUNSUPPORTED;
-  static PerDeviceFlag attr_set;
-  if (!attr_set()) {
-    if (cudaFuncSetAttribute(dense_kernel<C, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
-      return HLWQ_ECUDA;
-    attr_set() = true;
-  }
+  static PerDeviceOnce attr_set;
+  if (const int st = attr_set([&] {
+        return cudaFuncSetAttribute(dense_kernel<C, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024) == cudaSuccess;
+      }))
+    return st;
   dense_kernel<C, MT><<<grid, kEngineThreads, L.total, stream>>>(packed, norms, codebook, O, in, nb, X, ldx, M, Y,
                                                                   ldy, out_bf16 ? 1 : 0, max_rows);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;

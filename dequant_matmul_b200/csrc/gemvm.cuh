@@ -291,13 +291,12 @@ int launch_gemvm_cs(const CUtensorMap& map, const uint16_t* norms, const float* 
                     const uint16_t* X, int64_t ldx, int ntok, void* Y, int64_t ldy, bool out_bf16, int grid,
                     int pass_rows, cudaStream_t stream) {
   const GmLayout L = gm_layout(nb, pass_rows, (nb + C - 1) / C, S, MT);
-  static PerDeviceFlag attr_set;
-  if (!attr_set()) {
-    if (cudaFuncSetAttribute(gemvm_kernel<C, S, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess)
-      return HLWQ_ECUDA;
-    attr_set() = true;
-  }
+  static PerDeviceOnce attr_set;
+  if (const int st = attr_set([&] {
+        return cudaFuncSetAttribute(gemvm_kernel<C, S, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024) == cudaSuccess;
+      }))
+    return st;
   const int xvec = (reinterpret_cast<uintptr_t>(X) % 16 == 0 && in % 8 == 0 && ldx % 8 == 0) ? 1 : 0;
   gemvm_kernel<C, S, MT><<<grid, kG1Threads, L.total, stream>>>(map, norms, codebook, O, in, nb, X, ldx, ntok, Y, ldy,
                                                                 out_bf16 ? 1 : 0, pass_rows, xvec);

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "hlwq.h"
 
 namespace hlwq {
@@ -84,25 +87,39 @@ __device__ __forceinline__ uint32_t bits5(uint32_t lo, uint32_t hi) {
   }
 }
 
-// A flag per device, for host-side work done once per device (kernel
-// attributes belong to the device that was current when they were set).
-struct PerDeviceFlag {
-  bool done[64] = {};
-  bool& operator()() {
+// Host-side set-up done once per device (kernel attributes belong to the
+// device that was current when they were set).  Thread-safe; a device index
+// at or above kMaxDevices is refused with HLWQ_EUNSUPPORTED.
+constexpr int kMaxDevices = 64;
+
+struct PerDeviceOnce {
+  std::atomic<bool> done[kMaxDevices];
+  std::mutex mu;
+  // Runs f() (returning true on success) on the current device unless it has
+  // succeeded there before; HLWQ_OK, HLWQ_ECUDA or HLWQ_EUNSUPPORTED.
+  template <class F>
+  int operator()(F&& f) {
     int d = 0;
-    cudaGetDevice(&d);
-    return done[d & 63];
+    if (cudaGetDevice(&d) != cudaSuccess) return HLWQ_ECUDA;
+    if (d < 0 || d >= kMaxDevices) return HLWQ_EUNSUPPORTED;
+    if (done[d].load(std::memory_order_acquire)) return HLWQ_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[d].load(std::memory_order_relaxed)) return HLWQ_OK;
+    if (!f()) return HLWQ_ECUDA;
+    done[d].store(true, std::memory_order_release);
+    return HLWQ_OK;
   }
 };
 
+// Number of SMs of the current device (cached per device; 148 if the query fails).
 inline int sm_count() {
-  static int n[64] = {};
+  static std::atomic<int> n[kMaxDevices];
   int dev = 0;
-  cudaGetDevice(&dev);
-  int& v = n[dev & 63];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = n[dev].load(std::memory_order_relaxed);
   if (v == 0) {
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    if (v <= 0) v = 148;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    n[dev].store(v, std::memory_order_relaxed);
   }
   return v;
 }

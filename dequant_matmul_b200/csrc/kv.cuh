@@ -300,13 +300,12 @@ int launch_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const flo
 int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
                      const float* codebook, int64_t n, float* S, int64_t lds, cudaStream_t stream) {
   const int smem = static_cast<int>(m) * kKvQRow * 4;
-  static PerDeviceFlag attr;
-  if (!attr()) {
-    if (cudaFuncSetAttribute(kv_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kKvMaxQueries * kKvQRow * 4) != cudaSuccess)
-      return HLWQ_ECUDA;
-    attr() = true;
-  }
+  static PerDeviceOnce attr;
+  if (const int st = attr([&] {
+        return cudaFuncSetAttribute(kv_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kKvMaxQueries * kKvQRow * 4) == cudaSuccess;
+      }))
+    return st;
   const int64_t max_ctas = static_cast<int64_t>(sm_count()) * 4;
   const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(n, kKvThreads / 8)));
   kv_scores_kernel<<<grid, kKvThreads, smem, stream>>>(Q, static_cast<int>(m), ldq, packed, norms, codebook, n, S,

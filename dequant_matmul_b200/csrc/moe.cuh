@@ -397,14 +397,16 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
   const int smem_d = engine_layout(kMoePass, nbf, kHT, (nbf + cd - 1) / cd).total;
   if (smem_g > 227 * 1024 || smem_d > 227 * 1024) return HLWQ_EUNSUPPORTED;
   const int grid = sm_count();
-  static PerDeviceFlag attrs;
-  if (!attrs()) {
-    bool ok = set_smem_attr(gate_up_kernel<8>) && set_smem_attr(gate_up_kernel<4>) &&
-              set_smem_attr(gate_up_kernel<2>) && set_smem_attr(down_kernel<8>) &&
-              set_smem_attr(down_kernel<4>) && set_smem_attr(down_kernel<2>);
-    if (!ok) return HLWQ_ECUDA;
-    attrs() = true;
-  }
+  static PerDeviceOnce attrs;
+  if (const int st = attrs([&] {
+        return set_smem_attr(gate_up_kernel<8>) &&
+               set_smem_attr(gate_up_kernel<4>) &&
+               set_smem_attr(gate_up_kernel<2>) &&
+               set_smem_attr(down_kernel<8>) &&
+               set_smem_attr(down_kernel<4>) &&
+               set_smem_attr(down_kernel<2>);
+      }))
+    return st;
   switch (cg) {
     case 8: gate_up_kernel<8><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
     case 4: gate_up_kernel<4><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;

@@ -447,11 +447,11 @@ bool moe1_attr(K kernel) {
 template <int C, int S>
 int moe1_launch_gu(const CUtensorMap& gm, const CUtensorMap& sm, const Moe1Params& P, int grid, int part_rows,
                    int tok_max, int smem, cudaStream_t stream) {
-  static PerDeviceFlag attr;
-  if (!attr()) {
-    if (!moe1_attr(moe_gu1_kernel<C, S>)) return HLWQ_ECUDA;
-    attr() = true;
-  }
+  static PerDeviceOnce attr;
+  if (const int st = attr([&] {
+        return moe1_attr(moe_gu1_kernel<C, S>);
+      }))
+    return st;
   moe_gu1_kernel<C, S><<<grid, kG1Threads, smem, stream>>>(gm, sm, P, part_rows, tok_max);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
@@ -459,11 +459,11 @@ int moe1_launch_gu(const CUtensorMap& gm, const CUtensorMap& sm, const Moe1Param
 template <int C, int S>
 int moe1_launch_dn(const CUtensorMap& dm, const CUtensorMap& sm, const Moe1Params& P, int grid, int rows_max,
                    int pg_max, int smem, cudaStream_t stream) {
-  static PerDeviceFlag attr;
-  if (!attr()) {
-    if (!moe1_attr(moe_dn1_kernel<C, S>)) return HLWQ_ECUDA;
-    attr() = true;
-  }
+  static PerDeviceOnce attr;
+  if (const int st = attr([&] {
+        return moe1_attr(moe_dn1_kernel<C, S>);
+      }))
+    return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kG1Threads);

@@ -3,7 +3,8 @@
 // stream region that must not allocate, plug-ins embedded in a host that owns
 // every allocation, and allocator-less runtimes that only hand out input and
 // output buffers.  hlwq_gemm needs a scratch workspace for the rotated
-// activations when M >= 16; this entry point takes that scratch from a
+// activations when it runs on the tensor cores (M >= 5 and rows of at most
+// 8192 inputs); this entry point takes that scratch from a
 // fixed-size array in device memory that belongs to the library instead.
 //
 // The array is a file-scope static __device__ object: every GPU that loads the
@@ -25,6 +26,8 @@
 
 namespace hlwq {
 size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M);
+int gemm_check_args(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out, int64_t in,
+                    int64_t M, const uint16_t* X, int64_t ldx, const void* Y, int64_t ldy, int ydtype);
 }  // namespace hlwq
 
 namespace {
@@ -60,9 +63,11 @@ int scratch_for_current_device(void** out) {
 extern "C" int hlwq_gemm_noalloc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,
                                  int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy,
                                  int ydtype, void* stream) {
-  if (!packed || !norms || !codebook || !X || !Y || out <= 0 || in <= 0 || M <= 0) return HLWQ_EINVAL;
-  // the tensor-core path runs with its smallest workspace here; it uses the
-  // K split of its last tiles only when the scratch also holds the partials
+  // the same argument checks as hlwq_gemm, before any size is derived from them
+  if (const int st = hlwq::gemm_check_args(packed, norms, codebook, out, in, M, X, ldx, Y, ldy, ydtype)) return st;
+  // the tensor-core path runs with its smallest workspace here (it uses the K
+  // split of its last tiles only when the scratch also holds the partials);
+  // shapes that hlwq_gemm serves without a workspace need none
   const size_t need = hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
                           ? hlwq::gemm_tc_workspace_min_bytes(out, in, M) : 0;
   if (need > kNoallocScratchBytes) return HLWQ_ESCRATCH;

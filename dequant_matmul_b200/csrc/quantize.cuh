@@ -518,13 +518,14 @@ int launch_quantize(const void* W, bool bf16, int64_t rows, int in, const float*
   const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(warps_needed, kQThreads / 32)));
   const bool vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) &&
                    ((static_cast<int64_t>(in) * (bf16 ? 2 : 4)) % 16 == 0);
-  static PerDeviceFlag attrs;
-  if (!attrs()) {
-    if (!(quant_attr(quantize_kernel<true, true>) && quant_attr(quantize_kernel<true, false>) &&
-          quant_attr(quantize_kernel<false, true>) && quant_attr(quantize_kernel<false, false>)))
-      return HLWQ_ECUDA;
-    attrs() = true;
-  }
+  static PerDeviceOnce attrs;
+  if (const int st = attrs([&] {
+        return quant_attr(quantize_kernel<true, true>) &&
+               quant_attr(quantize_kernel<true, false>) &&
+               quant_attr(quantize_kernel<false, true>) &&
+               quant_attr(quantize_kernel<false, false>);
+      }))
+    return st;
   if (bf16) {
     if (vec) quantize_kernel<true, true><<<grid, kQThreads, kQSmemBytes, stream>>>(W, rows, in, nb, codebook, packed, norms);
     else quantize_kernel<true, false><<<grid, kQThreads, kQSmemBytes, stream>>>(W, rows, in, nb, codebook, packed, norms);

@@ -540,13 +540,12 @@ int launch_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* sig
   const int nb = static_cast<int>(ceil_div(in, kBlock));
   const int nslices = static_cast<int>(ceil_div(nb, kT3SliceGroups));
   const int C = std::min(nslices, kT3MaxCluster);
-  static PerDeviceFlag attr;
-  if (!attr()) {
-    if (cudaFuncSetAttribute(tq3_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kT3SmemBytes) !=
-        cudaSuccess)
-      return HLWQ_ECUDA;
-    attr() = true;
-  }
+  static PerDeviceOnce attr;
+  if (const int st = attr([&] {
+        return cudaFuncSetAttribute(tq3_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kT3SmemBytes) == cudaSuccess;
+      }))
+    return st;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;

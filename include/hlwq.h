@@ -237,7 +237,9 @@ int hlwq_gemv_ex(const uint8_t* packed, const uint16_t* norms, const float* code
  *   Y  device ydtype [M][ldy] (ldy >= out)
  *   workspace  device, ws_bytes >= hlwq_workspace_bytes(HLWQ_OP_GEMM, out, in, M, 1, 0)
  * M = 1..4 runs on the CUDA-core decode path (one launch streams the weights for
- * up to four tokens); M >= 5 on the tensor-core path (workspace needed).
+ * up to four tokens); M >= 5 on the tensor-core path (workspace needed) when
+ * in <= 8192.  Longer rows run on the CUDA-core path at every M and need no
+ * workspace (hlwq_workspace_bytes reports 0 for them).
  * On the tensor-core path the reported size includes fp32 partials for
  * splitting the K range of the tiles of a partial last wave over two CTAs
  * each (added in a fixed order, so results do not depend on timing).  Any
@@ -291,7 +293,9 @@ size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, 
  *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
  *   - Requests whose smallest tensor-core workspace (about
  *     M * ceil(in / 128) * 256 bytes, see hlwq_gemm) exceeds
- *     HLWQ_NOALLOC_SCRATCH_BYTES return HLWQ_ESCRATCH.
+ *     HLWQ_NOALLOC_SCRATCH_BYTES return HLWQ_ESCRATCH; shapes that hlwq_gemm
+ *     serves without a workspace (M <= 4, in > 8192) use no scratch.
+ *   - Invalid arguments return hlwq_gemm's errors before any size is derived.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
  *     stream capture.

@@ -98,3 +98,30 @@ def test_workspace_sizes(hl):
     a = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 1, 256, 8)
     b = hl.workspace_bytes(hl.HLWQ_OP_MOE, 2048, 512, 64, 256, 8)
     assert 0 < a < b
+
+
+def test_gemm_workspace_only_on_the_tensor_core_path(hl):
+    # rows of at most 8192 inputs take the tensor cores from M = 5 (workspace);
+    # longer rows run on the CUDA-core path at every M and need none
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 8192, 64) > 0
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 8193, 64) == 0
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 65536, 512) == 0
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 8192, 4) == 0
+
+
+def test_noalloc_validates_arguments_before_sizing_its_scratch(hl):
+    L = hl.lib
+    p = ctypes.c_void_p(256)
+    F32 = hl.HLWQ_F32
+    # out-of-range sizes are argument errors, not scratch errors
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 1 << 21, 64, p, 1 << 21, p, 128, F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 512, (1 << 20) + 1, p, 512, p, 128, F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 512, 64, p, 256, p, 128, F32, None) == hl.HLWQ_EINVAL  # ldx < in
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 512, 64, p, 512, p, 64, F32, None) == hl.HLWQ_EINVAL   # ldy < out
+    assert L.hlwq_gemm_noalloc(None, p, p, 128, 512, 64, p, 512, p, 128, F32, None) == hl.HLWQ_EINVAL
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 512, 64, p, 512, p, 128, 7, None) == hl.HLWQ_EUNSUPPORTED
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 512, 64, ctypes.c_void_p(257), 512, p, 128, F32,
+                               None) == hl.HLWQ_EALIGN
+    # a tensor-core request above the static scratch (512 x 64 blocks x 256 B)
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 128, 8192, 512) > hl.NOALLOC_SCRATCH_BYTES
+    assert L.hlwq_gemm_noalloc(p, p, p, 128, 8192, 512, p, 8192, p, 128, F32, None) == hl.HLWQ_ESCRATCH

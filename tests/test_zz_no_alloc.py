@@ -36,9 +36,25 @@ def test_noalloc_matches_gemm_on_consecutive_calls(hl):
 
 
 def test_noalloc_rejects_requests_beyond_the_scratch(hl):
-    need = hl.workspace_bytes(hl.HLWQ_OP_GEMM, 128, 65536, 64)
+    # stays on the tensor-core path (64 blocks per row) but needs 8 MiB of scratch
+    need = hl.workspace_bytes(hl.HLWQ_OP_GEMM, 128, 8192, 512)
     assert need > hl.NOALLOC_SCRATCH_BYTES
     p = ctypes.c_void_p(256)
-    st = hl.lib.hlwq_gemm_noalloc(p, p, p, 128, 65536, 64, p, 65536, p, 128, hl.HLWQ_F32, None)
+    st = hl.lib.hlwq_gemm_noalloc(p, p, p, 128, 8192, 512, p, 8192, p, 128, hl.HLWQ_F32, None)
     assert st == hl.HLWQ_ESCRATCH
     assert hl.lib.hlwq_status_string(st).decode().startswith("request exceeds")
+
+
+def test_noalloc_serves_long_rows_without_scratch(hl):
+    # rows longer than the tensor-core tile's 8192 inputs run on the CUDA-core
+    # path, which needs no scratch, so any M is served
+    cb = hl.codebook("cuda")
+    W = synth.student_t((256, 8320), df4_seed=78).cuda()
+    p, n = hl.quantize(W, cb)
+    assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 8320, 64) == 0
+    X = synth.activations(64, 8320, seed=4).cuda()
+    got = hl.gemm_noalloc(p, n, cb, X, out_dtype=torch.float32)
+    want = hl.gemm(p, n, cb, X, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert rel_l2(got.double().cpu().numpy(), want.double().cpu().numpy()) <= MATMUL_REL
+    assert hl.device_error() == 0
