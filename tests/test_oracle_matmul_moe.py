@@ -99,3 +99,108 @@ def test_moe_shared_expert_adds_with_weight_one():
     b, _, _ = O.moe_forward(gu, dn, H, F, 2, lg, x, sg, sd)
     shared_only, _, _ = O.moe_forward([sg], [sd], H, F, 1, np.zeros((1, 1)), x)
     assert np.allclose(b - a, shared_only, rtol=1e-12, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# The routing-weighted combine for k >= 2 ("Qwen3.6-35B-A3B -- HLWQ Q5",
+# Architecture table: 8 routed + 1 shared expert per token).  The weights are
+# fixed in closed form by the logits, and each expert's MLP is rebuilt here
+# from the dequantized matrices with SiLU written out, so a combine that drops
+# a weight, takes it from the wrong slot or normalises over all E fails.
+# --------------------------------------------------------------------------
+
+H_C, F_C, E_C = 128, 128, 5
+
+
+@pytest.fixture(scope="module")
+def experts():
+    mk = lambda shape, s: (lambda q: (q["packed"], q["norms"]))(O.quantize(synth.student_t(shape, df4_seed=s)))
+    gu = [mk((2 * F_C, H_C), 60 + e) for e in range(E_C)]
+    dn = [mk((H_C, F_C), 70 + e) for e in range(E_C)]
+    x = synth.activations(1, H_C, seed=9)
+    return gu, dn, x
+
+
+def _mlp(gu, dn, xt):
+    wg = O.dequantize(gu[0], gu[1], H_C)
+    wd = O.dequantize(dn[0], dn[1], F_C)
+    g, u = wg[:F_C] @ xt, wg[F_C:] @ xt
+    return wd @ ((g / (1.0 + np.exp(-g))) * u)
+
+
+def _logits(sel, offsets):
+    """Experts `sel` get logits 1.5 - offsets (the others -4): softmax over the
+    selected ones is proportional to exp(-offsets)."""
+    lg = np.full((1, E_C), -4.0)
+    for e, d in zip(sel, offsets):
+        lg[0, e] = 1.5 - d
+    return lg
+
+
+def _combine_matches_closed_form(forward, experts) -> bool:
+    gu, dn, x = experts
+    xt = x[0].double().numpy()
+    cases = [  # (selected experts in selection order, logit offsets, closed-form weights)
+        ((3, 1), (0.0, np.log(3.0)), (3 / 4, 1 / 4)),
+        ((0, 4, 2), (0.0, np.log(2.0), np.log(4.0)), (4 / 7, 2 / 7, 1 / 7)),
+    ]
+    for sel, offs, p in cases:
+        out = forward(gu, dn, H_C, F_C, len(sel), _logits(sel, offs), x)[0][0]
+        want = sum(pi * _mlp(gu[e], dn[e], xt) for e, pi in zip(sel, p))
+        if not np.allclose(out, want, rtol=1e-12, atol=1e-14):
+            return False
+    return True
+
+
+def test_moe_combine_weights_in_closed_form(experts):
+    """k = 2 with logits (a, a - ln 3) gives p = (3/4, 1/4); k = 3 with
+    (a, a - ln 2, a - ln 4) gives (4/7, 2/7, 1/7)."""
+    assert _combine_matches_closed_form(O.moe_forward, experts)
+
+
+def test_moe_combine_is_linear_in_the_weights(experts):
+    """Moving one selected logit changes the output by exactly
+    delta_p * (MLP_first - MLP_second) for k = 2."""
+    gu, dn, x = experts
+    xt = x[0].double().numpy()
+    m1, m2 = _mlp(gu[1], dn[1], xt), _mlp(gu[3], dn[3], xt)
+    a, _, wa = O.moe_forward(gu, dn, H_C, F_C, 2, _logits((1, 3), (0.0, 1.0)), x)
+    b, _, wb = O.moe_forward(gu, dn, H_C, F_C, 2, _logits((1, 3), (0.0, 0.25)), x)
+    pa, pb = 1 / (1 + np.exp(-1.0)), 1 / (1 + np.exp(-0.25))
+    assert wa[0, 0] == pytest.approx(pa, rel=1e-15) and wb[0, 0] == pytest.approx(pb, rel=1e-15)
+    assert np.allclose(b[0] - a[0], (pb - pa) * (m1 - m2), rtol=1e-11, atol=1e-14)
+
+
+def test_moe_combine_planted_mistakes_fail_the_pin(experts, monkeypatch):
+    """A router whose weights are dropped (all 1), normalised over all E, or
+    handed to the wrong slots; and a combine that takes every slot's weight
+    from slot 0: each fails the closed-form pin."""
+    from oracle import hlwq_oracle as HO
+    good = HO.router_topk
+
+    def ones(lg, k):
+        ids, w = good(lg, k)
+        return ids, np.ones_like(w)
+
+    def over_all(lg, k):
+        ids, _ = good(lg, k)
+        z = np.exp(lg - lg.max(axis=1, keepdims=True))
+        z /= z.sum(axis=1, keepdims=True)
+        return ids, np.take_along_axis(z, ids, axis=1)
+
+    def reversed_slots(lg, k):
+        ids, w = good(lg, k)
+        return ids, w[:, ::-1].copy()
+
+    for bad in (ones, over_all, reversed_slots):
+        monkeypatch.setattr(HO, "router_topk", bad)
+        assert not _combine_matches_closed_form(O.moe_forward, experts), bad.__name__
+    monkeypatch.setattr(HO, "router_topk", good)
+    assert _combine_matches_closed_form(O.moe_forward, experts)
+
+    def slot0_weight(gu, dn, hidden, inter, k, logits, X):
+        ids, w = O.router_topk(logits, k)
+        xt = X[0].double().numpy()
+        out = sum(w[0, 0] * _mlp(gu[int(e)], dn[int(e)], xt) for e in ids[0])
+        return out[None], ids, w
+    assert not _combine_matches_closed_form(slot0_weight, experts)
