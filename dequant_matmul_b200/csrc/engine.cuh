@@ -22,9 +22,9 @@
 // (c[k0], c[k1]); the table is replicated once per lane so that lane l always
 // reads bank l (conflict-free whatever the codes), i.e. one shared-memory
 // wavefront decodes 64 weights.  The rotated activation is stored as binary16,
-// scaled by a power of two per 128-block; products are formed with packed
-// half2 FMAs in short chains (at most 4 products per chain, combined pairwise)
-// and every 16 products are added to an fp32 accumulator.
+// scaled by a power of two per 128-block; every product of a binary16
+// centroid and a binary16 activation (exact in fp32) is added to an fp32
+// accumulator with the mixed-precision FMA.
 #pragma once
 
 #include "hlwq_common.cuh"
@@ -259,21 +259,25 @@ __device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+// fp32 accumulation of binary16 products (sm_100 mixed-precision FMA): the
+// product of two binary16 values is exact in fp32, so each term is added to
+// the fp32 accumulator with a single fp32 rounding.  fma_lo uses the low
+// halves of a and b, fma_hi the high halves.
+__device__ __forceinline__ float fma_lo(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{ .reg .b16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %3; }"
+      : "=f"(d) : "r"(a), "r"(b), "f"(c));
   return d;
 }
 
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+__device__ __forceinline__ float fma_hi(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{ .reg .b16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1; mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a1, b1, %3; }"
+      : "=f"(d) : "r"(a), "r"(b), "f"(c));
   return d;
 }
 
@@ -308,22 +312,18 @@ __device__ __forceinline__ void round_entries(const uint4 (&cw)[5], uint32_t lan
   ent[7] = lds_u32(pair_addr<80 * R8 + 70>(cw, lane_base));
 }
 
-// sum over 8 pairs of c-pair . x-pair: four half2 product chains of two pairs,
-// combined pairwise in half2, the last two halves added in fp32 (the rotated
-// activation is scaled so that |x| < 2^10, far from binary16 overflow).
+// sum over 8 pairs of c-pair . x-pair, every binary16 product added to an
+// fp32 accumulator (four accumulators: pair parity x half).
 __device__ __forceinline__ float round_dot(const uint32_t (&ent)[8], uint32_t x0, uint32_t x1, uint32_t x2,
                                            uint32_t x3, uint32_t x4, uint32_t x5, uint32_t x6, uint32_t x7) {
-  uint32_t h0 = hmul2(ent[0], x0);
-  uint32_t h1 = hmul2(ent[1], x1);
-  uint32_t h2 = hmul2(ent[2], x2);
-  uint32_t h3 = hmul2(ent[3], x3);
-  h0 = hfma2(ent[4], x4, h0);
-  h1 = hfma2(ent[5], x5, h1);
-  h2 = hfma2(ent[6], x6, h2);
-  h3 = hfma2(ent[7], x7, h3);
-  const uint32_t hs = hadd2(hadd2(h0, h1), hadd2(h2, h3));
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hs));
-  return f.x + f.y;
+  const uint32_t x[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
+  float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    a[2 * (p & 1)] = fma_lo(ent[p], x[p], a[2 * (p & 1)]);
+    a[2 * (p & 1) + 1] = fma_hi(ent[p], x[p], a[2 * (p & 1) + 1]);
+  }
+  return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 // Dot products of one (row, block) of codes with MT rotated activation blocks
@@ -385,17 +385,11 @@ __device__ __forceinline__ uint32_t half_pair_addr(const uint2 (&cw)[5], uint32_
   return (t & (0x3ffu << 7)) + lane_base;
 }
 
-__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 8 pairs: two half2 chains of 4 products each (even / odd pairs), one half2
-// add, widened to fp32 and added to a packed fp32 pair accumulator.
+// 8 pairs, every binary16 product added to the fp32 accumulators a[4]
+// (pair parity x half).
 template <int P0>
 __device__ __forceinline__ void half_round(const uint2 (&cw)[5], uint32_t lane_base, const uint32_t (&xr)[32],
-                                           uint64_t& acc2) {
+                                           float (&a)[4]) {
   uint32_t e[8];
   e[0] = lds_u32(half_pair_addr<P0 + 0>(cw, lane_base));
   e[1] = lds_u32(half_pair_addr<P0 + 1>(cw, lane_base));
@@ -405,28 +399,22 @@ __device__ __forceinline__ void half_round(const uint2 (&cw)[5], uint32_t lane_b
   e[5] = lds_u32(half_pair_addr<P0 + 5>(cw, lane_base));
   e[6] = lds_u32(half_pair_addr<P0 + 6>(cw, lane_base));
   e[7] = lds_u32(half_pair_addr<P0 + 7>(cw, lane_base));
-  uint32_t h0 = hmul2(e[0], xr[P0 + 0]);
-  uint32_t h1 = hmul2(e[1], xr[P0 + 1]);
-  h0 = hfma2(e[2], xr[P0 + 2], h0);
-  h1 = hfma2(e[3], xr[P0 + 3], h1);
-  h0 = hfma2(e[4], xr[P0 + 4], h0);
-  h1 = hfma2(e[5], xr[P0 + 5], h1);
-  h0 = hfma2(e[6], xr[P0 + 6], h0);
-  h1 = hfma2(e[7], xr[P0 + 7], h1);
-  const uint32_t hs = hadd2(h0, h1);
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hs));
-  acc2 = f32x2_add(acc2, (static_cast<uint64_t>(__float_as_uint(f.y)) << 32) | __float_as_uint(f.x));
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    a[2 * (p & 1)] = fma_lo(e[p], xr[P0 + p], a[2 * (p & 1)]);
+    a[2 * (p & 1) + 1] = fma_hi(e[p], xr[P0 + p], a[2 * (p & 1) + 1]);
+  }
 }
 
 // Single-token dot product of a half block (64 codes) with 64 rotated
 // activation values held in registers (xr[p] = (x[2p], x[2p+1])).
 __device__ __forceinline__ float half_dot_reg(const uint2 (&cw)[5], uint32_t lane_base, const uint32_t (&xr)[32]) {
-  uint64_t acc2 = 0;
-  half_round<0>(cw, lane_base, xr, acc2);
-  half_round<8>(cw, lane_base, xr, acc2);
-  half_round<16>(cw, lane_base, xr, acc2);
-  half_round<24>(cw, lane_base, xr, acc2);
-  return __uint_as_float(static_cast<uint32_t>(acc2)) + __uint_as_float(static_cast<uint32_t>(acc2 >> 32));
+  float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  half_round<0>(cw, lane_base, xr, a);
+  half_round<8>(cw, lane_base, xr, a);
+  half_round<16>(cw, lane_base, xr, a);
+  half_round<24>(cw, lane_base, xr, a);
+  return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 // Processes all items of a CTA's virtual-row range.  rowfn(vrow) returns the

@@ -4,8 +4,8 @@
 // y[m][o] = sum_i X[m][i] * w_hat[o][i] with w_hat the HLWQ Q5 weights
 // ("Qwen3.6-35B-A3B -- HLWQ Q5", Method), evaluated in the rotated domain by
 // the decode engine (engine.cuh): the CTA rotates its tokens' activations once
-// (FWHT per 128-block, binary16 in shared memory), then every weight costs one
-// table lookup and one fp32-accumulating FMA per token.
+// (FWHT per 128-block, binary16 in shared memory), then every pair of weights
+// costs one table lookup and two fp32-accumulating FMAs per token.
 //
 // One persistent CTA of 512 threads per SM (the 128 KiB lane-replicated pair
 // table fills most of the SM's shared memory); the O rows are split into equal
@@ -90,18 +90,16 @@ dense_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ no
 //
 // Per pair of codes: one shift that puts the 10-bit pair index at bit 7, one
 // and-or that forms the byte offset of (entry, lane) in the table, one shared
-// load and one half2 FMA.  The four fp16 chains of a lane (8 products each)
-// are added pairwise in fp16 and widened once per item, scaled
-// by n16 / 128 and the block's activation scale and summed over the row's 2C
-// lanes (the two rows of a lane are reduced together: log2(2C) shuffles); the
-// row sums over chunks are formed at the end in a fixed order
-// (deterministic).
+// load and two mixed-precision FMAs that add the binary16 products to fp32
+// accumulators.  A lane's row sums are scaled by n16 / 128 and the block's
+// activation scale and summed over the row's 2C lanes (the two rows of a lane
+// are reduced together: log2(2C) shuffles); the row sums over chunks are
+// formed at the end in a fixed order (deterministic).
 //
 // Launched with programmatic stream serialisation (HLWQ_FLAG_WEIGHTS_STATIC),
-// the first code boxes and their norms (issued first) and the codebook load do
-// not wait for the previous kernel on the stream (griddepcontrol.wait); x is
-// read and y written only after that wait, and the pair table is built while
-// the x loads are in flight.
+// the first code boxes and their norms (issued first) and the codebook load
+// do not wait for the previous kernel on the stream (griddepcontrol.wait); x
+// is read and y written only after that wait.
 constexpr int kG1Threads = 512;
 constexpr int kG1Warps = kG1Threads / 32;
 constexpr int kG1ItemBytes = 32 * kBlockBytes;  // 2G rows x C blocks = 32 blocks for every C
@@ -146,48 +144,24 @@ __device__ __forceinline__ uint32_t g1_off(const uint2 (&cw)[5], uint32_t lane4)
   return (t & 0x1ff80u) | lane4;
 }
 
-// Pair P goes to fp16 chain P % NC.  NC = 4: four chains of 8 products, added
-// pairwise in fp16 (a block's codes have sum c^2 ~ 128, so a 16-product sum
-// stays below sqrt(135) * 4 * 2^10 < 65504 for |x_tilde| < 2^10) and widened
-// once.  NC = 8: eight chains of 4 products, each widened to fp32 (smaller
-// rounding error, for chained products such as the MoE layer).
-template <int NC, int P>
+// Pair P: one table lookup gives the binary16 centroids (c[k_2P], c[k_2P+1]),
+// each multiplied by its binary16 rotated activation and added to an fp32
+// accumulator (exact products, one fp32 rounding per term).  Four
+// accumulators (pair parity x half) keep the dependent chains short.
+template <int P>
 __device__ __forceinline__ void g1_pair(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
-                                        const uint32_t (&xr)[32], uint32_t (&h)[NC]) {
+                                        const uint32_t (&xr)[32], float (&acc)[4]) {
   const uint32_t e = *reinterpret_cast<const uint32_t*>(tab + g1_off<P>(cw, lane4));
-  if constexpr (P < NC) h[P] = hmul2(e, xr[P]);
-  else h[P % NC] = hfma2(e, xr[P], h[P % NC]);
-}
-
-__device__ __forceinline__ float2 half2_to_float2(uint32_t v) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&v));
-}
-
-template <int NC, int... P>
-__device__ __forceinline__ float g1_dot_n(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
-                                          const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
-  uint32_t h[NC];
-  (g1_pair<NC, P>(tab, cw, lane4, xr, h), ...);
-  if constexpr (NC == 4) {
-    const float2 f0 = half2_to_float2(hadd2(h[0], h[1]));
-    const float2 f1 = half2_to_float2(hadd2(h[2], h[3]));
-    return (f0.x + f1.x) + (f0.y + f1.y);
-  } else {
-    float2 f[NC];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) f[c] = half2_to_float2(h[c]);
-#pragma unroll
-    for (int w = NC / 2; w > 0; w >>= 1)
-#pragma unroll
-      for (int c = 0; c < w; ++c) f[c] = make_float2(f[c].x + f[c + w].x, f[c].y + f[c + w].y);
-    return f[0].x + f[0].y;
-  }
+  acc[2 * (P & 1)] = fma_lo(e, xr[P], acc[2 * (P & 1)]);
+  acc[2 * (P & 1) + 1] = fma_hi(e, xr[P], acc[2 * (P & 1) + 1]);
 }
 
 template <int... P>
 __device__ __forceinline__ float g1_dot(const uint8_t* tab, const uint2 (&cw)[5], uint32_t lane4,
-                                        const uint32_t (&xr)[32], std::integer_sequence<int, P...> seq) {
-  return g1_dot_n<4>(tab, cw, lane4, xr, seq);
+                                        const uint32_t (&xr)[32], std::integer_sequence<int, P...>) {
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  (g1_pair<P>(tab, cw, lane4, xr, acc), ...);
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // Lane l's centroid c = c[l] as binary16 (a warp with `check` set, warp 0 in
@@ -204,6 +178,21 @@ __device__ __forceinline__ uint32_t g1_codebook_half(float c, bool check) {
 
 __device__ __forceinline__ uint32_t g1_codebook_lane(const float* __restrict__ codebook) {
   return g1_codebook_half(__ldg(codebook + (threadIdx.x & 31)), threadIdx.x < 32);
+}
+
+// The binary16 centroids the pair table is expected to hold, passed by value
+// as a kernel parameter (two per word, c[2i] in the low half), so that the
+// table can be built at once instead of after the codebook's memory latency.
+// The host fills it with the Lloyd-Max N(0,1) codebook; every CTA still loads
+// the caller's codebook and rebuilds the table from it when any centroid
+// differs, so the result never depends on this guess.
+struct G1Centroids {
+  uint32_t c16[kLevels / 2];
+};
+
+__device__ __forceinline__ uint32_t g1_expected_half(const G1Centroids& e) {
+  const int lane = threadIdx.x & 31;
+  return (e.c16[lane >> 1] >> (16 * (lane & 1))) & 0xffffu;
 }
 
 // Warps [w0, w0 + nw) write the lane-replicated pair table, word (v * 32 +
@@ -342,8 +331,8 @@ __device__ __forceinline__ void g1_rot_f32(const float* __restrict__ x, int64_t 
 template <int C, int S>
 __global__ void __launch_bounds__(kG1Threads, 1)
 gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restrict__ norms,
-             const float* __restrict__ codebook, int64_t O, int in, int nb, const uint16_t* __restrict__ x,
-             void* __restrict__ Y, int out_bf16, int pass_rows, int xvec) {
+             const float* __restrict__ codebook, const __grid_constant__ G1Centroids expect, int64_t O, int in,
+             int nb, const uint16_t* __restrict__ x, void* __restrict__ Y, int out_bf16, int pass_rows, int xvec) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int L2C = 2 * C;   // lanes per row
   constexpr int G = 32 / L2C;  // rows of one half item
@@ -420,23 +409,29 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
 
     if (p0 == 0) {
       // set-up while the first boxes are in flight.  x may be produced by the
-      // previous kernel on the stream, so the dependency wait comes first and
-      // every thread passes it before it touches x or y; the x loads are then
-      // in flight while the pair table is built (the codebook load was issued
-      // before the wait), and the rotation consumes them.  The barrier below
-      // publishes table and x.
+      // previous kernel on the stream: every thread passes the dependency
+      // wait before it touches x or y.  The x loads are then in flight while
+      // the pair table is built from the expected centroids (a kernel
+      // parameter, no memory latency); the caller's codebook, loaded first,
+      // is compared with them at the barrier that publishes table and x, and
+      // a codebook that differs rebuilds the table before any lookup.
       const float cl = __ldg(codebook + lane);
+      const uint32_t c16x = g1_expected_half(expect);
       pdl_wait();
       uint32_t xw[8];
       const int rb0 = 4 * warp;
       if (rb0 < nb) g1_rot_load(x, in, in, nb, nb, xvec != 0, rb0, xw);
-      g1_build_table(smem, g1_codebook_half(cl, warp == 0), 0, kG1Warps);
+      g1_build_table(smem, c16x, 0, kG1Warps);
       if (rb0 < nb) g1_rot_store(xw, nb, nb, rb0, xs, xinv);
       for (int b0 = rb0 + 4 * kG1Warps; b0 < nb; b0 += 4 * kG1Warps) {
         g1_rot_load(x, in, in, nb, nb, xvec != 0, b0, xw);
         g1_rot_store(xw, nb, nb, b0, xs, xinv);
       }
-      __syncthreads();
+      const uint32_t c16 = g1_codebook_half(cl, warp == 0);
+      if (__syncthreads_or(c16 != c16x)) {
+        g1_build_table(smem, c16, 0, kG1Warps);
+        __syncthreads();
+      }
       pdl_trigger();
     }
 
@@ -579,6 +574,20 @@ inline int g1_pass_rows(int nb, int C, int S, int rows_cta) {
   return cap < RG ? 0 : std::min(rows_cta, cap);
 }
 
+// Binary16 bits of the Lloyd-Max N(0,1) codebook (hlwq_lloyd_codebook),
+// computed once per process.
+inline const G1Centroids& g1_lloyd_max_centroids() {
+  static const G1Centroids e = [] {
+    G1Centroids r{};
+    float c[kLevels];
+    if (hlwq_lloyd_codebook(kLevels, c, nullptr, nullptr) == HLWQ_OK)
+      for (int i = 0; i < kLevels; ++i)
+        r.c16[i >> 1] |= static_cast<uint32_t>(__half_as_ushort(__float2half_rn(c[i]))) << (16 * (i & 1));
+    return r;
+  }();
+  return e;
+}
+
 template <int C, int S>
 int launch_gemv1_cs(const CUtensorMap& map, const uint16_t* norms, const float* codebook, int64_t O, int in,
                     int nb, const uint16_t* x, void* Y, bool out_bf16, unsigned flags, int grid, int pass_rows,
@@ -602,8 +611,8 @@ int launch_gemv1_cs(const CUtensorMap& map, const uint16_t* norms, const float* 
   cfg.attrs = attr;
   cfg.numAttrs = (flags & HLWQ_FLAG_WEIGHTS_STATIC) ? 1 : 0;
   const int ob = out_bf16 ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, gemv1_kernel<C, S>, map, norms, codebook, O, in, nb, x, Y, ob, pass_rows, xvec) !=
-      cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemv1_kernel<C, S>, map, norms, codebook, g1_lloyd_max_centroids(), O, in, nb, x, Y,
+                         ob, pass_rows, xvec) != cudaSuccess)
     return HLWQ_ECUDA;
   return HLWQ_OK;
 }

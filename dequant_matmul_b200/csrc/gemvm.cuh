@@ -7,14 +7,13 @@
 // Items, lanes, code ring and pair table are those of gemv1_kernel: a lane
 // decodes the same half block of two rows per item, every pair of codes costs
 // a shift, an and-or and one shared load per row, and each table entry then
-// feeds one half2 FMA per token.  The tokens' rotated activations live in
+// feeds two fp32-accumulating mixed-precision FMAs per token.  The tokens' rotated activations live in
 // shared memory interleaved by token: for (block b, pair pp of the block) the
 // MT half2 values sit side by side, so one 8- or 16-byte load gives a lane all
 // tokens' values for a pair; each half block's units are padded by one so
 // that the lanes of a warp (different blocks and halves, same pair) hit
-// different banks.  Each (row, token) accumulates in two fp16 chains of 16 products
-// (a block's codes have sum c^2 ~ 128, so |sum| <= sqrt(135) * 4 * 2^10 <
-// 65504), widened once per item; the two rows of a lane are reduced over the
+// different banks.  Each (row, token) accumulates in two fp32 sums (the
+// pair's halves); the two rows of a lane are reduced over the
 // row's 2C lanes together, per token, and the chunk partials are summed at the
 // end in a fixed order (deterministic).
 
@@ -57,24 +56,22 @@ struct XVec<4> {
   __device__ static void get(const T& v, uint32_t (&o)[4]) { o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w; }
 };
 
-// Pair P of both rows against all tokens; chain P & 1.
+// Pair P of both rows against all tokens: every binary16 product is added to
+// an fp32 accumulator (two per row and token: the pair's halves).
 template <int MT, int P>
 __device__ __forceinline__ void gm_pair(const uint8_t* tab, const uint2 (&cw0)[5], const uint2 (&cw1)[5],
                                         uint32_t lane4, const typename XVec<MT>::T* xrow,
-                                        uint32_t (&h0)[MT][2], uint32_t (&h1)[MT][2]) {
+                                        float (&h0)[MT][2], float (&h1)[MT][2]) {
   const uint32_t e0 = *reinterpret_cast<const uint32_t*>(tab + g1_off<P>(cw0, lane4));
   const uint32_t e1 = *reinterpret_cast<const uint32_t*>(tab + g1_off<P>(cw1, lane4));
   uint32_t x[MT];
   XVec<MT>::get(xrow[P], x);
 #pragma unroll
   for (int t = 0; t < MT; ++t) {
-    if constexpr (P < 2) {
-      h0[t][P] = hmul2(e0, x[t]);
-      h1[t][P] = hmul2(e1, x[t]);
-    } else {
-      h0[t][P & 1] = hfma2(e0, x[t], h0[t][P & 1]);
-      h1[t][P & 1] = hfma2(e1, x[t], h1[t][P & 1]);
-    }
+    h0[t][0] = fma_lo(e0, x[t], h0[t][0]);
+    h0[t][1] = fma_hi(e0, x[t], h0[t][1]);
+    h1[t][0] = fma_lo(e1, x[t], h1[t][0]);
+    h1[t][1] = fma_hi(e1, x[t], h1[t][1]);
   }
 }
 
@@ -82,14 +79,14 @@ template <int MT, int... P>
 __device__ __forceinline__ void gm_dot(const uint8_t* tab, const uint2 (&cw0)[5], const uint2 (&cw1)[5],
                                        uint32_t lane4, const typename XVec<MT>::T* xrow, float (&a0)[MT],
                                        float (&a1)[MT], std::integer_sequence<int, P...>) {
-  uint32_t h0[MT][2], h1[MT][2];
+  float h0[MT][2], h1[MT][2];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) h0[t][0] = h0[t][1] = h1[t][0] = h1[t][1] = 0.0f;
   (gm_pair<MT, P>(tab, cw0, cw1, lane4, xrow, h0, h1), ...);
 #pragma unroll
   for (int t = 0; t < MT; ++t) {
-    const float2 f0 = half2_to_float2(hadd2(h0[t][0], h0[t][1]));
-    const float2 f1 = half2_to_float2(hadd2(h1[t][0], h1[t][1]));
-    a0[t] = f0.x + f0.y;
-    a1[t] = f1.x + f1.y;
+    a0[t] = h0[t][0] + h0[t][1];
+    a1[t] = h1[t][0] + h1[t][1];
   }
 }
 

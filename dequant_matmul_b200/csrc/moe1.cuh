@@ -239,9 +239,9 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
           const int b = cch * C + s;
           moe1_load_x(xs, xinv, (t - t_lo) * nb + b, b < nb, hh, xr, xi);
         }
-        const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+        const float a0 = g1_dot(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
                          (half_bits_to_float(static_cast<uint16_t>(nr0)) * xi);
-        const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+        const float a1 = g1_dot(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
                          (half_bits_to_float(static_cast<uint16_t>(nr1)) * xi);
         const bool hi = (u & C) != 0;
         float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);
@@ -396,9 +396,9 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
             const int b = cch * C + s;
             moe1_load_x(xs, xinv, (cp - pg0) * nb + b, b < nb, hh, xr, xi);
           }
-          const float a0 = g1_dot_n<8>(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+          const float a0 = g1_dot(smem, cw0, lane4, xr, std::make_integer_sequence<int, 32>{}) *
                            (half_bits_to_float(static_cast<uint16_t>(nq0)) * xi);
-          const float a1 = g1_dot_n<8>(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
+          const float a1 = g1_dot(smem, cw1, lane4, xr, std::make_integer_sequence<int, 32>{}) *
                            (half_bits_to_float(static_cast<uint16_t>(nq1)) * xi);
           const bool hi = (u & C) != 0;
           float acc = (hi ? a1 : a0) + __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, C);

@@ -92,6 +92,28 @@ def test_gemv_ex_weights_static_chain(hl, cb):
         assert rel_l2(y.double().cpu().numpy(), want) <= MATMUL_REL
 
 
+@pytest.mark.parametrize("flags", [0, 1])
+def test_gemv_caller_codebook_replaces_the_expected_one(hl, cb, flags):
+    """The single-token GEMV builds its table from the Lloyd-Max centroids it
+    expects and rebuilds it when the caller's codebook differs.  With every
+    centroid doubled (exact in binary16 and fp32) each product and each fp32
+    partial sum doubles exactly, so y must be exactly 2 y; a codebook scaled
+    by 1.6 must give 1.6 y within the matmul tolerance."""
+    W, q = _layer((1024, 5120), seed=31)
+    p, n = oracle_to_dev(q)
+    x = synth.activations(1, 5120, seed=32)[0].cuda()
+    y1 = hl.gemv(p, n, cb, x, flags=flags)
+    y2 = hl.gemv(p, n, (cb * 2).contiguous(), x, flags=flags)
+    y3 = hl.gemv(p, n, (cb * 1.6).contiguous(), x, flags=flags)
+    y4 = hl.gemv(p, n, cb, x, flags=flags)   # back to the expected codebook
+    torch.cuda.synchronize()
+    assert torch.equal(y2, 2 * y1)
+    assert torch.equal(y4, y1)
+    want = O.matmul(q["packed"], q["norms"], 5120, x.cpu()[None])[0]
+    assert rel_l2(y3.double().cpu().numpy(), 1.6 * want) <= MATMUL_REL
+    assert hl.device_error() == 0
+
+
 def test_gemv_ex_rejects_unknown_flags(hl, cb):
     W, q = _layer((64, 256), seed=3)
     p, n = oracle_to_dev(q)
