@@ -271,6 +271,21 @@ extern "C" size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, 
   return 0;
 }
 
+extern "C" int hlwq_fault_inject(unsigned int skip_tma, unsigned long long wait_ns) {
+#ifdef HLWQ_FAULT_INJECTION
+  if (wait_ns == 0 || wait_ns > hlwq::kWaitTimeoutNs) return HLWQ_EINVAL;
+  const unsigned int skip = skip_tma ? 1u : 0u;
+  if (cudaDeviceSynchronize() != cudaSuccess) return HLWQ_ECUDA;
+  if (cudaMemcpyToSymbol(hlwq::g_fault_skip_tma, &skip, sizeof(skip)) != cudaSuccess) return HLWQ_ECUDA;
+  if (cudaMemcpyToSymbol(hlwq::g_fault_wait_ns, &wait_ns, sizeof(wait_ns)) != cudaSuccess) return HLWQ_ECUDA;
+  return HLWQ_OK;
+#else
+  (void)skip_tma;
+  (void)wait_ns;
+  return HLWQ_EUNSUPPORTED;
+#endif
+}
+
 extern "C" int hlwq_device_error(uint32_t* bits) {
   if (!bits) return HLWQ_EINVAL;
   if (cudaDeviceSynchronize() != cudaSuccess) return HLWQ_ECUDA;

@@ -46,7 +46,6 @@ constexpr int kTcTileRows = 128;
 constexpr int kTcKChunk = 64;                 // K elements per pipeline stage (one half block)
 constexpr int kTcAccCols = 256;               // TMEM columns reserved for the accumulator
 constexpr int kTcAllocCols = 512;   // accumulator (256) + 3 A stages of 64
-constexpr uint64_t kTcTimeoutNs = kWaitTimeoutNs;
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -268,7 +267,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   }
   const int64_t o0 = static_cast<int64_t>(tt % row_tiles) * kTcTileRows;
   const int n0 = (tt / row_tiles) * n_box;
-  const uint64_t deadline = globaltimer_ns() + kTcTimeoutNs;
+  const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
 
   // ---- set-up: codebook, barriers, TMEM
   if (threadIdx.x < kLevels) {
@@ -476,36 +475,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // ---------------------------------------------------------- TMA producer: code tiles
     if (lane == 0) {
       bool ok = true;
+      int last = -1;  // last block whose copy was issued
       for (int b = kb0; b < kb1; ++b) {
         const int cs = tc_code_stage(b - kb0, G);
         ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
+        if (fault_skip_tma()) continue;
         mbar_arrive_expect_tx(c_full0 + 8 * cs, kTcCodeBytes);
         tma_load_2d(cst + cs * kTcCodeBytes, &cmap, kBlockBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
+        last = b;
       }
       if (!ok) {
         misc_g[1] = 1u;
         raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
+      // no copy may still be landing when the CTA exits: wait (bounded) for
+      // the last copy issued into each code stage
+      const uint64_t dl = globaltimer_ns() + wait_limit_ns();
+      for (int b = std::max(kb0, last - CS + 1); b <= last; ++b)
+        mbar_wait(c_full0 + 8 * tc_code_stage(b - kb0, G), tc_code_parity(b - kb0, G), dl);
     }
   } else if (warp == kTcWB) {
     // ---------------------------------------------------------- TMA producer: B tiles
     if (lane == 0) {
       const uint32_t half_bytes = static_cast<uint32_t>(n_box) * 128u;
       bool ok = true;
+      int last = -1;  // last block whose copies were issued
       for (int b = kb0; b < kb1; ++b) {
         const int st = tc_ab_stage(b - kb0, G);
         ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
+        if (fault_skip_tma()) continue;
         mbar_arrive_expect_tx(full0 + 8 * st, 2 * half_bytes);
         const uint32_t dst = bst + st * n_box * 256;
         tma_load_2d(dst, &bmap, kTcKChunk * (2 * b), n0, full0 + 8 * st);
         tma_load_2d(dst + half_bytes, &bmap, kTcKChunk * (2 * b + 1), n0, full0 + 8 * st);
+        last = b;
       }
       if (!ok) {
         misc_g[1] = 1u;
         raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
+      // wait (bounded) for the last copies issued into each A/B stage (the
+      // decode warps arrive on every stage they take, so a stage's phase
+      // completes once its bytes have landed)
+      const uint64_t dl = globaltimer_ns() + wait_limit_ns();
+      for (int b = std::max(kb0, last - G + 1); b <= last; ++b)
+        mbar_wait(full0 + 8 * tc_ab_stage(b - kb0, G), tc_ab_parity(b - kb0, G), dl);
     }
   } else if (warp == kTcWMma) {
     // ---------------------------------------------------------- MMA issuer
@@ -533,6 +549,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
       tc_commit(accum);  // fires once every MMA issued above has completed
+      // the commit's arrival lands before the CTA can exit (bounded)
+      mbar_wait(accum, 0, globaltimer_ns() + wait_limit_ns());
     }
   }
 

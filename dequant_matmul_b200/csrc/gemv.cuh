@@ -363,7 +363,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     fence_barrier_init();
   }
   __syncwarp();
-  const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
+  const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
   bool ok = true;
   uint32_t phase = 0;    // parity of the next completion, one bit per slot
   uint32_t pending = 0;  // slots with a box in flight
@@ -382,7 +382,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     const uint16_t* nptr = norms + (prow0 + ig * RG + r) * nb + ich * C + s;
     uint32_t nlo[S], nhi[S];  // the two rows' norms, kept apart so that no instruction waits on them before use
     auto issue = [&](int d) {
-      if (lane == 0) {
+      if (lane == 0 && !fault_skip_tma()) {
         mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
         tma_load_3d(ring + d * kG1ItemBytes, &cmap, 0, ich * C, static_cast<int>(prow0 + ig * RG), bar + 8 * d);
       }
@@ -498,7 +498,7 @@ gemv1_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restric
     }
     if (!ok) {
       // a box never arrived: drain what is still in flight (bounded), then stop
-      const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
+      const uint64_t dl = globaltimer_ns() + wait_limit_ns();
       for (int d = 0; d < S; ++d)
         if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
       if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);

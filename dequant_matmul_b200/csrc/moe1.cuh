@@ -160,7 +160,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
   g1_build_table(smem, c16r, nroute, kG1Warps - nroute);
   __syncthreads();  // routing, table, barriers
 
-  const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
+  const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
   bool ok = true;
   uint32_t phase = 0, pending = 0;
   const int nitems = nq * nch;  // chunk-major: item k = (chunk k / nq, group q0 + k % nq)
@@ -173,7 +173,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
     const int e = rid[p];
     const bool sh = e == P.E;
     const int64_t rbase = sh ? 0 : static_cast<int64_t>(e) * F2;
-    if (lane == 0) {
+    if (lane == 0 && !fault_skip_tma()) {
       mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
       const CUtensorMap* m = sh ? &smap : &gmap;
       tma_load_3d(ring + d * kG1ItemBytes, m, 0, ich * C, static_cast<int>(rbase + j0), bar + 8 * d);
@@ -253,7 +253,7 @@ moe_gu1_kernel(const __grid_constant__ CUtensorMap gmap, const __grid_constant__
     }
   }
   if (!ok) {
-    const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
+    const uint64_t dl = globaltimer_ns() + wait_limit_ns();
     for (int d = 0; d < S; ++d)
       if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
     if (lane == 0) raise_device_error(HLWQ_DEVERR_TIMEOUT);
@@ -316,7 +316,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
   g1_build_table(smem, c16r, nroute, kG1Warps - nroute);
   __syncthreads();  // routing, table, barriers
 
-  const uint64_t deadline = globaltimer_ns() + kWaitTimeoutNs;
+  const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
   bool ok = true;
   uint32_t phase = 0, pending = 0;
   for (int pg0 = 0; pg0 < NP; pg0 += pg_max) {
@@ -331,7 +331,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
       const bool sh = e == P.E;
       const int64_t rbase = sh ? 0 : static_cast<int64_t>(e) * H;
       const int lrow = (g0 + ilg) * RG;  // first output row of the item
-      if (lane == 0) {
+      if (lane == 0 && !fault_skip_tma()) {
         mbar_arrive_expect_tx(bar + 8 * d, kG1ItemBytes);
         tma_load_3d(ring + d * kG1ItemBytes, sh ? &smap : &dmap, 0, ich * C, static_cast<int>(rbase + lrow),
                     bar + 8 * d);
@@ -413,7 +413,7 @@ moe_dn1_kernel(const __grid_constant__ CUtensorMap dmap, const __grid_constant__
       }
     }
     if (!ok) {
-      const uint64_t dl = globaltimer_ns() + kWaitTimeoutNs;
+      const uint64_t dl = globaltimer_ns() + wait_limit_ns();
       for (int d = 0; d < S; ++d)
         if ((pending >> d) & 1u) mbar_wait(bar + 8 * d, (phase >> d) & 1u, dl);
       pending = 0;

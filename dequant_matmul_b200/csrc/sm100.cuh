@@ -12,6 +12,24 @@ namespace hlwq {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // every mbarrier wait gives up after 2 s
 
+#ifdef HLWQ_FAULT_INJECTION
+// Failure-detection test build only (libhlwq_fault.so; hlwq_fault_inject):
+// the TMA producers can be told to issue nothing, so that every consumer's
+// bounded wait runs out with no copy in flight, and the wait limit can be
+// shortened.  The product library compiles these to constants.
+__device__ unsigned int g_fault_skip_tma = 0u;
+__device__ unsigned long long g_fault_wait_ns = kWaitTimeoutNs;
+__device__ __forceinline__ bool fault_skip_tma() {
+  return *reinterpret_cast<volatile unsigned int*>(&g_fault_skip_tma) != 0u;
+}
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_fault_wait_ns);
+}
+#else
+__device__ __forceinline__ constexpr bool fault_skip_tma() { return false; }
+__device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitTimeoutNs; }
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

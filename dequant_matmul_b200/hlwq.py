@@ -48,6 +48,7 @@ SIGNATURES = {
     "hlwq_gemm_noalloc": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P]),
     "hlwq_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I64, _I64]),
     "hlwq_device_error": (_I, [_P]),
+    "hlwq_fault_inject": (_I, [ctypes.c_uint, ctypes.c_ulonglong]),
     "hlwq_status_string": (ctypes.c_char_p, [_I]),
     "hlwq_version": (_I, []),
 }
@@ -57,10 +58,16 @@ class HLWQError(RuntimeError):
     pass
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libhlwq.so not built ({LIB_PATH}); run __graft_entry__.build()")
-    lib = ctypes.CDLL(LIB_PATH)
+# Failure-detection test build (hlwq_fault_inject is live there); never used by
+# the functions below unless a test swaps it in as `lib`.
+FAULT_LIB_PATH = os.path.join(_PKG, "libhlwq_fault.so")
+
+
+def load_library(path: str):
+    """Loads a build of the library and declares the header's signatures."""
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built ({path}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.restype = res
@@ -68,7 +75,7 @@ def _load():
     return lib
 
 
-lib = _load()
+lib = load_library(LIB_PATH)
 
 
 def _check(status: int, what: str):

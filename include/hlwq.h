@@ -307,6 +307,23 @@ int hlwq_gemm_noalloc(const uint8_t* packed, const uint16_t* norms, const float*
                       int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx,
                       void* Y, int64_t ldy, int ydtype, void* stream);
 
+/*
+ * Failure-detection test hook.  No counterpart in the paper.  Only the test
+ * build of the library (libhlwq_fault.so, compiled with HLWQ_FAULT_INJECTION)
+ * implements it; the product library returns HLWQ_EUNSUPPORTED and its
+ * kernels contain none of this.
+ *   skip_tma  nonzero: the TMA producers of the GEMV, few-token, fused-MoE and
+ *             tensor-core GEMM kernels issue no copies, so every consumer's
+ *             bounded wait runs out (no copy is ever in flight); the kernel
+ *             then raises HLWQ_DEVERR_TIMEOUT, frees its tensor memory and
+ *             returns without writing a result it could not compute.
+ *   wait_ns   the limit of every bounded wait (1 .. 2e9 ns; 2e9 is the
+ *             product value).
+ * Synchronises the current device first.  Errors: HLWQ_EINVAL (wait_ns),
+ * HLWQ_ECUDA, HLWQ_EUNSUPPORTED (product build).
+ */
+int hlwq_fault_inject(unsigned int skip_tma, unsigned long long wait_ns);
+
 /* Reads (after synchronising the current device) and clears the device error word. */
 int hlwq_device_error(uint32_t* bits);
 
