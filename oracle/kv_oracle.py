@@ -27,9 +27,13 @@ Readings where the pages are silent (pinned in tests/test_oracle_kv.py):
       the lower index (a zero vector gets code 3 everywhere).
   K4  Pack: code j at bits [3j, 3j + 3) of the vector's little-endian 768-bit
       field, i.e. 8 codes per 3 bytes, LSB first (as reading R6 with 3 bits).
-  K5  The residual buffer is the cache's policy, not an encoding step: the 128
-      most recent tokens of a sequence are kept in bf16 and enter the encoded
-      cache (this encoding) as they leave that window.
+  K5  The 128-token residual buffer of recent tokens kept without
+      quantization: the cache of one head is the encoded tokens followed by the window of the
+      most recent min(128, total) tokens, kept exactly as given (bf16).  A
+      token is encoded when it leaves the window, oldest first
+      (kv_window_append), and attention scores cover every cached token in
+      order: decoded keys for the encoded ones, the exact keys for the window
+      (kv_scores_window).
 """
 
 from __future__ import annotations
@@ -75,3 +79,36 @@ def kv_scores(Q, packed, norms) -> np.ndarray:
     if q.ndim == 1:
         q = q[None, :]
     return q @ kv_dequantize(packed, norms).T
+
+
+def kv_window_append(packed, norms, window, x_new, capacity: int = RESIDUAL_TOKENS):
+    """The cache after appending the tokens x_new [t][256] (reading K5).
+
+    The window's tokens (oldest first) are followed by the new ones; all but
+    the `capacity` most recent leave the window in order and are encoded with
+    kv_quantize and appended to (packed, norms).  Returns (packed uint8 [n][96],
+    norms float16 [n], window float64 [w][256], w <= capacity)."""
+    if capacity < 1:
+        raise ValueError("capacity must be >= 1")
+    win = _as_f64(window).reshape(-1, HEAD_DIM)
+    new = _as_f64(x_new).reshape(-1, HEAD_DIM)
+    tokens = np.concatenate([win, new], axis=0)
+    leave = max(0, tokens.shape[0] - capacity)
+    packed = np.asarray(packed, dtype=np.uint8).reshape(-1, KV_BYTES)
+    norms = np.asarray(norms, dtype=np.float16).reshape(-1)
+    if leave:
+        q = kv_quantize(tokens[:leave])
+        packed = np.concatenate([packed, q["packed"]], axis=0)
+        norms = np.concatenate([norms, q["norms"]])
+    return packed, norms, tokens[leave:]
+
+
+def kv_scores_window(Q, packed, norms, window) -> np.ndarray:
+    """scores [M][n + w] against every cached token in order: the n encoded
+    keys (kv_scores) followed by the w window keys, exact (q . k in fp64)."""
+    q = _as_f64(Q)
+    if q.ndim == 1:
+        q = q[None, :]
+    win = _as_f64(window).reshape(-1, HEAD_DIM)
+    enc = kv_scores(q, packed, norms) if np.asarray(packed).shape[0] else np.zeros((q.shape[0], 0))
+    return np.concatenate([enc, q @ win.T], axis=1)

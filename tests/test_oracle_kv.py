@@ -90,3 +90,101 @@ def test_scores_in_the_rotated_domain():
     alt = (qt @ c32.astype(np.float64)[r["codes"]].T) * (r["norms"].astype(np.float64) / 256.0)[None, :]
     assert np.allclose(s, alt, rtol=1e-12, atol=1e-12)
     assert s.shape == (4, 30)
+
+
+# --------------------------------------------------------------------------
+# The 128-token residual window (reading K5; "Qwopus3.6-27B-v2 . HLWQ Q5",
+# Methodology notes, KV-cache bullet).
+# --------------------------------------------------------------------------
+
+def _tokens(n, seed):
+    g = np.random.default_rng(seed)
+    return g.standard_normal((n, 256)).astype(np.float32)
+
+
+def _append_all(tokens, chunks, capacity=O.RESIDUAL_TOKENS, append=None):
+    append = append or O.kv_window_append
+    p = np.zeros((0, 96), np.uint8)
+    n = np.zeros((0,), np.float16)
+    w = np.zeros((0, 256))
+    i = 0
+    for c in chunks:
+        p, n, w = append(p, n, w, tokens[i:i + c], capacity)
+        i += c
+    return p, n, w
+
+
+def _window_is_the_recent_tokens(append) -> bool:
+    """After appending N tokens in any batching, the encoded part is
+    kv_quantize of tokens [0, N - 128) and the window holds tokens
+    [N - 128, N) exactly, oldest first."""
+    X = _tokens(400, 5)
+    for chunks in ([400], [1] * 130 + [270], [5, 200, 1, 128, 66], [127, 1, 1, 271]):
+        p, n, w = _append_all(X, chunks, append=append)
+        want = O.kv_quantize(X[:400 - 128])
+        if not (np.array_equal(p, want["packed"]) and np.array_equal(n.view(np.uint16), want["norms"].view(np.uint16))
+                and np.array_equal(w, X[400 - 128:].astype(np.float64))):
+            return False
+    return True
+
+
+def test_window_keeps_the_128_most_recent_tokens():
+    assert O.RESIDUAL_TOKENS == 128
+    assert _window_is_the_recent_tokens(O.kv_window_append)
+
+
+def test_window_encodes_nothing_until_it_is_full():
+    X = _tokens(128, 6)
+    p, n, w = _append_all(X, [100, 28])
+    assert p.shape == (0, 96) and n.shape == (0,)
+    assert np.array_equal(w, X.astype(np.float64))
+    p, n, w = _append_all(X[:1], [1], capacity=1)
+    assert p.shape == (0, 96) and w.shape == (1, 256)
+
+
+def test_window_scores_with_an_empty_window_are_the_encoded_scores():
+    X = _tokens(300, 7)
+    Q = _tokens(3, 8)
+    r = O.kv_quantize(X)
+    s = O.kv_scores_window(Q, r["packed"], r["norms"], np.zeros((0, 256)))
+    assert np.array_equal(s, O.kv_scores(Q, r["packed"], r["norms"]))
+
+
+def test_window_scores_of_exact_keys_equal_integer_dot_products():
+    """With small-integer keys and queries every product and sum is an integer,
+    computed here in Python integers: the window part is the exact dot."""
+    g = np.random.default_rng(9)
+    K = g.integers(-8, 9, size=(128, 256))
+    Q = g.integers(-8, 9, size=(2, 256))
+    s = O.kv_scores_window(Q.astype(np.float32), np.zeros((0, 96), np.uint8), np.zeros(0, np.float16),
+                           K.astype(np.float32))
+    want = [[sum(int(a) * int(b) for a, b in zip(q, k)) for k in K] for q in Q]
+    assert np.array_equal(s, np.array(want, dtype=np.float64))
+
+
+def test_window_scores_cover_every_cached_token_in_order():
+    X = _tokens(200, 10)
+    Q = _tokens(2, 11)
+    p, n, w = _append_all(X, [3, 197])
+    s = O.kv_scores_window(Q, p, n, w)
+    assert s.shape == (2, 200)
+    assert np.array_equal(s[:, :72], O.kv_scores(Q, p, n))
+    assert np.allclose(s[:, 72:], Q.astype(np.float64) @ X[72:].astype(np.float64).T, rtol=0, atol=1e-9)
+
+
+def test_window_planted_mistakes_fail_the_pin():
+    """Evicting the newest tokens instead of the oldest, or keeping one token
+    too many, fails the recent-tokens pin."""
+    def newest_first(p, n, w, x, cap):
+        t = np.concatenate([np.asarray(w, np.float64).reshape(-1, 256), np.asarray(x, np.float64).reshape(-1, 256)])
+        leave = max(0, t.shape[0] - cap)
+        if leave:
+            q = O.kv_quantize(t[t.shape[0] - leave:])
+            p, n = np.concatenate([p, q["packed"]]), np.concatenate([n, q["norms"]])
+        return p, n, t[:t.shape[0] - leave]
+
+    def one_too_many(p, n, w, x, cap):
+        return O.kv_window_append(p, n, w, x, cap + 1)
+
+    assert not _window_is_the_recent_tokens(newest_first)
+    assert not _window_is_the_recent_tokens(one_too_many)
