@@ -415,7 +415,40 @@ def bench_kv(hl, peaks, stream):
     b = N * (96 + 2 + 6 * 4)
     res["scores_6q"] = {"ms": round(ms, 4), "keys_per_s_G": round(N / ms / 1e6, 2), "gbs": round(b / ms / 1e6, 1),
                         "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
-    del X, packed, norms, out16, Q, S
+    # the residual window: one head's 32768 tokens, the last 128 kept exact
+    # (scores of the GQA group over encoded + window keys in one launch), and
+    # a decode step's append of one token (which encodes the token leaving
+    # the window)
+    T1 = 32768
+    cache = hl.KVWindowCache(capacity=T1, R=128, cb8=cb8)
+    cache.append(X[:T1 - 1])
+    Sw = torch.empty(6, T1 - 1, dtype=torch.float32, device="cuda")
+    ms, _ = time_graph(lambda: cache.scores(Q, S=Sw, stream=stream), reps=10, warmup=3, stream=stream)
+    b = cache.n_enc * (96 + 2) + 128 * 512 + (T1 - 1) * 6 * 4
+    res["window_scores_6q_32767tok"] = {"ms": round(ms, 4), "keys_per_s_G": round((T1 - 1) / ms / 1e6, 2),
+                                        "gbs": round(b / ms / 1e6, 1), "encoded": cache.n_enc, "window": 128}
+    x1 = X[T1 - 1:T1]
+    st = (cache.n_enc, cache.n_total)
+    win0 = cache.window.clone()
+
+    def append_one():
+        # restore the state each replay so every step appends the same token
+        cache.n_enc, cache.n_total = st
+        cache.append(x1, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            append_one()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(20):
+            append_one()
+        e1.record(stream)
+        e1.synchronize()
+    cache.window.copy_(win0)
+    res["window_append_1tok"] = {"us": round(e0.elapsed_time(e1) * 1e3 / 20, 2),
+                                 "note": "eager calls (host bookkeeping between launches): encodes 1 token, copies 1"}
+    del X, packed, norms, out16, Q, S, cache, Sw
     return {"kv_q3_131072x256": res}
 
 

@@ -30,7 +30,11 @@ int launch_kv_quantize(const uint16_t* X, int64_t n, int64_t ldx, const float* c
 int launch_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t n, void* out,
                          bool bf16, cudaStream_t stream);
 int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
-                     const float* codebook, int64_t n, float* S, int64_t lds, cudaStream_t stream);
+                     const float* codebook, int64_t n_enc, const uint16_t* window, int64_t R, int64_t n_total,
+                     float* S, int64_t lds, cudaStream_t stream);
+int launch_kv_window_append(const uint16_t* X, int64_t t, int64_t ldx, uint16_t* window, int64_t R, int64_t n_enc,
+                            int64_t n_total, const float* codebook, uint8_t* packed, uint16_t* norms,
+                            int64_t* n_enc_out, cudaStream_t stream);
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
                  const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
 int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
@@ -164,7 +168,39 @@ extern "C" int hlwq_kv_scores(const uint16_t* q, int64_t m, int64_t ldq, const u
   if (!aligned2(q) || (reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms) ||
       (reinterpret_cast<uintptr_t>(scores) & 3u))
     return HLWQ_EALIGN;
-  return hlwq::launch_kv_scores(q, m, ldq, packed, norms, codebook8, n, scores, lds, as_stream(stream));
+  return hlwq::launch_kv_scores(q, m, ldq, packed, norms, codebook8, n, nullptr, 1, n, scores, lds,
+                                as_stream(stream));
+}
+
+extern "C" int hlwq_kv_scores_window(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* packed,
+                                     const uint16_t* norms, const float* codebook8, int64_t n_enc,
+                                     const uint16_t* window, int64_t R, int64_t n_total, float* scores, int64_t lds,
+                                     void* stream) {
+  constexpr int64_t kMaxTokens = int64_t(1) << 40;
+  if (!q || !codebook8 || !scores || m <= 0 || ldq < 256 || n_enc < 0 || n_total > kMaxTokens || n_total <= 0 ||
+      n_enc > n_total || lds < n_total || R < 1 || R > kMaxIn || n_total - n_enc > R)
+    return HLWQ_EINVAL;
+  if (n_enc > 0 && (!packed || !norms)) return HLWQ_EINVAL;
+  if (n_total > n_enc && !window) return HLWQ_EINVAL;
+  if (m > 64) return HLWQ_EUNSUPPORTED;
+  if (!aligned2(q) || (reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms) || !aligned16(window) ||
+      (reinterpret_cast<uintptr_t>(scores) & 3u))
+    return HLWQ_EALIGN;
+  return hlwq::launch_kv_scores(q, m, ldq, packed, norms, codebook8, n_enc, window, R, n_total, scores, lds,
+                                as_stream(stream));
+}
+
+extern "C" int hlwq_kv_window_append(const uint16_t* x, int64_t t, int64_t ldx, uint16_t* window, int64_t R,
+                                     int64_t n_enc, int64_t n_total, const float* codebook8, uint8_t* packed,
+                                     uint16_t* norms, int64_t* n_enc_out, void* stream) {
+  constexpr int64_t kMaxTokens = int64_t(1) << 40;
+  if (!window || !codebook8 || !packed || !norms || t < 0 || (t > 0 && !x) || ldx < 256 || R < 1 || R > kMaxIn ||
+      n_enc < 0 || n_enc > n_total || n_total - n_enc > R || n_total > kMaxTokens || t > kMaxTokens - n_total)
+    return HLWQ_EINVAL;
+  if (!aligned2(x) || !aligned16(window) || (reinterpret_cast<uintptr_t>(packed) & 3u) || !aligned2(norms))
+    return HLWQ_EALIGN;
+  return hlwq::launch_kv_window_append(x, t, ldx, window, R, n_enc, n_total, codebook8, packed, norms, n_enc_out,
+                                       as_stream(stream));
 }
 
 extern "C" int hlwq_gemv(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t out,

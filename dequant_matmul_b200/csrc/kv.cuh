@@ -218,10 +218,15 @@ kv_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restr
 constexpr int kKvQRow = kKvDim + 32;
 __host__ __device__ inline int kv_qpos(int m, int p) { return m * kKvQRow + p + 4 * (p >> 5); }
 
+// Scores against the cached keys 0 .. n_total - 1: keys r < n_enc from their
+// codes, keys n_enc <= r < n_total exactly from the residual window (bf16 ring
+// of R slots, key r in slot r % R), rotated here like the queries, so that
+// q . k = (q H) . (k H) / 256 in both cases.
 __global__ void __launch_bounds__(kKvThreads)
 kv_scores_kernel(const uint16_t* __restrict__ Q, int m_count, int64_t ldq, const uint8_t* __restrict__ packed,
-                 const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t n,
-                 float* __restrict__ S, int64_t lds) {
+                 const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t n_enc,
+                 const uint16_t* __restrict__ window, int64_t R, int64_t n_total, float* __restrict__ S,
+                 int64_t lds) {
   extern __shared__ __align__(16) float qs[];  // [m_count][288]
   __shared__ float cb[kKvLevels];
   kv_check_codebook(codebook);
@@ -245,21 +250,49 @@ kv_scores_kernel(const uint16_t* __restrict__ Q, int m_count, int64_t ldq, const
   __syncthreads();
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kKvThreads + threadIdx.x) >> 5;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kKvThreads / 32);
-  for (int64_t first = gwarp * 4; first < n; first += nwarps * 4) {
+  for (int64_t first = gwarp * 4; first < n_total; first += nwarps * 4) {
     const int64_t r = first + (lane >> 3);
-    const bool active = r < n;
-    uint32_t w[3] = {0u, 0u, 0u};
-    float sc = 0.0f;
-    if (active) {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + r * kKvBytes + 12 * l8);
-      w[0] = __ldg(src);
-      w[1] = __ldg(src + 1);
-      w[2] = __ldg(src + 2);
-      sc = half_bits_to_float(__ldg(norms + r)) * (1.0f / 256.0f);
-    }
+    const bool active = r < n_total;
+    const bool exact = active && r >= n_enc;  // a window key
     float c[32];
+    float sc = 0.0f;
+    if (__any_sync(0xffffffffu, exact)) {
+      // window keys of this warp's four keys (zero for the others), rotated
+      // with the queries' butterflies
+      float v[32];
+      if (exact) {
+        const uint4* src = reinterpret_cast<const uint4*>(window + (r % R) * kKvDim + 32 * l8);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) c[e] = cb[kv_code(w, e)];
+        for (int k = 0; k < 4; ++k) {
+          const uint4 u = __ldg(src + k);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            v[8 * k + 2 * h] = bf16x2_lo(w4[h]);
+            v[8 * k + 2 * h + 1] = bf16x2_hi(w4[h]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+      }
+      kv_fwht(v, lane);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) c[e] = v[e];
+      if (exact) sc = 1.0f / 256.0f;
+    }
+    if (!exact) {
+      uint32_t w[3] = {0u, 0u, 0u};
+      if (active) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + r * kKvBytes + 12 * l8);
+        w[0] = __ldg(src);
+        w[1] = __ldg(src + 1);
+        w[2] = __ldg(src + 2);
+        sc = half_bits_to_float(__ldg(norms + r)) * (1.0f / 256.0f);
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) c[e] = cb[kv_code(w, e)];
+    }
     for (int m = 0; m < m_count; ++m) {
       const float4* qm = reinterpret_cast<const float4*>(qs + kv_qpos(m, 32 * l8));
       float acc = 0.0f;
@@ -298,7 +331,8 @@ int launch_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const flo
 }
 
 int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
-                     const float* codebook, int64_t n, float* S, int64_t lds, cudaStream_t stream) {
+                     const float* codebook, int64_t n_enc, const uint16_t* window, int64_t R, int64_t n_total,
+                     float* S, int64_t lds, cudaStream_t stream) {
   const int smem = static_cast<int>(m) * kKvQRow * 4;
   static PerDeviceOnce attr;
   if (const int st = attr([&] {
@@ -307,10 +341,50 @@ int launch_kv_scores(const uint16_t* Q, int64_t m, int64_t ldq, const uint8_t* p
       }))
     return st;
   const int64_t max_ctas = static_cast<int64_t>(sm_count()) * 4;
-  const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(n, kKvThreads / 8)));
-  kv_scores_kernel<<<grid, kKvThreads, smem, stream>>>(Q, static_cast<int>(m), ldq, packed, norms, codebook, n, S,
-                                                       lds);
+  const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(n_total, kKvThreads / 8)));
+  kv_scores_kernel<<<grid, kKvThreads, smem, stream>>>(Q, static_cast<int>(m), ldq, packed, norms, codebook, n_enc,
+                                                       window, R > 0 ? R : 1, n_total, S, lds);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+}
+
+// Appends t tokens to a cache of n_enc encoded tokens and a residual window
+// (ring of R slots) holding tokens n_enc .. n_total - 1: the tokens that leave
+// the window (oldest first) are encoded into rows n_enc .. n_enc2 - 1, then
+// the new tokens that stay are copied into their slots.  Stream order keeps
+// every window slot read (encoded) before it is overwritten: a new token that
+// stays in slot i % R replaces token i - R, which always leaves.
+int launch_kv_window_append(const uint16_t* X, int64_t t, int64_t ldx, uint16_t* window, int64_t R, int64_t n_enc,
+                            int64_t n_total, const float* codebook, uint8_t* packed, uint16_t* norms,
+                            int64_t* n_enc_out, cudaStream_t stream) {
+  const int64_t n_total2 = n_total + t;
+  const int64_t n_enc2 = std::max(n_enc, n_total2 - R);
+  // old window tokens that leave: [n_enc, min(n_enc2, n_total)), in ring segments
+  for (int64_t i = n_enc; i < std::min(n_enc2, n_total);) {
+    const int64_t slot = i % R;
+    const int64_t cnt = std::min(std::min(n_enc2, n_total) - i, R - slot);
+    const int st = launch_kv_quantize(window + slot * kKvDim, cnt, kKvDim, codebook, packed + i * kKvBytes,
+                                      norms + i, stream);
+    if (st != HLWQ_OK) return st;
+    i += cnt;
+  }
+  // new tokens that leave at once: [max(n_total, n_enc), n_enc2)
+  const int64_t d0 = std::max(n_total, n_enc);
+  if (n_enc2 > d0) {
+    const int st = launch_kv_quantize(X + (d0 - n_total) * ldx, n_enc2 - d0, ldx, codebook, packed + d0 * kKvBytes,
+                                      norms + d0, stream);
+    if (st != HLWQ_OK) return st;
+  }
+  // new tokens that stay: [max(n_total, n_enc2), n_total2), in ring segments
+  for (int64_t i = std::max(n_total, n_enc2); i < n_total2;) {
+    const int64_t slot = i % R;
+    const int64_t cnt = std::min(n_total2 - i, R - slot);
+    if (cudaMemcpy2DAsync(window + slot * kKvDim, kKvDim * 2, X + (i - n_total) * ldx, ldx * 2, kKvDim * 2,
+                          cnt, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+      return HLWQ_ECUDA;
+    i += cnt;
+  }
+  if (n_enc_out) *n_enc_out = n_enc2;
+  return HLWQ_OK;
 }
 
 }  // namespace hlwq

@@ -40,6 +40,8 @@ SIGNATURES = {
     "hlwq_kv_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_dequantize": (_I, [_P, _P, _P, _I64, _P, _I, _P]),
     "hlwq_kv_scores": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _I64, _P]),
+    "hlwq_kv_window_append": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "hlwq_kv_scores_window": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _I64, _I64, _P, _I64, _P]),
     "hlwq_gemv": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
     "hlwq_gemv_ex": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _I, ctypes.c_uint, _P]),
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
@@ -298,6 +300,43 @@ def kv_scores(Q: torch.Tensor, packed, norms, cb8, S=None, stream=None):
     _check(lib.hlwq_kv_scores(_ptr(Q), M, Q.stride(0), _ptr(packed), _ptr(norms), _ptr(cb8), N, _ptr(S), S.stride(0),
                               _stream(stream)), "hlwq_kv_scores")
     return S
+
+
+class KVWindowCache:
+    """One head's Q3 KV cache with its residual window (hlwq_kv_window_append /
+    hlwq_kv_scores_window): `capacity` encoded rows preallocated, a bf16 ring
+    of R slots for the most recent tokens.  Bookkeeping only; the device work
+    is the library's."""
+
+    def __init__(self, capacity: int, R: int = 128, device="cuda", cb8=None):
+        self.packed = torch.zeros(capacity, 96, dtype=torch.uint8, device=device)
+        self.norms = torch.zeros(capacity, dtype=torch.uint16, device=device)
+        self.window = torch.zeros(R, 256, dtype=torch.bfloat16, device=device)
+        self.R, self.n_enc, self.n_total = R, 0, 0
+        self.cb8 = cb8 if cb8 is not None else kv_codebook(device)
+
+    def append(self, X: torch.Tensor, stream=None):
+        """X bf16 [t][256] (row pitch X.stride(0))."""
+        _cuda_rows(X, "X")
+        t = X.shape[0]
+        if self.n_total + t - self.R > self.packed.shape[0]:
+            raise HLWQError("KVWindowCache: capacity of encoded rows exceeded")
+        out = ctypes.c_int64()
+        _check(lib.hlwq_kv_window_append(_ptr(X), t, X.stride(0), _ptr(self.window), self.R, self.n_enc,
+                                         self.n_total, _ptr(self.cb8), _ptr(self.packed), _ptr(self.norms),
+                                         ctypes.byref(out), _stream(stream)), "hlwq_kv_window_append")
+        self.n_enc, self.n_total = out.value, self.n_total + t
+
+    def scores(self, Q: torch.Tensor, S=None, stream=None):
+        """Q bf16 [M][256] (M <= 64) -> S fp32 [M][n_total] over every cached token."""
+        _cuda_rows(Q, "Q")
+        M = Q.shape[0]
+        if S is None:
+            S = torch.empty(M, self.n_total, dtype=torch.float32, device=Q.device)
+        _check(lib.hlwq_kv_scores_window(_ptr(Q), M, Q.stride(0), _ptr(self.packed), _ptr(self.norms), _ptr(self.cb8),
+                                         self.n_enc, _ptr(self.window), self.R, self.n_total, _ptr(S), S.stride(0),
+                                         _stream(stream)), "hlwq_kv_scores_window")
+        return S
 
 
 def gemv(packed, norms, cb, x: torch.Tensor, out_dtype=torch.float32, y=None, stream=None, flags: int = 0):

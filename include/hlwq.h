@@ -163,10 +163,30 @@ int hlwq_requantize_int4(const uint8_t* packed, const uint16_t* norms, const flo
  *   aligned) = n16 * (c[code] @ H256) / 256.
  * hlwq_kv_scores: S[m][i] = q_m . x_hat_i for M <= 64 bf16 queries [M][ldq]
  *   (fp32, row pitch lds >= N); evaluated with each query rotated once.
- * The 128 most recent tokens (the residual buffer) are the caller's: they stay
- * in bf16 and are encoded as they leave that window.
  * Errors: HLWQ_EINVAL, HLWQ_EALIGN (packed 4-byte, norms / x / q 2-byte
  * alignment), HLWQ_EUNSUPPORTED (dtype; M > 64), HLWQ_ECUDA.
+ *
+ * The residual window (same card and bullet: the most recent 128 tokens stay
+ * unquantized).  A cache of one head holds n_total tokens: tokens
+ * 0 .. n_enc - 1 encoded (packed / norms rows), tokens n_enc .. n_total - 1 in
+ * the window, a bf16 ring of R slots [R][256] (token i in slot i % R,
+ * n_total - n_enc <= R; R = 128 for the cards' buffer).  The caller owns
+ * every buffer and gives packed / norms room for the rows that get encoded.
+ * hlwq_kv_window_append: appends t bf16 tokens x [t][ldx]; with
+ *   n_total' = n_total + t and n_enc' = max(n_enc, n_total' - R), tokens
+ *   n_enc .. n_enc' - 1 (oldest first, from the window or, when t > R, from
+ *   x) are encoded into rows n_enc .. n_enc' - 1 exactly as hlwq_kv_quantize
+ *   would, and the new tokens that stay are copied into their slots.
+ *   *n_enc_out (host, may be NULL) receives n_enc'.  Asynchronous on stream;
+ *   window, packed and norms must not be used by other streams meanwhile.
+ * hlwq_kv_scores_window: S[m][i] for every cached token i < n_total: the
+ *   decoded key for i < n_enc (as hlwq_kv_scores), the exact window key
+ *   otherwise (q . k in fp32); one launch.  window may be NULL when
+ *   n_total == n_enc, packed / norms when n_enc == 0.
+ * Errors: HLWQ_EINVAL (counts out of range: n_enc > n_total, more than R
+ * tokens in the window, lds < n_total), HLWQ_EALIGN (window 16-byte,
+ * packed 4-byte, norms / x / q 2-byte), HLWQ_EUNSUPPORTED (M > 64),
+ * HLWQ_ECUDA.
  */
 int hlwq_kv_quantize(const uint16_t* x, int64_t n, int64_t ldx, const float* codebook8, uint8_t* packed,
                      uint16_t* norms, void* stream);
@@ -174,6 +194,13 @@ int hlwq_kv_dequantize(const uint8_t* packed, const uint16_t* norms, const float
                        void* out, int odtype, void* stream);
 int hlwq_kv_scores(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* packed, const uint16_t* norms,
                    const float* codebook8, int64_t n, float* scores, int64_t lds, void* stream);
+int hlwq_kv_window_append(const uint16_t* x, int64_t t, int64_t ldx, uint16_t* window, int64_t R,
+                          int64_t n_enc, int64_t n_total, const float* codebook8, uint8_t* packed,
+                          uint16_t* norms, int64_t* n_enc_out, void* stream);
+int hlwq_kv_scores_window(const uint16_t* q, int64_t m, int64_t ldq, const uint8_t* packed,
+                          const uint16_t* norms, const float* codebook8, int64_t n_enc,
+                          const uint16_t* window, int64_t R, int64_t n_total, float* scores, int64_t lds,
+                          void* stream);
 
 /*
  * TQ3 weights, the scalar case of HIGGS ("Qwen3.6-35B-A3B-TQ3-native", "What

@@ -125,3 +125,22 @@ def test_noalloc_validates_arguments_before_sizing_its_scratch(hl):
     # a tensor-core request above the static scratch (512 x 64 blocks x 256 B)
     assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 128, 8192, 512) > hl.NOALLOC_SCRATCH_BYTES
     assert L.hlwq_gemm_noalloc(p, p, p, 128, 8192, 512, p, 8192, p, 128, F32, None) == hl.HLWQ_ESCRATCH
+
+
+def test_kv_window_validation(hl):
+    L = hl.lib
+    p = ctypes.c_void_p(256)
+    out = ctypes.c_int64()
+    # more tokens in the window than its R slots
+    assert L.hlwq_kv_window_append(p, 1, 256, p, 128, 0, 129, p, p, p, ctypes.byref(out), None) == hl.HLWQ_EINVAL
+    assert L.hlwq_kv_window_append(p, 1, 256, p, 128, 5, 4, p, p, p, None, None) == hl.HLWQ_EINVAL    # n_enc > n_total
+    assert L.hlwq_kv_window_append(p, 1, 128, p, 128, 0, 0, p, p, p, None, None) == hl.HLWQ_EINVAL    # ldx < 256
+    assert L.hlwq_kv_window_append(None, 1, 256, p, 128, 0, 0, p, p, p, None, None) == hl.HLWQ_EINVAL # no x
+    assert L.hlwq_kv_window_append(p, 1, 256, ctypes.c_void_p(264), 128, 0, 0, p, p, p, None,
+                                   None) == hl.HLWQ_EALIGN                                         # window 8-byte
+    assert L.hlwq_kv_window_append(p, 1, 256, p, 0, 0, 0, p, p, p, None, None) == hl.HLWQ_EINVAL      # R = 0
+    assert L.hlwq_kv_scores_window(p, 2, 256, p, p, p, 10, p, 128, 9, p, 16, None) == hl.HLWQ_EINVAL  # n_enc > n_total
+    assert L.hlwq_kv_scores_window(p, 2, 256, p, p, p, 0, p, 128, 200, p, 256, None) == hl.HLWQ_EINVAL  # > R in window
+    assert L.hlwq_kv_scores_window(p, 2, 256, p, p, p, 10, None, 128, 20, p, 20, None) == hl.HLWQ_EINVAL  # no window
+    assert L.hlwq_kv_scores_window(p, 2, 256, p, p, p, 10, p, 128, 20, p, 19, None) == hl.HLWQ_EINVAL  # lds < n_total
+    assert L.hlwq_kv_scores_window(p, 65, 256, p, p, p, 10, p, 128, 20, p, 20, None) == hl.HLWQ_EUNSUPPORTED

@@ -95,3 +95,80 @@ def test_kv_codebook_error_word(hl, cb8):
     torch.cuda.synchronize()
     assert hl.device_error() & 0x1
     assert hl.device_error() == 0
+
+
+# --------------------------------------------------------------------------
+# Residual window: appends encode the tokens that leave the window, oldest
+# first, bit-exact with the oracle; scores cover encoded and exact keys.
+# --------------------------------------------------------------------------
+
+def _window_state_matches(cache, Xall, n_total, R):
+    """Encoded rows and window slots against the oracle's state after the
+    same tokens."""
+    n_enc = max(0, n_total - R)
+    assert cache.n_enc == n_enc and cache.n_total == n_total
+    if n_enc:
+        want = O.kv_quantize(Xall[:n_enc])
+        assert np.array_equal(cache.packed[:n_enc].cpu().numpy(), want["packed"])
+        assert np.array_equal(cache.norms[:n_enc].cpu().numpy(), want["norms"].view(np.uint16))
+    win = cache.window.cpu()
+    for i in range(n_enc, n_total):
+        assert torch.equal(win[i % R], Xall[i]), i
+
+
+@pytest.mark.parametrize("R,chunks", [(128, [1, 3, 200, 1, 128, 50, 7]), (5, [2, 2, 9, 1, 1, 13]),
+                                      (128, [300])])
+def test_kv_window_append_matches_the_oracle(hl, cb8, R, chunks):
+    Xall = _keys(sum(chunks), seed=R + len(chunks))
+    cache = hl.KVWindowCache(capacity=sum(chunks), R=R, cb8=cb8)
+    n = 0
+    for c in chunks:
+        cache.append(Xall[n:n + c].cuda())
+        n += c
+        torch.cuda.synchronize()
+        _window_state_matches(cache, Xall, n, R)
+    assert hl.device_error() == 0
+
+
+@pytest.mark.parametrize("R,n_tokens,m", [(128, 1000, 6), (128, 100, 3), (7, 40, 64), (128, 128, 1)])
+def test_kv_scores_window_one_launch(hl, cb8, R, n_tokens, m):
+    Xall = _keys(n_tokens, seed=n_tokens + m)
+    Q = synth.activations(m, 256, seed=19 + m)
+    cache = hl.KVWindowCache(capacity=n_tokens, R=R, cb8=cb8)
+    cache.append(Xall.cuda())
+    S = cache.scores(Q.cuda())
+    torch.cuda.synchronize()
+    p, nrm, w = O.kv_window_append(np.zeros((0, 96), np.uint8), np.zeros(0, np.float16), np.zeros((0, 256)),
+                                   Xall, capacity=R)
+    want = O.kv_scores_window(Q, p, nrm, w)
+    got = S.cpu().numpy()
+    assert got.shape == want.shape == (m, n_tokens)
+    ne = cache.n_enc
+    if ne:
+        assert rel_l2(got[:, :ne], want[:, :ne]) <= 1e-5
+    # exact keys: fp32 rotation and dot against the fp64 dot of the bf16 values
+    assert rel_l2(got[:, ne:], want[:, ne:]) <= 1e-6
+
+
+def test_kv_scores_window_edges(hl, cb8):
+    """A cache with no window tokens (window may be NULL) equals hlwq_kv_scores;
+    a cache with no encoded tokens scores only exact keys."""
+    K = _keys(300, seed=23)
+    Q = synth.activations(4, 256, seed=24).cuda()
+    kq = O.kv_quantize(K)
+    p = torch.from_numpy(kq["packed"]).cuda()
+    nr = torch.from_numpy(kq["norms"].view(np.uint16)).cuda()
+    S0 = hl.kv_scores(Q, p, nr, cb8)
+    S1 = torch.empty(4, 300, dtype=torch.float32, device="cuda")
+    st = hl.lib.hlwq_kv_scores_window(hl._ptr(Q), 4, 256, hl._ptr(p), hl._ptr(nr), hl._ptr(cb8), 300, None, 128, 300,
+                                      hl._ptr(S1), 300, None)
+    assert st == hl.HLWQ_OK
+    win = K[:100].cuda()
+    S2 = torch.empty(4, 100, dtype=torch.float32, device="cuda")
+    st = hl.lib.hlwq_kv_scores_window(hl._ptr(Q), 4, 256, None, None, hl._ptr(cb8), 0, hl._ptr(win), 128, 100,
+                                      hl._ptr(S2), 100, None)
+    assert st == hl.HLWQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(S0, S1)
+    want = Q.cpu().double().numpy() @ K[:100].double().numpy().T
+    assert rel_l2(S2.cpu().numpy(), want) <= 1e-6
