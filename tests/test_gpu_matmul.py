@@ -114,6 +114,35 @@ def test_gemv_caller_codebook_replaces_the_expected_one(hl, cb, flags):
     assert hl.device_error() == 0
 
 
+@pytest.mark.parametrize("M", [1, 3, 16])
+def test_accumulation_with_one_dominant_rotated_value_per_block(hl, cb, M):
+    """Each 128-block of x is 4 H[j] plus noise of std 0.1 (kept by bf16), so
+    its rotated block is one value 512 beside values ~500x smaller, and a few
+    rows have norms 1000x the others; y (fp32 and bf16 out) must stay within
+    the matmul tolerance (every product is added to an fp32 accumulator)."""
+    O_, I = 512, 2048
+    W = synth.student_t((O_, I), df4_seed=33).double()
+    W[::37] *= 1000.0
+    W = W.to(torch.bfloat16)
+    q = O.quantize(W)
+    p, n = oracle_to_dev(q)
+    H = O.sylvester_hadamard(128).astype(np.float64)
+    g = np.random.default_rng(34)
+    X = np.empty((M, I))
+    for m in range(M):
+        for b in range(I // 128):
+            j = int(g.integers(0, 128))
+            X[m, 128 * b:128 * (b + 1)] = 4.0 * H[j] + 0.1 * g.standard_normal(128)
+    Xb = torch.from_numpy(X).to(torch.bfloat16)
+    want = O.matmul(q["packed"], q["norms"], I, Xb)
+    for odt in (torch.float32, torch.bfloat16):
+        Y = hl.gemm(p, n, cb, Xb.cuda(), out_dtype=odt)
+        torch.cuda.synchronize()
+        err = rel_l2(Y.double().cpu().numpy(), want)
+        print(f"[margin] dominant rotated value, M={M}, {odt}: rel L2 {err:.2e} (bar {MATMUL_REL})")
+        assert err <= MATMUL_REL, (odt, err)
+
+
 def test_gemv_ex_rejects_unknown_flags(hl, cb):
     W, q = _layer((64, 256), seed=3)
     p, n = oracle_to_dev(q)
