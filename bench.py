@@ -136,10 +136,6 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- helpers
-def flush_l2(buf):
-    buf.zero_()
-
-
 def time_graph(fn, reps: int, warmup: int, stream):
     """Captures fn() in a CUDA graph and times `reps` replays with CUDA events."""
     import torch
@@ -190,14 +186,13 @@ def components(hl, cb, peaks, stream, parts=("quantize", "gemm", "moe", "int4", 
     from dequant_matmul_b200 import synth
     out = {}
     torch.cuda.synchronize()
-    scrub = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     if "quantize" in parts:
         out.update(bench_quantize(hl, cb, peaks, stream))
     if "gemm" in parts:
         out.update(bench_gemm(hl, cb, peaks, stream))
     if "moe" in parts:
-        out.update(bench_moe(hl, cb, peaks, stream, scrub))
+        out.update(bench_moe(hl, cb, peaks, stream))
     if "int4" in parts:
         out.update(bench_int4(hl, cb, peaks, stream))
     if "kv" in parts:
@@ -452,11 +447,43 @@ def bench_kv(hl, peaks, stream):
     return {"kv_q3_131072x256": res}
 
 
-def bench_moe(hl, cb, peaks, stream, scrub):
+def bench_moe(hl, cb, peaks, stream):
+    """MoE layers.  Each timed call routes its own tokens: a graph replays R
+    calls with R different routings (logits and activations), R chosen so
+    that the experts the calls read add up to more than twice the L2, so
+    every call reads its experts from HBM without an L2 scrub.  GB/s counts
+    each call's distinct experts once."""
     import torch
     from dequant_matmul_b200 import synth
     out = {}
-    # MoE: 256 experts + shared, hidden 2048, intermediate 512, top-8.
+
+    def layer(gu, dn, shared, E, H, F, T, per_expert, seed):
+        n_sh = 1 if shared is not None else 0
+        est = min(E, T * 8) + n_sh                                   # distinct experts, upper estimate
+        R = max(2, min(32, -(-2 * 126 * 2 ** 20 // (est * per_expert))))
+        sets = []
+        for r in range(R):
+            g = torch.Generator(device="cuda").manual_seed(seed + 1000 * r + T)
+            sets.append((torch.randn(T, E, generator=g, device="cuda"),
+                         synth.activations_device(T, H, seed=seed + 7 * r + T),
+                         torch.empty(T, H, dtype=torch.float32, device="cuda"),
+                         torch.empty(T, 8, dtype=torch.int32, device="cuda"),
+                         torch.empty(T, 8, dtype=torch.float32, device="cuda")))
+        ws = torch.empty(hl.workspace_bytes(hl.HLWQ_OP_MOE, H, F, T, E, 8), dtype=torch.uint8, device="cuda")
+
+        def run():
+            for lg, X, Y, ids, wts in sets:
+                hl.moe_gemv(gu, dn, cb, lg, X, 8, shared=shared, Y=Y, ids=ids, weights=wts, workspace=ws,
+                            stream=stream)
+
+        ms, _ = time_graph(run, reps=10, warmup=3, stream=stream)
+        ms /= R
+        distinct = sum(int(torch.unique(st[3]).numel()) + n_sh for st in sets) / R
+        byts = distinct * per_expert
+        return {"ms": round(ms, 4), "distinct_experts": round(distinct, 1), "routings": R,
+                "gbs": round(byts / ms / 1e6, 1), "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
+
+    # 256 experts + shared, hidden 2048, intermediate 512, top-8.
     E4, H4, F4 = 256, 2048, 512
     gu_w = synth.student_t_device((E4, 2 * F4, H4), seed=70)
     dn_w = synth.student_t_device((E4, H4, F4), seed=71)
@@ -466,54 +493,16 @@ def bench_moe(hl, cb, peaks, stream, scrub):
     sh = (hl.quantize(synth.student_t_device((2 * F4, H4), seed=72), cb, stream=stream),
           hl.quantize(synth.student_t_device((H4, F4), seed=73), cb, stream=stream))
     per_expert = (2 * F4 * 16 + H4 * 4) * 82
-    moe = {}
-    for T in (1, 8, 64):
-        logits = torch.randn(T, E4, generator=torch.Generator(device="cuda").manual_seed(T), device="cuda")
-        X = synth.activations_device(T, H4, seed=80 + T)
-        Y = torch.empty(T, H4, dtype=torch.float32, device="cuda")
-        ids = torch.empty(T, 8, dtype=torch.int32, device="cuda")
-        wts = torch.empty(T, 8, dtype=torch.float32, device="cuda")
-        ws = torch.empty(hl.workspace_bytes(hl.HLWQ_OP_MOE, H4, F4, T, E4, 8), dtype=torch.uint8, device="cuda")
-
-        def run_moe():
-            flush_l2(scrub)
-            hl.moe_gemv(gu, dn, cb, logits, X, 8, shared=sh, Y=Y, ids=ids, weights=wts, workspace=ws, stream=stream)
-
-        ms_all, _ = time_graph(run_moe, reps=20, warmup=3, stream=stream)
-        ms_flush, _ = time_graph(lambda: flush_l2(scrub), reps=20, warmup=3, stream=stream)
-        ms = max(ms_all - ms_flush, 1e-6)
-        distinct = int(torch.unique(ids).numel()) + 1
-        byts = distinct * per_expert
-        moe[f"T{T}"] = {"ms": round(ms, 4), "distinct_experts": distinct, "gbs": round(byts / ms / 1e6, 1),
-                        "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
-    out["moe_256x(1024x2048+2048x512)_top8_shared"] = moe
+    out["moe_256x(1024x2048+2048x512)_top8_shared"] = {f"T{T}": layer(gu, dn, sh, E4, H4, F4, T, per_expert, 80)
+                                                       for T in (1, 8, 64)}
     del gu, dn, sh
-    # MoE: the 128-expert layer, hidden 2816, intermediate 704 (tail block
+    # the 128-expert layer, hidden 2816, intermediate 704 (tail block
     # zero-padded), top-8, no shared expert, T = 1 and 16.
     E5, H5, F5 = 128, 2816, 704
     gu5 = hl.quantize(synth.student_t_device((E5, 2 * F5, H5), seed=90), cb, stream=stream)
     dn5 = hl.quantize(synth.student_t_device((E5, H5, F5), seed=91), cb, stream=stream)
     per_expert5 = (2 * F5 * 22 + H5 * 6) * 82
-    moe5 = {}
-    for T in (1, 16):
-        logits = torch.randn(T, E5, generator=torch.Generator(device="cuda").manual_seed(100 + T), device="cuda")
-        X = synth.activations_device(T, H5, seed=110 + T)
-        Y = torch.empty(T, H5, dtype=torch.float32, device="cuda")
-        ids = torch.empty(T, 8, dtype=torch.int32, device="cuda")
-        wts = torch.empty(T, 8, dtype=torch.float32, device="cuda")
-        ws = torch.empty(hl.workspace_bytes(hl.HLWQ_OP_MOE, H5, F5, T, E5, 8), dtype=torch.uint8, device="cuda")
-
-        def run_moe5():
-            flush_l2(scrub)
-            hl.moe_gemv(gu5, dn5, cb, logits, X, 8, Y=Y, ids=ids, weights=wts, workspace=ws, stream=stream)
-
-        ms_all, _ = time_graph(run_moe5, reps=20, warmup=3, stream=stream)
-        ms_flush, _ = time_graph(lambda: flush_l2(scrub), reps=20, warmup=3, stream=stream)
-        ms = max(ms_all - ms_flush, 1e-6)
-        distinct = int(torch.unique(ids).numel())
-        byts = distinct * per_expert5
-        moe5[f"T{T}"] = {"ms": round(ms, 4), "distinct_experts": distinct, "gbs": round(byts / ms / 1e6, 1),
-                         "hbm_frac": frac(byts / ms / 1e6, peaks["hbm_gbs"])}
+    moe5 = {f"T{T}": layer(gu5, dn5, None, E5, H5, F5, T, per_expert5, 110) for T in (1, 16)}
     out["moe_128x(1408x2816+2816x704)_top8"] = moe5
     return out
 
