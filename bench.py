@@ -457,7 +457,7 @@ def bench_moe(hl, cb, peaks, stream):
     from dequant_matmul_b200 import synth
     out = {}
 
-    def layer(gu, dn, shared, E, H, F, T, per_expert, seed):
+    def layer(gu, dn, shared, E, H, F, T, per_expert, seed, flags=0):
         n_sh = 1 if shared is not None else 0
         est = min(E, T * 8) + n_sh                                   # distinct experts, upper estimate
         R = max(2, min(32, -(-2 * 126 * 2 ** 20 // (est * per_expert))))
@@ -474,7 +474,7 @@ def bench_moe(hl, cb, peaks, stream):
         def run():
             for lg, X, Y, ids, wts in sets:
                 hl.moe_gemv(gu, dn, cb, lg, X, 8, shared=shared, Y=Y, ids=ids, weights=wts, workspace=ws,
-                            stream=stream)
+                            stream=stream, flags=flags)
 
         ms, _ = time_graph(run, reps=10, warmup=3, stream=stream)
         ms /= R
@@ -493,8 +493,12 @@ def bench_moe(hl, cb, peaks, stream):
     sh = (hl.quantize(synth.student_t_device((2 * F4, H4), seed=72), cb, stream=stream),
           hl.quantize(synth.student_t_device((H4, F4), seed=73), cb, stream=stream))
     per_expert = (2 * F4 * 16 + H4 * 4) * 82
-    out["moe_256x(1024x2048+2048x512)_top8_shared"] = {f"T{T}": layer(gu, dn, sh, E4, H4, F4, T, per_expert, 80)
-                                                       for T in (1, 8, 64)}
+    moe4 = {f"T{T}": layer(gu, dn, sh, E4, H4, F4, T, per_expert, 80) for T in (1, 8, 64)}
+    # the grouped path (HLWQ_FLAG_MOE_GROUPED: each active expert read once
+    # for all its tokens), for comparison at the larger token counts
+    for T in (8, 64):
+        moe4[f"T{T}_grouped"] = layer(gu, dn, sh, E4, H4, F4, T, per_expert, 80, flags=hl.HLWQ_FLAG_MOE_GROUPED)
+    out["moe_256x(1024x2048+2048x512)_top8_shared"] = moe4
     del gu, dn, sh
     # the 128-expert layer, hidden 2816, intermediate 704 (tail block
     # zero-padded), top-8, no shared expert, T = 1 and 16.

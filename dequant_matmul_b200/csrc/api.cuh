@@ -258,12 +258,13 @@ extern "C" int hlwq_gemm(const uint8_t* packed, const uint16_t* norms, const flo
                             ydtype == HLWQ_BF16, as_stream(stream));
 }
 
-extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
-                             const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
-                             const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook,
-                             int64_t E, int64_t H, int64_t F, int64_t topk, int64_t T, const float* router_logits,
-                             const uint16_t* X, void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
-                             void* workspace, size_t ws_bytes, void* stream) {
+extern "C" int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+                                const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                                const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook,
+                                int64_t E, int64_t H, int64_t F, int64_t topk, int64_t T, const float* router_logits,
+                                const uint16_t* X, void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
+                                void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+  if (flags & ~static_cast<unsigned>(HLWQ_FLAG_MOE_GROUPED)) return HLWQ_EINVAL;
   if (!gu_packed || !gu_norms || !dn_packed || !dn_norms || !codebook || !router_logits || !X || !Y)
     return HLWQ_EINVAL;
   if (E <= 0 || E > 1024 || H <= 0 || H > kMaxIn || F <= 0 || F > kMaxIn || T <= 0 || T > 65535 || topk <= 0 ||
@@ -286,7 +287,7 @@ extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
   // path that reads each active expert once for all its tokens
   hlwq::MoeWs ws;
   hlwq::moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
-  const int st = hlwq::launch_moe1(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+  const int st = (flags & HLWQ_FLAG_MOE_GROUPED) ? HLWQ_EUNSUPPORTED : hlwq::launch_moe1(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
                                    sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H),
                                    static_cast<int>(F), static_cast<int>(topk), static_cast<int>(T), router_logits, X,
                                    Y, ydtype == HLWQ_BF16, topk_ids, topk_weights, ws.h, as_stream(stream));
@@ -295,6 +296,17 @@ extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
                           sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H), static_cast<int>(F),
                           static_cast<int>(topk), static_cast<int>(T), router_logits, X, Y, ydtype == HLWQ_BF16,
                           topk_ids, topk_weights, workspace, as_stream(stream));
+}
+
+extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+                             const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                             const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook,
+                             int64_t E, int64_t H, int64_t F, int64_t topk, int64_t T, const float* router_logits,
+                             const uint16_t* X, void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  return hlwq_moe_gemv_ex(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+                          sh_dn_norms, codebook, E, H, F, topk, T, router_logits, X, Y, ydtype, topk_ids, topk_weights,
+                          workspace, ws_bytes, 0u, stream);
 }
 
 extern "C" size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk) {

@@ -22,6 +22,7 @@ NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 + 64 * 1024
 HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
 HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
 HLWQ_FLAG_WEIGHTS_STATIC = 1
+HLWQ_FLAG_MOE_GROUPED = 2
 DEVERR_CODEBOOK, DEVERR_TIMEOUT, DEVERR_CODE_RANGE = 0x1, 0x2, 0x4
 BLOCK, BLOCK_BYTES, LEVELS = 128, 80, 32
 
@@ -47,6 +48,8 @@ SIGNATURES = {
     "hlwq_gemm": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "hlwq_moe_gemv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _I,
                            _P, _P, _P, _SZ, _P]),
+    "hlwq_moe_gemv_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _I,
+                              _P, _P, _P, _SZ, ctypes.c_uint, _P]),
     "hlwq_gemm_noalloc": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P]),
     "hlwq_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I64, _I64]),
     "hlwq_device_error": (_I, [_P]),
@@ -373,7 +376,7 @@ def gemm(packed, norms, cb, X: torch.Tensor, out_dtype=torch.bfloat16, Y=None, w
 
 
 def moe_gemv(gu, dn, cb, logits, X, topk: int, shared=None, out_dtype=torch.float32, Y=None, ids=None,
-             weights=None, workspace=None, stream=None):
+             weights=None, workspace=None, stream=None, flags: int = 0):
     """gu = (packed [E][2F][NBh][80], norms [E][2F][NBh]); dn = (packed [E][H][NBf][80], norms [E][H][NBf]);
     shared = ((packed, norms) of gate_up, (packed, norms) of down) or None.
     logits fp32 [T][E], X bf16 [T][H].  Returns (Y, ids, weights)."""
@@ -393,10 +396,16 @@ def moe_gemv(gu, dn, cb, logits, X, topk: int, shared=None, out_dtype=torch.floa
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     sg = shared[0] if shared is not None else (None, None)
     sd = shared[1] if shared is not None else (None, None)
-    _check(lib.hlwq_moe_gemv(_ptr(gu[0]), _ptr(gu[1]), _ptr(dn[0]), _ptr(dn[1]), _ptr(sg[0]), _ptr(sg[1]),
-                             _ptr(sd[0]), _ptr(sd[1]), _ptr(cb), E, H, F, topk, T, _ptr(logits), _ptr(X), _ptr(Y),
-                             _dtype_code(Y.dtype), _ptr(ids), _ptr(weights), _ptr(workspace), workspace.numel(),
-                             _stream(stream)), "hlwq_moe_gemv")
+    if flags:
+        _check(lib.hlwq_moe_gemv_ex(_ptr(gu[0]), _ptr(gu[1]), _ptr(dn[0]), _ptr(dn[1]), _ptr(sg[0]), _ptr(sg[1]),
+                                    _ptr(sd[0]), _ptr(sd[1]), _ptr(cb), E, H, F, topk, T, _ptr(logits), _ptr(X),
+                                    _ptr(Y), _dtype_code(Y.dtype), _ptr(ids), _ptr(weights), _ptr(workspace),
+                                    workspace.numel(), flags, _stream(stream)), "hlwq_moe_gemv_ex")
+    else:
+        _check(lib.hlwq_moe_gemv(_ptr(gu[0]), _ptr(gu[1]), _ptr(dn[0]), _ptr(dn[1]), _ptr(sg[0]), _ptr(sg[1]),
+                                 _ptr(sd[0]), _ptr(sd[1]), _ptr(cb), E, H, F, topk, T, _ptr(logits), _ptr(X),
+                                 _ptr(Y), _dtype_code(Y.dtype), _ptr(ids), _ptr(weights), _ptr(workspace),
+                                 workspace.numel(), _stream(stream)), "hlwq_moe_gemv")
     return Y, ids, weights
 
 

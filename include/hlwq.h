@@ -70,7 +70,7 @@ typedef enum { HLWQ_F32 = 0, HLWQ_BF16 = 1, HLWQ_F16 = 2 } hlwq_dtype;
 typedef enum { HLWQ_OP_GEMM = 1, HLWQ_OP_MOE = 2 } hlwq_op;
 
 /* Launch flags of the *_ex calls. */
-typedef enum { HLWQ_FLAG_WEIGHTS_STATIC = 1 } hlwq_flags;
+typedef enum { HLWQ_FLAG_WEIGHTS_STATIC = 1, HLWQ_FLAG_MOE_GROUPED = 2 } hlwq_flags;
 
 /* Device error bits (hlwq_device_error). */
 #define HLWQ_DEVERR_CODEBOOK 0x1u  /* codebook not strictly ascending or not finite */
@@ -299,6 +299,25 @@ int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
                   int64_t T, const float* router_logits, const uint16_t* X,
                   void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
                   void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * hlwq_moe_gemv with launch flags.  flags = 0 is hlwq_moe_gemv (the fused
+ * two-kernel path when its shared memory fits -- few tokens -- else the
+ * grouped path).  HLWQ_FLAG_MOE_GROUPED selects the grouped path at any T:
+ * four launches (routing and per-expert assignment lists with every token's
+ * rotated activation; gate_up over (active expert, 32 columns) units that
+ * read each active expert's codes once for all its tokens; down over (active
+ * expert, 128 rows) units; a fixed-order combine).  Same arguments, results
+ * and workspace; other bits are HLWQ_EINVAL.
+ */
+int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_norms,
+                     const uint8_t* dn_packed, const uint16_t* dn_norms,
+                     const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                     const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms,
+                     const float* codebook, int64_t E, int64_t H, int64_t F, int64_t topk,
+                     int64_t T, const float* router_logits, const uint16_t* X,
+                     void* Y, int ydtype, int32_t* topk_ids, float* topk_weights,
+                     void* workspace, size_t ws_bytes, unsigned flags, void* stream);
 
 /*
  * Scratch bytes for an operation (0 when none is needed).

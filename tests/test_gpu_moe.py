@@ -28,7 +28,7 @@ def expert_weights(E, H, F, seed):
     return gu, dn
 
 
-def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_only=False):
+def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_only=False, flags=0):
     """Oracle-quantized experts on both sides (only the experts the oracle's
     router picks are encoded when used_only; the others stay zero on the GPU)."""
     logits = synth.router_logits(T, E, seed=seed)
@@ -58,7 +58,7 @@ def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_onl
               (torch.from_numpy(qd["packed"]).cuda(), torch.from_numpy(qd["norms"].view(np.uint16)).cuda()))
     gu = (torch.from_numpy(gu_p).cuda(), torch.from_numpy(gu_n).cuda())
     dn = (torch.from_numpy(dn_p).cuda(), torch.from_numpy(dn_n).cuda())
-    Y, ids, w = hl.moe_gemv(gu, dn, cb, logits.cuda(), X.cuda(), topk, shared=sh, out_dtype=odt)
+    Y, ids, w = hl.moe_gemv(gu, dn, cb, logits.cuda(), X.cuda(), topk, shared=sh, out_dtype=odt, flags=flags)
     torch.cuda.synchronize()
     want, ids_o, w_o = O.moe_forward(gu_o, dn_o, H, F, topk, logits, X, sg_o, sd_o)
     assert np.array_equal(ids.cpu().numpy(), ids_o)
@@ -71,6 +71,47 @@ def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_onl
 @pytest.mark.parametrize("T,topk,shared", [(1, 8, True), (5, 2, False), (17, 8, True), (3, 1, False)])
 def test_moe_small(hl, cb, T, topk, shared):
     run_case(hl, cb, E=16, H=256, F=128, T=T, topk=topk, shared=shared, seed=100 + T)
+
+
+# ----------------------------------------------------------------------------
+# The grouped path (four launches, each active expert read once for all its
+# tokens): selected with HLWQ_FLAG_MOE_GROUPED, and taken by default when the
+# fused path's shared memory does not fit (many tokens).
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,topk,shared", [(1, 8, True), (5, 2, False), (17, 8, True), (64, 8, True)])
+def test_moe_grouped_path(hl, cb, T, topk, shared):
+    run_case(hl, cb, E=16, H=256, F=128, T=T, topk=topk, shared=shared, seed=600 + T, flags=hl.HLWQ_FLAG_MOE_GROUPED)
+
+
+def test_moe_grouped_path_ragged_and_bf16(hl, cb):
+    run_case(hl, cb, E=8, H=320, F=176, T=6, topk=3, shared=True, seed=607, flags=hl.HLWQ_FLAG_MOE_GROUPED)
+    run_case(hl, cb, E=8, H=256, F=128, T=4, topk=2, shared=False, seed=608, odt=torch.bfloat16,
+             flags=hl.HLWQ_FLAG_MOE_GROUPED)
+
+
+def test_moe_grouped_path_full_shapes_t1(hl, cb):
+    run_case(hl, cb, E=256, H=2048, F=512, T=1, topk=8, shared=True, seed=610, used_only=True,
+             flags=hl.HLWQ_FLAG_MOE_GROUPED)
+    run_case(hl, cb, E=128, H=2816, F=704, T=1, topk=8, shared=False, seed=611, used_only=True,
+             flags=hl.HLWQ_FLAG_MOE_GROUPED)
+
+
+def test_moe_many_tokens_default_falls_back_to_grouped(hl, cb):
+    """T = 400 tokens x (8 + 1) slots: the fused path's per-pair partial sums
+    no longer fit in shared memory, so the default call runs the grouped path;
+    its result must equal the one the flag selects, and the oracle's."""
+    err = run_case(hl, cb, E=32, H=256, F=128, T=400, topk=8, shared=True, seed=612)
+    err_g = run_case(hl, cb, E=32, H=256, F=128, T=400, topk=8, shared=True, seed=612,
+                     flags=hl.HLWQ_FLAG_MOE_GROUPED)
+    assert err == err_g   # the same kernels ran
+
+
+def test_moe_ex_rejects_unknown_flags(hl, cb):
+    p = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    args = [hl._ptr(p)] * 4 + [None] * 4 + [hl._ptr(cb), 2, 128, 128, 1, 1, hl._ptr(p), hl._ptr(p), hl._ptr(p),
+                                             hl.HLWQ_F32, None, None, hl._ptr(p), 1 << 20]
+    assert hl.lib.hlwq_moe_gemv_ex(*args, 4, None) == hl.HLWQ_EINVAL
 
 
 def test_moe_ragged_intermediate(hl, cb):
