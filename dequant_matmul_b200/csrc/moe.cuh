@@ -11,8 +11,9 @@
 //   Y[t]   = sum_s p_s * w_hat_dn[ids_s] @ h_s  (+ shared expert with weight 1).
 //
 // Four launches, no atomics, deterministic:
-//   1. router (one CTA): top-k + softmax per token, per-expert assignment lists
-//      sorted by (expert, token), and the rotated activations of every token;
+//   1. router: CTA 0 does top-k + softmax per token and the per-expert
+//      assignment lists sorted by (expert, token); the other CTAs rotate the
+//      activations of every token;
 //   2. gate_up: persistent CTAs over units (active expert, 32 intermediate
 //      columns); each unit decodes its gate and up rows against the tokens
 //      routed to that expert (each expert's codes are read once per call) and
@@ -150,6 +151,24 @@ router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, 
               int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
   __shared__ int s_count[1025];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x > 0) {
+    // CTAs 1.. rotate the tokens' activations (binary16, per-block power-of-
+    // two scale), one 128-block per warp at a time
+    const int nbh = (H + kBlock - 1) / kBlock;
+    const int nwarps = (gridDim.x - 1) * (kRouterThreads / 32);
+    for (int q = (blockIdx.x - 1) * (kRouterThreads / 32) + warp; q < T * nbh; q += nwarps) {
+      const int m = q / nbh, b = q - m * nbh;
+      float e4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = kBlock * b + 4 * lane + k;
+        e4[k] = i < H ? bf16_bits_to_float(__ldg(X + static_cast<int64_t>(m) * H + i)) : 0.0f;
+      }
+      const float inv = rotate_block_store(e4, ws.xt + static_cast<int64_t>(q) * kXsStride);
+      if (lane == 0) ws.xt_inv[q] = inv;
+    }
+    return;
+  }
 
   // 1. top-k + softmax, one warp per token.
   for (int t = warp; t < T; t += kRouterThreads / 32) {
@@ -211,10 +230,6 @@ router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, 
   }
   if (!has_shared)
     for (int t = threadIdx.x; t < T; t += kRouterThreads) ws.tok_asg[t * (topk + 1) + topk] = -1;
-
-  // 3. rotated activations of every token (binary16, per-block power-of-two scale).
-  const int nbh = (H + kBlock - 1) / kBlock;
-  rotate_tokens_bf16(X, H, H, nbh, T, T, ws.xt, ws.xt_inv);
 }
 
 // One pass of up to MT tokens of a gate_up unit: prefetch codes, stage the
@@ -258,8 +273,8 @@ __device__ __forceinline__ void down_pass(const uint8_t* pk, const uint16_t* nm,
   __syncthreads();
 }
 
-__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : 2; }
-constexpr int kMoePass = 2;  // tokens per decode pass of a unit
+__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : (ntok == 2 ? 2 : 4); }
+constexpr int kMoePass = 4;  // tokens per decode pass of a unit
 
 template <int C>
 __global__ void __launch_bounds__(kEngineThreads, 1)
@@ -293,7 +308,8 @@ gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict
       const int ntok = min(kMoePass, ne - m0), mt = pass_mt(ntok);
       auto rowfn = [=](int v) { return static_cast<int64_t>(v < jt ? j0 + v : F + j0 + (v - jt)); };
       if (mt == 1) gate_up_pass<C, 1>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
-      else gate_up_pass<C, 2>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
+      else if (mt == 2) gate_up_pass<C, 2>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
+      else gate_up_pass<C, 4>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
       const int nv = 2 * jt;
       for (int idx = threadIdx.x; idx < ntok * jt; idx += blockDim.x) {
         const int m = idx / jt, j = idx - m * jt;
@@ -341,7 +357,8 @@ down_kernel(const uint8_t* __restrict__ dn_packed, const uint16_t* __restrict__ 
       const float* hbase = ws.h + static_cast<int64_t>(a0 + m0) * F;
       auto rowfn = [=](int v) { return static_cast<int64_t>(r0 + v); };
       if (mt == 1) down_pass<C, 1>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
-      else down_pass<C, 2>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
+      else if (mt == 2) down_pass<C, 2>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
+      else down_pass<C, 4>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
       for (int idx = threadIdx.x; idx < ntok * nr; idx += blockDim.x) {
         const int m = idx / nr, v = idx - m * nr;
         const float* sl = slots + (m * nr + v) * nch;
@@ -388,7 +405,12 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
   MoeWs ws;
   moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
   const bool shared = sh_gu_packed != nullptr;
-  router_kernel<<<1, kRouterThreads, 0, stream>>>(logits, X, E, H, T, topk, shared ? 1 : 0, ids_out, w_out, ws);
+  // CTA 0 routes; the others rotate every token's activation, about one
+  // 128-block per warp
+  const int64_t rot_warps = static_cast<int64_t>(T) * ceil_div(H, kBlock);
+  const int rot_ctas = static_cast<int>(std::min<int64_t>(4 * sm_count(), ceil_div(rot_warps, kRouterThreads / 32)));
+  router_kernel<<<1 + rot_ctas, kRouterThreads, 0, stream>>>(logits, X, E, H, T, topk, shared ? 1 : 0, ids_out,
+                                                              w_out, ws);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
 
   const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
