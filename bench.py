@@ -80,7 +80,7 @@ def load_traffic():
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
 
-    def __init__(self, torch_dev: int, period_s: float = 0.01):
+    def __init__(self, torch_dev: int, period_s: float = 0.001):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
@@ -555,9 +555,13 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="distinct 5120x5120 layers per step (fewer only for small profiling captures; "
+                         "keep their bytes above the L2)")
     ap.add_argument("--only", choices=["components", "quantize", "gemm", "moe", "int4", "kv", "codes", "tq3"], default=None,
                     help="run only the component measurements (used for profiling captures)")
     args = ap.parse_args()
+    nl = max(1, args.layers)
     warmup = max(3, args.warmup)
 
     rank = int(os.environ.get("RANK", "0"))
@@ -597,15 +601,15 @@ def main():
         parts = ("quantize", "gemm", "moe", "int4", "kv", "codes", "tq3") if args.only == "components" else (args.only,)
         print(json.dumps({"components": components(hl, cb, peaks, stream, parts)}), flush=True)
         return
-    # 64 distinct layers (quantized on the device from seeded synthetic weights)
+    # nl (default 64) distinct layers (quantized on the device from seeded synthetic weights)
     layers = []
     with torch.cuda.stream(stream):
-        for l in range(LAYERS):
+        for l in range(nl):
             w = synth.student_t_device((O_DIM, I_DIM), seed=1000 + 7 * rank + l)
             layers.append(hl.quantize(w, cb, stream=stream))
             del w
-        xs = synth.activations_device(LAYERS, I_DIM, seed=2)
-        ys = torch.empty(LAYERS, O_DIM, dtype=torch.float32, device="cuda")
+        xs = synth.activations_device(nl, I_DIM, seed=2)
+        ys = torch.empty(nl, O_DIM, dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
 
     flags = hl.HLWQ_FLAG_WEIGHTS_STATIC   # weights are static across the decode pass
@@ -640,13 +644,13 @@ def main():
         dist.barrier()
     ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
     ms_step = ms_total / args.steps
-    value = whole_job_gbs(world, LAYERS * WEIGHT_BYTES, args.steps, ms_total)
-    launch_ms = ms_step / LAYERS
+    value = whole_job_gbs(world, nl * WEIGHT_BYTES, args.steps, ms_total)
+    launch_ms = ms_step / nl
     achieved = GEMV_ALGO_BYTES / launch_ms / 1e6
 
     # end-to-end through the public API with host buffers (pinned), no graph
     x_host = xs.cpu().pin_memory()
-    y_host = torch.empty(LAYERS, O_DIM, dtype=torch.float32).pin_memory()
+    y_host = torch.empty(nl, O_DIM, dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
@@ -665,7 +669,7 @@ def main():
             e2e_step()
         e2.record(stream)
         e2.synchronize()
-    e2e_val = whole_job_gbs(world, LAYERS * WEIGHT_BYTES, e2e_steps, max_over_ranks(s2.elapsed_time(e2), world, "cuda"))
+    e2e_val = whole_job_gbs(world, nl * WEIGHT_BYTES, e2e_steps, max_over_ranks(s2.elapsed_time(e2), world, "cuda"))
 
     comp = None
     if world == 1 and not args.no_components:
@@ -682,20 +686,20 @@ def main():
             "warmup": warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16*f16->f32", "data": "synthetic",
             "config": {"workload": "dense decode GEMV 5120x5120 HLWQ-Q5 (bf16 Student-t(4) std 0.02 weights, "
-                                   "x bf16 N(0,1)), M=1, 64 distinct layers per step",
-                       "global_batch": 1, "bytes_per_step_per_gpu": LAYERS * WEIGHT_BYTES,
+                                   f"x bf16 N(0,1)), M=1, {nl} distinct layers per step",
+                       "global_batch": 1, "bytes_per_step_per_gpu": nl * WEIGHT_BYTES,
                        "launch": "hlwq_gemv_ex(HLWQ_FLAG_WEIGHTS_STATIC): programmatic dependent launch, "
                                  "x read after the previous kernel completes",
-                       "l2": "inputs larger than L2 (64 layers x 16.8 MB = 1.07 GB)",
+                       "l2": f"inputs larger than L2 ({nl} layers x 16.8 MB = {nl * 16.8e-3:.2f} GB)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": frac(achieved, peaks["hbm_gbs"]), "traffic": traffic,
                          "peak_source": peaks["source"], "algo_bytes_per_launch": GEMV_ALGO_BYTES,
                          "launch_us": round(launch_ms * 1e3, 3)},
             "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": LAYERS * I_DIM * 2,
-                    "d2h_bytes_per_step": LAYERS * O_DIM * 4},
-            "gpu_launches": LAYERS * args.steps,
+            "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": nl * I_DIM * 2,
+                    "d2h_bytes_per_step": nl * O_DIM * 4},
+            "gpu_launches": nl * args.steps,
             "clocks": clk.summary(),
         }
         if comp is not None:
