@@ -376,6 +376,26 @@ def bench_tq3(hl, peaks, stream):
         res[f"gemv_{Og}x{Ig}"] = {"ms": round(ms, 5), "us": round(ms * 1e3, 2), "gbs": round(b / ms / 1e6, 1),
                                   "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"]), "copies": len(copies),
                                   "algo_bytes": b}
+        if Og == O3:
+            # small-M GEMM on the tensor cores (bf16 out), the same weight copies
+            for M in (16, 64):
+                X = synth.activations_device(M, Ig, seed=102 + M)
+                Y = torch.empty(M, Og, dtype=torch.bfloat16, device="cuda")
+                ws = torch.empty(max(1, hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, Og, Ig, M)), dtype=torch.uint8,
+                                 device="cuda")
+
+                def run_gemm():
+                    for p, n in copies:
+                        hl.tq3_gemm(p, n, signs, cb8, X, Y=Y, workspace=ws, stream=stream)
+
+                ms, _ = time_graph(run_gemm, reps=5, warmup=3, stream=stream)
+                ms /= len(copies)
+                b = wbytes + M * Ig * 2 + M * Og * 2
+                tf = 2.0 * M * Og * Ig / ms / 1e9
+                res[f"gemm_{Og}x{Ig}_M{M}"] = {"ms": round(ms, 4), "tflops": round(tf, 2),
+                                               "gbs": round(b / ms / 1e6, 1),
+                                               "tensor_frac": frac(tf, peaks["bf16_tflops"]),
+                                               "hbm_frac": frac(b / ms / 1e6, peaks["hbm_gbs"])}
         del copies
     del w, packed, norms
     return {"tq3": res}

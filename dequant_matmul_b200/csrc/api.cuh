@@ -42,6 +42,11 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
                    size_t ws_bytes, cudaStream_t stream);
 size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M);
 size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M);
+size_t tq3_tc_workspace_bytes(int64_t O, int64_t in, int64_t M);
+size_t tq3_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M);
+int launch_tq3_gemm(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook,
+                    int64_t O, int in, const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16,
+                    void* workspace, size_t ws_bytes, cudaStream_t stream);
 size_t moe_workspace_bytes(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk);
 int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
                const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
@@ -128,6 +133,26 @@ extern "C" int hlwq_tq3_gemv(const uint8_t* packed, const float* norms, const in
       !aligned2(y) || (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(y) & 3u)))
     return HLWQ_EALIGN;
   return hlwq::launch_tq3_gemv(packed, norms, signs, codebook8, out, static_cast<int>(in), x, y, ydtype == HLWQ_BF16,
+                               as_stream(stream));
+}
+
+extern "C" int hlwq_tq3_gemm(const uint8_t* packed, const float* norms, const int8_t* signs,
+                             const float* codebook8, int64_t out, int64_t in, int64_t M, const uint16_t* X,
+                             int64_t ldx, void* Y, int64_t ldy, int ydtype, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!packed || !norms || !signs || !codebook8 || !X || !Y || out <= 0 || in <= 0 || in > kMaxIn ||
+      out > (int64_t(1) << 40) || M <= 0 || M > (1 << 20))
+    return HLWQ_EINVAL;
+  if (ldx < in || ldy < out) return HLWQ_EINVAL;
+  if (ydtype != HLWQ_F32 && ydtype != HLWQ_BF16) return HLWQ_EUNSUPPORTED;
+  if (!aligned16(packed) || (reinterpret_cast<uintptr_t>(norms) & 3u) || !aligned2(X) || !aligned2(Y) ||
+      (ydtype == HLWQ_F32 && (reinterpret_cast<uintptr_t>(Y) & 3u)))
+    return HLWQ_EALIGN;
+  const size_t need = M >= 2 ? hlwq::tq3_tc_workspace_min_bytes(out, in, M) : 0;
+  if (need && (!workspace || ws_bytes < need)) return HLWQ_EWORKSPACE;
+  if (need && !aligned16(workspace)) return HLWQ_EALIGN;
+  return hlwq::launch_tq3_gemm(packed, norms, signs, codebook8, out, static_cast<int>(in), X, ldx,
+                               static_cast<int>(M), Y, ldy, ydtype == HLWQ_BF16, workspace, ws_bytes,
                                as_stream(stream));
 }
 
@@ -312,6 +337,7 @@ extern "C" int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
 extern "C" size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk) {
   if (a <= 0 || b <= 0 || c <= 0) return 0;
   if (op == HLWQ_OP_GEMM) return c >= kTensorCoreMinM ? hlwq::gemm_tc_workspace_bytes(a, b, c) : 0;
+  if (op == HLWQ_OP_TQ3_GEMM) return c >= 2 ? hlwq::tq3_tc_workspace_bytes(a, b, c) : 0;
   if (op == HLWQ_OP_MOE) {
     if (E <= 0 || topk <= 0) return 0;
     return hlwq::moe_workspace_bytes(E, a, b, c, topk);

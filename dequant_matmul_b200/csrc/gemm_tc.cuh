@@ -111,22 +111,46 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n) {
          (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
+// Weight formats the kernel decodes.  HLWQ Q5: 5-bit codes, 80-byte blocks,
+// binary16 norms, 32 centroids.  TQ3 (the scalar case of HIGGS,
+// "Qwen3.6-35B-A3B-TQ3-native", "What TQ3 actually does"): 3-bit codes,
+// 48-byte groups, fp32 shape-gain norms, 8 centroids.  Both are dotted in the
+// rotated domain, sum_b scale_b / 128 * sum_j c[k_bj] x_tilde_bj; only the
+// rotation of x differs (TQ3: x_tilde = s2 * H128 (s1 * x) per group).
+struct TcQ5 {
+  static constexpr int kBits = 5, kLevels = 32, kBytes = 80;
+  using Norm = uint16_t;
+  __device__ static float norm(Norm v) { return half_bits_to_float(v); }
+};
+struct TcTq3 {
+  static constexpr int kBits = 3, kLevels = 8, kBytes = 48;
+  using Norm = float;
+  __device__ static float norm(Norm v) { return v; }
+};
+
+template <int NW>
+__device__ __forceinline__ uint32_t code_word(const uint2 (&c)[NW], int i) {
+  const uint2 u = c[i >> 1];
+  return (i & 1) ? u.y : u.x;
+}
+
 // Shared address of the fp32 centroid of the code at bit POS of a half block
-// (10 words): the 5-bit field moved to bit 2 with one shift, masked and or-ed
-// with the (1024-byte aligned) table address.
+// (NW 8-byte words): the field moved to bit 2 with one shift, masked and
+// or-ed with the (1024-byte aligned) table address.
 // (pos is a compile-time constant after unrolling.)
-__device__ __forceinline__ uint32_t code_addr(const uint2 (&cw)[5], int pos, uint32_t tab) {
+template <class F, int NW>
+__device__ __forceinline__ uint32_t code_addr(const uint2 (&cw)[NW], int pos, uint32_t tab) {
   const int wi = pos >> 5, sh = pos & 31;
-  const uint32_t lo = word10(cw, wi);
+  const uint32_t lo = code_word(cw, wi);
   uint32_t t;
-  if (sh > 27) {
-    t = __funnelshift_r(lo, word10(cw, wi + 1), sh - 2);
+  if (sh + F::kBits > 32) {
+    t = __funnelshift_r(lo, code_word(cw, wi + 1), sh - 2);
   } else if (sh >= 2) {
     t = lo >> (sh - 2);
   } else {
     t = lo << (2 - sh);
   }
-  return (t & 0x7cu) | tab;  // tab is 1024-byte aligned: or == add, one and-or instruction
+  return (t & (4u * (F::kLevels - 1))) | tab;  // tab is 1024-byte aligned: or == add, one and-or instruction
 }
 
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
@@ -148,23 +172,32 @@ __device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
 constexpr int kRotThreads = 256;
 
 // One CTA per token: B[m][:] = binary16(x_tilde[m][:] * s_m), inv_s[m] = 1 / s_m;
-// CTA 0 also clears the GEMM's K-split counters.
+// CTA 0 also clears the GEMM's K-split counters.  x_tilde_b = x_b @ H128, or
+// with signs (TQ3; int8 [2][128], negative = -1): s2 * (H128 (s1 * x_b)).
 __global__ void __launch_bounds__(kRotThreads)
-rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, uint16_t* __restrict__ B,
-                float* __restrict__ inv_s, unsigned* __restrict__ part_cnt, int nsplit) {
+rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, const int8_t* __restrict__ signs,
+                uint16_t* __restrict__ B, float* __restrict__ inv_s, unsigned* __restrict__ part_cnt, int nsplit) {
   extern __shared__ __align__(16) float buf[];  // [nb * 128]
   __shared__ float red[kRotThreads / 32];
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (m == 0)  // the K-split counters of the GEMM that follows start at zero
     for (int i = threadIdx.x; i < nsplit; i += kRotThreads) part_cnt[i] = 0u;
   const uint16_t* x = X + static_cast<int64_t>(m) * ldx;
+  float s1[4] = {1.0f, 1.0f, 1.0f, 1.0f}, s2[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+  if (signs) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      s1[k] = __ldg(signs + 4 * lane + k) < 0 ? -1.0f : 1.0f;
+      s2[k] = __ldg(signs + kBlock + 4 * lane + k) < 0 ? -1.0f : 1.0f;
+    }
+  }
   float mx = 0.0f;
   for (int b = warp; b < nb; b += kRotThreads / 32) {
     float e4[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = kBlock * b + 4 * lane + k;
-      e4[k] = i < in ? bf16_bits_to_float(__ldg(x + i)) : 0.0f;
+      e4[k] = i < in ? bf16_bits_to_float(__ldg(x + i)) * s1[k] : 0.0f;  // sign flips are exact
     }
     float a = e4[0] + e4[1], bb = e4[0] - e4[1], c = e4[2] + e4[3], d = e4[2] - e4[3];
     e4[0] = a + c; e4[1] = bb + d; e4[2] = a - c; e4[3] = bb - d;
@@ -178,7 +211,7 @@ rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, uin
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      buf[kBlock * b + 4 * lane + k] = e4[k];
+      buf[kBlock * b + 4 * lane + k] = e4[k] * s2[k];
       mx = fmaxf(mx, fabsf(e4[k]));
     }
   }
@@ -202,13 +235,13 @@ rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, uin
 // Rings: codes (one 128-row x 80-byte block column per stage, TMA) and A/B
 // stages (one 128-wide K block: A decoded into 64 TMEM columns, B as two
 // 64-wide TMA boxes with 128-byte swizzle); see tc_groups for the mapping.
-constexpr int kTcCodeBytes = kTcTileRows * kBlockBytes;  // 10240
-constexpr int kTcAS = 4;   // A stages in TMEM (64 columns each) after the 256-column accumulator
+template <class F>
+__host__ __device__ constexpr int tc_code_bytes() { return kTcTileRows * F::kBytes; }  // one code stage
 
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcSmemFixed = 1024 /*align slack*/ + 1024 /*centroid table, barriers, misc*/;
-static_assert(4 * kLevels + 8 * (2 * kTcGroups + 4 * kTcGroups + 1) + 8 <= 1024, "barrier block overflows");
-constexpr int kTcMaxNb = 64;  // tile norms in shared memory: 128 x nb binary16 (in <= 8192)
+static_assert(4 * TcQ5::kLevels + 8 * (2 * kTcGroups + 4 * kTcGroups + 1) + 8 <= 1024, "barrier block overflows");
+constexpr int kTcMaxNb = 64;  // tile norms in shared memory: 128 x nb (in <= 8192)
 
 // Decode groups: G groups of 8 warps take blocks b = g (mod G).  Every ring
 // stage belongs to exactly one group, so each stage is consumed in order by a
@@ -219,10 +252,15 @@ __host__ __device__ inline int tc_groups(int n_box) { return n_box > 128 ? 2 : k
 __host__ __device__ inline int tc_cstages(int n_box) { return 2 * tc_groups(n_box); }
 __host__ __device__ inline int tc_stages(int n_box, int) { return tc_groups(n_box); }
 
-__host__ __device__ inline int tc_norm_bytes(int nb) { return (kTcTileRows * nb * 2 + 15) & ~15; }
+template <class F>
+__host__ __device__ inline int tc_norm_bytes(int nb) {
+  return (kTcTileRows * nb * static_cast<int>(sizeof(typename F::Norm)) + 15) & ~15;
+}
 
+template <class F>
 __host__ __device__ inline int tc_smem_bytes(int n_box, int nb) {
-  return kTcSmemFixed + tc_stages(n_box, nb) * n_box * 256 + tc_cstages(n_box) * kTcCodeBytes + tc_norm_bytes(nb);
+  return kTcSmemFixed + tc_stages(n_box, nb) * n_box * 256 + tc_cstages(n_box) * tc_code_bytes<F>() +
+         tc_norm_bytes<F>(nb);
 }
 
 __host__ __device__ inline int tc_ab_stage(int b, int G) { return b % G; }
@@ -230,9 +268,10 @@ __host__ __device__ inline uint32_t tc_ab_parity(int b, int G) { return static_c
 __host__ __device__ inline int tc_code_stage(int b, int G) { return 2 * (b % G) + ((b / G) & 1); }
 __host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static_cast<uint32_t>(b / G / 2) & 1u; }
 
+template <class F>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
-               const uint16_t* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
+               const typename F::Norm* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
                const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box,
                int row_tiles, int nfull, float* __restrict__ part, unsigned* __restrict__ part_cnt) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -243,8 +282,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   const uint32_t tab = base;                 // 32 fp32 centroids
   const uint32_t bst = base + 1024;
   const uint32_t cst = bst + S * n_box * 256;
-  const uint32_t nst = cst + CS * kTcCodeBytes;          // tile norms [128][nb] (binary16)
-  const uint32_t bars = base + 4 * kLevels;              // after the table, inside the first 1 KiB
+  constexpr int kCode = tc_code_bytes<F>();
+  using Norm = typename F::Norm;
+  const uint32_t nst = cst + CS * kCode;                 // tile norms [128][nb]
+  const uint32_t bars = base + 4 * TcQ5::kLevels;        // after the table, inside the first 1 KiB
   // barrier block: full[S] empty[S] c_full[CS] c_empty[CS] accum, then misc
   // (TMEM base, abort flag, split count): at most 128 + 8 (2 S + 2 CS + 1) + 16 = 296 bytes
   const uint32_t full0 = bars, empty0 = full0 + 8 * S, c_full0 = empty0 + 8 * S, c_empty0 = c_full0 + 8 * CS,
@@ -270,10 +311,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
 
   // ---- set-up: codebook, barriers, TMEM
-  if (threadIdx.x < kLevels) {
+  if (threadIdx.x < F::kLevels) {
     const float c = __ldg(codebook + threadIdx.x);
     c32[threadIdx.x] = c;
-    if (threadIdx.x + 1 < kLevels && !(c < __ldg(codebook + threadIdx.x + 1))) raise_device_error(HLWQ_DEVERR_CODEBOOK);
+    if (threadIdx.x + 1 < F::kLevels && !(c < __ldg(codebook + threadIdx.x + 1)))
+      raise_device_error(HLWQ_DEVERR_CODEBOOK);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -297,26 +339,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc_g[0];
-  uint16_t* nrm_s = reinterpret_cast<uint16_t*>(gbase + (nst - base));
+  Norm* nrm_s = reinterpret_cast<Norm*>(gbase + (nst - base));
 
   if (warp < kTcDecWarps) {
     // The tile's norms [128][nb] are one contiguous run of the norm array
     // (rows past O read as zero); they are staged while the producers start
     // on the first code and B boxes, then a barrier of the decode warps only.
     const int64_t nvalid = std::min<int64_t>(kTcTileRows, O - o0) * nb;
-    const uint16_t* nsrc = norms + o0 * nb;
-    const int ntot = kTcTileRows * nb;  // a multiple of 8
+    const Norm* nsrc = norms + o0 * nb;
+    const int ntot = kTcTileRows * nb;                                   // a multiple of 8
+    constexpr int kPer16 = 16 / static_cast<int>(sizeof(Norm));          // norms per 16-byte load
     if ((reinterpret_cast<uintptr_t>(nsrc) & 15u) == 0) {
-      for (int q = threadIdx.x; q < ntot / 8; q += 32 * kTcDecWarps) {
-        if (8 * q + 8 <= nvalid) {
+      for (int q = threadIdx.x; q < ntot / kPer16; q += 32 * kTcDecWarps) {
+        if (kPer16 * q + kPer16 <= nvalid) {
           reinterpret_cast<uint4*>(nrm_s)[q] = __ldg(reinterpret_cast<const uint4*>(nsrc) + q);
         } else {
-          for (int k = 8 * q; k < 8 * q + 8; ++k) nrm_s[k] = k < nvalid ? __ldg(nsrc + k) : static_cast<uint16_t>(0);
+          for (int k = kPer16 * q; k < kPer16 * q + kPer16; ++k) nrm_s[k] = k < nvalid ? __ldg(nsrc + k) : Norm(0);
         }
       }
     } else {
-      for (int q = threadIdx.x; q < ntot; q += 32 * kTcDecWarps)
-        nrm_s[q] = q < nvalid ? __ldg(nsrc + q) : static_cast<uint16_t>(0);
+      for (int q = threadIdx.x; q < ntot; q += 32 * kTcDecWarps) nrm_s[q] = q < nvalid ? __ldg(nsrc + q) : Norm(0);
     }
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcDecWarps) : "memory");
 
@@ -325,9 +367,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // decodes half block hh of rows 32 q4 + lane
     const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod kTcGroups
     const int r = 32 * q4 + lane;
-    const uint16_t* rown = nrm_s + r * nb;
+    const Norm* rown = nrm_s + r * nb;
     float nmax = 0.0f;
-    for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, half_bits_to_float(rown[b]));
+    for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, F::norm(rown[b]));
     int erow = 0;
     if (nmax > 0.0f && isfinite(nmax)) frexpf(nmax, &erow);
     const float rs = ldexpf(1.0f, -erow);
@@ -336,20 +378,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     for (int b = kb0 + dg; b < kb1 && dg < G; b += G) {
       const int lb = b - kb0;
       const int cs = tc_code_stage(lb, G), as = tc_ab_stage(lb, G);
-      const float nsc = half_bits_to_float(rown[b]) * rs;
-      uint2 cw[5];
+      const float nsc = F::norm(rown[b]) * rs;
+      constexpr int NW = F::kBytes / 16;  // 8-byte words of a half block
+      uint2 cw[NW];
       if (ok) ok = mbar_wait(c_full0 + 8 * cs, tc_code_parity(lb, G), deadline);
-      const uint2* src = reinterpret_cast<const uint2*>(codes_g + cs * kTcCodeBytes + r * kBlockBytes + 40 * hh);
+      const uint2* src = reinterpret_cast<const uint2*>(codes_g + cs * kCode + r * F::kBytes + (F::kBytes / 2) * hh);
 #pragma unroll
-      for (int k = 0; k < 5; ++k) cw[k] = src[k];
+      for (int k = 0; k < NW; ++k) cw[k] = src[k];
       __syncwarp();
       if (lane == 0) mbar_arrive(c_empty0 + 8 * cs);
       const float2 sc2 = make_float2(nsc, nsc);
       uint32_t v[32];
 #pragma unroll
       for (int p = 0; p < 32; ++p) {
-        const float2 c = make_float2(__uint_as_float(lds_u32(code_addr(cw, 10 * p, tab))),
-                                     __uint_as_float(lds_u32(code_addr(cw, 10 * p + 5, tab))));
+        const float2 c = make_float2(__uint_as_float(lds_u32(code_addr<F>(cw, 2 * F::kBits * p, tab))),
+                                     __uint_as_float(lds_u32(code_addr<F>(cw, 2 * F::kBits * p + F::kBits, tab))));
         const float2 a = fmul2(c, sc2);
         v[p] = cvt_half2(a.x, a.y);
       }
@@ -382,7 +425,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         misc_g[1] = 1u;
         raise_device_error(HLWQ_DEVERR_TIMEOUT);
       }
-      const float rscale = ldexpf(1.0f, erow) * (1.0f / 128.0f);
+      const float rscale = ldexpf(1.0f, erow - 7);  // 2^erow / 128 (no overflow for fp32 norms)
       constexpr int kCStep = 16 * (kTcDecWarps / 4);
       bool write_tile = true;
       const float* p0 = nullptr;
@@ -481,8 +524,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
         if (fault_skip_tma()) continue;
-        mbar_arrive_expect_tx(c_full0 + 8 * cs, kTcCodeBytes);
-        tma_load_2d(cst + cs * kTcCodeBytes, &cmap, kBlockBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
+        mbar_arrive_expect_tx(c_full0 + 8 * cs, kCode);
+        tma_load_2d(cst + cs * kCode, &cmap, F::kBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
         last = b;
       }
       if (!ok) {
@@ -576,12 +619,13 @@ struct TcPlan {
   size_t inv_off, cnt_off, part_off, base_bytes, split_bytes;
 };
 
-inline TcPlan tc_plan(int64_t O, int64_t in, int64_t M) {
+template <class F>
+TcPlan tc_plan(int64_t O, int64_t in, int64_t M) {
   auto r256 = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
   TcPlan P;
   P.nb = static_cast<int>(ceil_div(in, kBlock));
   int n_box = static_cast<int>(std::min<int64_t>(256, (std::min<int64_t>(M, 256) + 15) / 16 * 16));
-  while (n_box > 16 && tc_smem_bytes(n_box, P.nb) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
+  while (n_box > 16 && tc_smem_bytes<F>(n_box, P.nb) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
   P.n_box = n_box;
   P.row_tiles = static_cast<int>(ceil_div(O, kTcTileRows));
   P.n_tiles = static_cast<int>(ceil_div(M, n_box));
@@ -597,28 +641,39 @@ inline TcPlan tc_plan(int64_t O, int64_t in, int64_t M) {
 }
 
 // Rows longer than kTcMaxNb blocks do not fit the tile-norm staging and run
-// on the CUDA-core path, which needs no workspace.
+// on the CUDA-core kernels, which need no workspace.
 inline bool gemm_tc_takes(int64_t in) { return ceil_div(in, kBlock) <= kTcMaxNb; }
 
-size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
+template <class F>
+size_t tc_workspace_bytes(int64_t O, int64_t in, int64_t M) {
   if (!gemm_tc_takes(in)) return 0;
-  const TcPlan P = tc_plan(O, in, M);
+  const TcPlan P = tc_plan<F>(O, in, M);
   return P.nsplit ? std::max(P.split_bytes, P.base_bytes) : P.base_bytes;
 }
 
-size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
-  return gemm_tc_takes(in) ? tc_plan(O, in, M).base_bytes : 0;
+template <class F>
+size_t tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
+  return gemm_tc_takes(in) ? tc_plan<F>(O, in, M).base_bytes : 0;
 }
 
-int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
-                 const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
+size_t gemm_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) { return tc_workspace_bytes<TcQ5>(O, in, M); }
+size_t gemm_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
+  return tc_workspace_min_bytes<TcQ5>(O, in, M);
+}
+size_t tq3_tc_workspace_bytes(int64_t O, int64_t in, int64_t M) { return tc_workspace_bytes<TcTq3>(O, in, M); }
+size_t tq3_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
+  return tc_workspace_min_bytes<TcTq3>(O, in, M);
+}
 
-int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
-                   const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
-                   size_t ws_bytes, cudaStream_t stream) {
+// Rotation of X into the workspace, then the tensor-core kernel (in <= 8192;
+// the workspace holds at least the plan's base_bytes).  signs: TQ3's sign
+// vectors, or nullptr for Q5.
+template <class F>
+int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float* codebook, const int8_t* signs,
+              int64_t O, int in, const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16,
+              void* workspace, size_t ws_bytes, cudaStream_t stream) {
   const int nb = static_cast<int>(ceil_div(in, kBlock));
-  if (!gemm_tc_takes(in)) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
-  const TcPlan P = tc_plan(O, in, M);
+  const TcPlan P = tc_plan<F>(O, in, M);
   if (ws_bytes < P.base_bytes) return HLWQ_EWORKSPACE;
   const int nsplit = ws_bytes >= P.split_bytes ? P.nsplit : 0;
   char* ws = static_cast<char*>(workspace);
@@ -634,7 +689,7 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
                                     200 * 1024) == cudaSuccess;
       }))
     return st;
-  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, B, inv_s, part_cnt, nsplit);
+  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, signs, B, inv_s, part_cnt, nsplit);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
 
   const int n_box = P.n_box;
@@ -649,28 +704,60 @@ int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* co
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
-  // Codes viewed as a 2-D byte tensor [O][NB * 80]; one box = 128 rows x one 80-byte block.
+  // Codes viewed as a 2-D byte tensor [O][NB * bytes]; one box = 128 rows x
+  // one block (80 or 48 bytes: multiples of 16, as is every box's x offset).
   CUtensorMap cmap;
-  const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(nb) * kBlockBytes, static_cast<cuuint64_t>(O)};
-  const cuuint64_t cstride[1] = {static_cast<cuuint64_t>(nb) * kBlockBytes};
-  const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(kTcTileRows)};
+  const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(nb) * F::kBytes, static_cast<cuuint64_t>(O)};
+  const cuuint64_t cstride[1] = {static_cast<cuuint64_t>(nb) * F::kBytes};
+  const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(F::kBytes), static_cast<cuuint32_t>(kTcTileRows)};
+  static_assert(F::kBytes % 16 == 0, "code boxes start on 16-byte boundaries");
   if (encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), cdim, cstride, cbox, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
-  const int smem = tc_smem_bytes(n_box, nb);
+  const int smem = tc_smem_bytes<F>(n_box, nb);
   static PerDeviceOnce attr;
   if (const int st = attr([&] {
-        return cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        return cudaFuncSetAttribute(gemm_tc_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     227 * 1024) == cudaSuccess;
       }))
     return st;
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const int nfull = P.row_tiles * P.n_tiles - nsplit;
-  gemm_tc_kernel<<<nfull + 2 * nsplit, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
-                                                                   ldy, out_bf16 ? 1 : 0, n_box, P.row_tiles, nfull,
-                                                                   part, part_cnt);
+  gemm_tc_kernel<F><<<nfull + 2 * nsplit, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s,
+                                                                      Y, ldy, out_bf16 ? 1 : 0, n_box, P.row_tiles,
+                                                                      nfull, part, part_cnt);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+}
+
+int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                 const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, cudaStream_t stream);
+
+int launch_gemm_tc(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,
+                   const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16, void* workspace,
+                   size_t ws_bytes, cudaStream_t stream) {
+  if (!gemm_tc_takes(in)) return launch_dense(packed, norms, codebook, O, in, X, ldx, M, Y, ldy, out_bf16, stream);
+  return launch_tc<TcQ5>(packed, norms, codebook, nullptr, O, in, X, ldx, M, Y, ldy, out_bf16, workspace, ws_bytes,
+                         stream);
+}
+
+int launch_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook,
+                    int64_t O, int in, const uint16_t* x, void* y, bool out_bf16, cudaStream_t stream);
+
+// TQ3 for M tokens: the tensor-core kernel when M >= 2 and in <= 8192,
+// otherwise one TQ3 GEMV launch per token (no workspace).
+int launch_tq3_gemm(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook,
+                    int64_t O, int in, const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16,
+                    void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (M >= 2 && gemm_tc_takes(in))
+    return launch_tc<TcTq3>(packed, norms, codebook, signs, O, in, X, ldx, M, Y, ldy, out_bf16, workspace, ws_bytes,
+                            stream);
+  const int es = out_bf16 ? 2 : 4;
+  for (int m = 0; m < M; ++m)
+    if (const int st = launch_tq3_gemv(packed, norms, signs, codebook, O, in, X + static_cast<int64_t>(m) * ldx,
+                                       static_cast<char*>(Y) + static_cast<int64_t>(m) * ldy * es, out_bf16, stream))
+      return st;
+  return HLWQ_OK;
 }
 
 }  // namespace hlwq

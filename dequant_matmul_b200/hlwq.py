@@ -20,7 +20,7 @@ HLWQ_OK, HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_ECUDA, HLWQ_EWORKSPAC
 HLWQ_ESCRATCH = -6
 NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 + 64 * 1024
 HLWQ_F32, HLWQ_BF16, HLWQ_F16 = 0, 1, 2
-HLWQ_OP_GEMM, HLWQ_OP_MOE = 1, 2
+HLWQ_OP_GEMM, HLWQ_OP_MOE, HLWQ_OP_TQ3_GEMM = 1, 2, 3
 HLWQ_FLAG_WEIGHTS_STATIC = 1
 HLWQ_FLAG_MOE_GROUPED = 2
 DEVERR_CODEBOOK, DEVERR_TIMEOUT, DEVERR_CODE_RANGE = 0x1, 0x2, 0x4
@@ -37,6 +37,7 @@ SIGNATURES = {
     "hlwq_tq3_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "hlwq_tq3_dequantize": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _I, _P]),
     "hlwq_tq3_gemv": (_I, [_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P]),
+    "hlwq_tq3_gemm": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "hlwq_requantize_int4": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_quantize": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "hlwq_kv_dequantize": (_I, [_P, _P, _P, _I64, _P, _I, _P]),
@@ -252,6 +253,24 @@ def tq3_gemv(packed, norms, signs, cb8, x: torch.Tensor, out_dtype=torch.float32
     _check(lib.hlwq_tq3_gemv(_ptr(packed), _ptr(norms), _ptr(signs), _ptr(cb8), out_f, x.shape[-1], _ptr(x), _ptr(y),
                              _dtype_code(y.dtype), _stream(stream)), "hlwq_tq3_gemv")
     return y
+
+
+def tq3_gemm(packed, norms, signs, cb8, X: torch.Tensor, out_dtype=torch.float32, Y=None, workspace=None,
+             stream=None):
+    """X bf16 [M][in] (row pitch X.stride(0)) -> Y [M][out] = X @ W_hat^T."""
+    _cuda(X, "X")
+    out_f = packed.shape[0]
+    M, in_f = X.shape
+    if Y is None:
+        Y = torch.empty(M, out_f, dtype=out_dtype, device=X.device)
+    need = workspace_bytes(HLWQ_OP_TQ3_GEMM, out_f, in_f, M)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.hlwq_tq3_gemm(_ptr(packed), _ptr(norms), _ptr(signs), _ptr(cb8), out_f, in_f, M, _ptr(X), X.stride(0),
+                             _ptr(Y), Y.stride(0), _dtype_code(Y.dtype), _ptr(workspace), ws_bytes, _stream(stream)),
+           "hlwq_tq3_gemm")
+    return Y
 
 
 def requantize_int4(packed, norms, cb, in_features: int, q4=None, scale=None, zero=None, stream=None):

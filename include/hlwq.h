@@ -67,7 +67,7 @@ typedef enum {
 typedef enum { HLWQ_F32 = 0, HLWQ_BF16 = 1, HLWQ_F16 = 2 } hlwq_dtype;
 
 /* Operations whose scratch size hlwq_workspace_bytes() reports. */
-typedef enum { HLWQ_OP_GEMM = 1, HLWQ_OP_MOE = 2 } hlwq_op;
+typedef enum { HLWQ_OP_GEMM = 1, HLWQ_OP_MOE = 2, HLWQ_OP_TQ3_GEMM = 3 } hlwq_op;
 
 /* Launch flags of the *_ex calls. */
 typedef enum { HLWQ_FLAG_WEIGHTS_STATIC = 1, HLWQ_FLAG_MOE_GROUPED = 2 } hlwq_flags;
@@ -234,6 +234,30 @@ int hlwq_tq3_gemv(const uint8_t* packed, const float* norms, const int8_t* signs
                   int64_t out, int64_t in, const uint16_t* x, void* y, int ydtype, void* stream);
 
 /*
+ * TQ3 small-M GEMM (the same weights as hlwq_tq3_gemv, "a second encoding on
+ * the same kernels"): Y[m][o] = sum_i X[m][i] w_hat[o][i], fp32 accumulation,
+ * evaluated in the rotated domain, sum over groups b of gamma_b / 128 *
+ * sum_j c[code_bj] xt_bj with xt_b = s2 * (H128 (s1 * x_b)).
+ *   X  device bf16 [M][in], row pitch ldx >= in elements
+ *   Y  device ydtype [M][out] (HLWQ_F32 or HLWQ_BF16), row pitch ldy >= out
+ *   packed must be 16-byte aligned (its 48-byte groups are tensor-memory-
+ *   access boxes); norms 4-byte; X, Y as hlwq_gemm.
+ *   workspace  device, 16-byte aligned, ws_bytes >=
+ *              hlwq_workspace_bytes(HLWQ_OP_TQ3_GEMM, out, in, M, 1, 0) when
+ *              that is non-zero (a smaller workspace of at least the
+ *              tensor-core path's minimum runs without its K split)
+ * Paths: M >= 2 and in <= 8192 run the tcgen05 tensor-core kernel of
+ * hlwq_gemm with the TQ3 decode (3-bit codes, fp32 gammas, 8 centroids, the
+ * sign-vector rotation of X); M = 1, and rows longer than 8192, run the TQ3
+ * GEMV once per token and need no workspace.
+ * Errors: HLWQ_EINVAL, HLWQ_EALIGN, HLWQ_EUNSUPPORTED, HLWQ_EWORKSPACE,
+ * HLWQ_ECUDA.
+ */
+int hlwq_tq3_gemm(const uint8_t* packed, const float* norms, const int8_t* signs, const float* codebook8,
+                  int64_t out, int64_t in, int64_t M, const uint16_t* X, int64_t ldx, void* Y, int64_t ldy,
+                  int ydtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Decode GEMV: y[o] = sum_i x[i] * w_hat[o][i], fp32 accumulation, without
  * materialising w_hat (the activation is rotated once per 128-block and dotted
  * with centroid values in the rotated domain).
@@ -323,6 +347,7 @@ int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_norms,
  * Scratch bytes for an operation (0 when none is needed).
  *   HLWQ_OP_GEMM: a = out, b = in, c = M
  *   HLWQ_OP_MOE : a = H,   b = F,  c = T, E = experts, topk
+ *   HLWQ_OP_TQ3_GEMM: a = out, b = in, c = M
  */
 size_t hlwq_workspace_bytes(int op, int64_t a, int64_t b, int64_t c, int64_t E, int64_t topk);
 

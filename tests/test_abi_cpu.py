@@ -109,6 +109,37 @@ def test_gemm_workspace_only_on_the_tensor_core_path(hl):
     assert hl.workspace_bytes(hl.HLWQ_OP_GEMM, 256, 8192, 4) == 0
 
 
+def test_tq3_gemm_validation_and_workspace(hl):
+    L = hl.lib
+    p = ctypes.c_void_p(256)        # fake, 16-byte aligned, never dereferenced
+    p8 = ctypes.c_void_p(264)       # 8-byte aligned only
+    p2 = ctypes.c_void_p(258)       # 2-byte aligned only
+
+    def call(packed=p, norms=p, signs=p, cb=p, out=256, in_f=512, M=16, X=p, ldx=512, Y=p, ldy=256,
+             dt=hl.HLWQ_F32, ws=None, ws_bytes=0):
+        return L.hlwq_tq3_gemm(packed, norms, signs, cb, out, in_f, M, X, ldx, Y, ldy, dt, ws, ws_bytes, None)
+
+    assert call(packed=None) == hl.HLWQ_EINVAL
+    assert call(signs=None) == hl.HLWQ_EINVAL
+    assert call(M=0) == hl.HLWQ_EINVAL
+    assert call(ldx=511) == hl.HLWQ_EINVAL
+    assert call(ldy=255) == hl.HLWQ_EINVAL
+    assert call(in_f=(1 << 20) + 1, ldx=(1 << 20) + 1) == hl.HLWQ_EINVAL
+    assert call(dt=hl.HLWQ_F16) == hl.HLWQ_EUNSUPPORTED
+    assert call(packed=p8) == hl.HLWQ_EALIGN          # 48-byte groups are copied by TMA boxes
+    assert call(norms=p2) == hl.HLWQ_EALIGN
+    assert call(Y=p2) == hl.HLWQ_EALIGN               # fp32 output
+    assert call() == hl.HLWQ_EWORKSPACE               # M >= 2: the tensor-core path needs its workspace
+    need = hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, 256, 512, 16)
+    assert need > 0
+    assert call(ws=p, ws_bytes=need - 1) == hl.HLWQ_EWORKSPACE   # two row tiles: no K split, need = minimum
+    assert call(ws=p8, ws_bytes=need) == hl.HLWQ_EALIGN
+    # no workspace for one token or for rows longer than 8192 (the GEMV per token)
+    assert hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, 256, 512, 1) == 0
+    assert hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, 256, 8193, 64) == 0
+    assert hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, 256, 8192, 2) > 0
+
+
 def test_noalloc_validates_arguments_before_sizing_its_scratch(hl):
     L = hl.lib
     p = ctypes.c_void_p(256)

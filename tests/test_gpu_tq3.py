@@ -149,3 +149,96 @@ def test_tq3_bad_codebook_sets_the_error_bit(hl, signs):
     p, n = hl.tq3_quantize(W, signs.cuda(), bad)
     hl.tq3_gemv(p, n, signs.cuda(), bad, synth.activations(1, 256, seed=2)[0].cuda())
     assert hl.device_error() & hl.DEVERR_CODEBOOK
+
+
+# TQ3 small-M GEMM: the tensor-core kernel from M = 2 (in <= 8192), the GEMV
+# once per token for M = 1 and for longer rows.
+TQ3_GEMM_CASES = [
+    (256, 512, 2),      # two tokens, one 16-token tile
+    (300, 704, 5),      # ragged rows (300 = 2 x 128 + 44) and inputs (704 = 5.5 groups)
+    (129, 300, 37),     # one row past a tile, 3 groups with a zero-padded tail, tokens past a 16-multiple
+    (1000, 2048, 16),
+    (512, 5120, 64),
+    (200, 8192, 300),   # the longest rows the tensor-core path takes; two token tiles of 256
+    (64, 9316, 3),      # rows longer than 8192: one GEMV per token
+    (96, 640, 1),       # M = 1: the GEMV
+]
+
+
+@pytest.mark.parametrize("O_,I_,M", TQ3_GEMM_CASES)
+def test_tq3_gemm(hl, cb8, signs, O_, I_, M):
+    W = synth.student_t((O_, I_), df4_seed=5 * O_ + I_ + M)
+    p, n, want = _quant(hl, cb8, signs, W)
+    X = synth.activations(M, I_, seed=O_ + M)
+    s = signs.numpy()
+    ref = T.tq3_matmul(want["packed"], want["norms"], I_, s[0], s[1], X)
+    Y = hl.tq3_gemm(p, n, signs.cuda(), cb8, X.cuda())
+    Yb = hl.tq3_gemm(p, n, signs.cuda(), cb8, X.cuda(), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    e = rel(Y.cpu().numpy(), ref)
+    assert e <= 2e-3, e
+    assert rel(Yb.double().cpu().numpy(), ref) <= 4e-3
+    assert hl.device_error() == 0
+
+
+def test_tq3_gemm_strided_operands(hl, cb8, signs):
+    """X and Y inside wider buffers (ldx > in, ldy > out): the columns past
+    out are left untouched."""
+    O_, I_, M = 384, 1000, 24
+    W = synth.student_t((O_, I_), df4_seed=9)
+    p, n, want = _quant(hl, cb8, signs, W)
+    Xw = torch.zeros(M, I_ + 24, dtype=torch.bfloat16)
+    Xw[:, :I_] = synth.activations(M, I_, seed=10)
+    Yw = torch.full((M, O_ + 8), 7.0, dtype=torch.float32, device="cuda")
+    hl.tq3_gemm(p, n, signs.cuda(), cb8, Xw.cuda()[:, :I_], Y=Yw[:, :O_])
+    torch.cuda.synchronize()
+    s = signs.numpy()
+    ref = T.tq3_matmul(want["packed"], want["norms"], I_, s[0], s[1], Xw[:, :I_])
+    assert rel(Yw[:, :O_].cpu().numpy(), ref) <= 2e-3
+    assert torch.all(Yw[:, O_:] == 7.0)
+
+
+def test_tq3_gemm_k_split_and_minimum_workspace(hl, cb8, signs):
+    """160 row tiles on 148 SMs: the last 12 tiles are split in K (full
+    workspace); with only the minimum workspace nothing is split.  Both match
+    the oracle on sampled rows."""
+    O_, I_, M = 160 * 128, 1000, 24
+    W = synth.student_t_device((O_, I_), seed=91)
+    p, n = hl.tq3_quantize(W, signs.cuda(), cb8)
+    X = synth.activations(M, I_, seed=92)
+    Xd = X.cuda()
+    Y = hl.tq3_gemm(p, n, signs.cuda(), cb8, Xd)
+    ws_min = (M * 8 * 128 * 2 + 255) // 256 * 256 + M * 4 + 256
+    assert hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, O_, I_, M) > ws_min
+    Y2 = hl.tq3_gemm(p, n, signs.cuda(), cb8, Xd, workspace=torch.empty(ws_min, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(O_ - 12 * 128 - 8, O_ - 12 * 128 + 8),
+                                     np.arange(O_ - 64, O_), np.random.default_rng(93).integers(0, O_, 64)]))
+    ri = torch.from_numpy(rows).cuda()
+    s = signs.numpy()
+    ref = T.tq3_matmul(p[ri].cpu().numpy(), n[ri].cpu().numpy(), I_, s[0], s[1], X)
+    assert rel(Y.cpu().numpy()[:, rows], ref) <= 2e-3
+    assert rel(Y2.cpu().numpy()[:, rows], ref) <= 2e-3
+
+
+def test_tq3_gemm_full_size_sampled(hl, cb8, signs):
+    """27648 x 5120 at M = 64 (216 row tiles: 148 whole tiles and 68 split in
+    K over the second wave) and M = 16; outputs of sampled rows against the
+    oracle's matmul of the GPU's own codes (those codes are pinned bit-exact
+    by test_tq3_full_size_sampled)."""
+    O_, I_ = 27648, 5120
+    W = synth.student_t_device((O_, I_), seed=81)
+    p, n = hl.tq3_quantize(W, signs.cuda(), cb8)
+    del W
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, O_ - 129, O_ - 1],
+                                     np.random.default_rng(82).integers(0, O_, 58)]))
+    ri = torch.from_numpy(rows).cuda()
+    ps, ns = p[ri].cpu().numpy(), n[ri].cpu().numpy()
+    s = signs.numpy()
+    for M in (16, 64):
+        X = synth.activations(M, I_, seed=83 + M)
+        Y = hl.tq3_gemm(p, n, signs.cuda(), cb8, X.cuda())
+        torch.cuda.synchronize()
+        ref = T.tq3_matmul(ps, ns, I_, s[0], s[1], X)
+        assert rel(Y.cpu().numpy()[:, rows], ref) <= 2e-3
+    assert hl.device_error() == 0
