@@ -258,11 +258,12 @@ def tq3_gemv(packed, norms, signs, cb8, x: torch.Tensor, out_dtype=torch.float32
 def tq3_gemm(packed, norms, signs, cb8, X: torch.Tensor, out_dtype=torch.float32, Y=None, workspace=None,
              stream=None):
     """X bf16 [M][in] (row pitch X.stride(0)) -> Y [M][out] = X @ W_hat^T."""
-    _cuda(X, "X")
+    _cuda_rows(X, "X")
     out_f = packed.shape[0]
     M, in_f = X.shape
     if Y is None:
         Y = torch.empty(M, out_f, dtype=out_dtype, device=X.device)
+    _cuda_rows(Y, "Y")
     need = workspace_bytes(HLWQ_OP_TQ3_GEMM, out_f, in_f, M)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
