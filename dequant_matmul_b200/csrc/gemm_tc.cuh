@@ -12,22 +12,28 @@
 //
 // Kernel 1 (rotate_x_kernel): one CTA per token rotates X once per call into
 // the workspace (binary16 B matrix, K-major) and records 1/s_m.
-// Kernel 2 (gemm_tc_kernel): one CTA per 128-row tile of W (and up to 256-token
-// tile of X).  Roles, 864 threads:
-//   warps 0-23 decode, in G groups of 8 (G = 3, or 2 for 256-token tiles)
-//              taking blocks b = g (mod G): each lane owns one weight row of
-//              the tile and decodes one half block (code -> fp32 centroid from
-//              a shared table, times the block scale, rounded to binary16) and
-//              writes it straight into tensor memory with tcgen05.st (the A
-//              operand lives in TMEM, so decoding costs no shared-memory
-//              bandwidth that the MMA needs for B);
-//   warp 24    TMA producer of the code tiles (128 rows x 80 bytes per block);
-//   warp 26    TMA producer of B: two 64 x N boxes per block, 128-byte swizzled
-//              (no multicast);
-//   warp 25    allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
+// Kernel 2 (gemm_tc_kernel<F, NG>): one CTA per 128-row tile of W (and up to
+// 256-token tile of X).  Roles, D = 8 NG decode warps plus three:
+//   warps 0..D-1 decode, in NG groups of 8 taking blocks b = g (mod NG): each
+//              lane owns one weight row of the tile and decodes one half block
+//              (code -> fp32 centroid from a shared table, times the block
+//              scale, rounded to binary16) and writes it straight into tensor
+//              memory with tcgen05.st (the A operand lives in TMEM, so
+//              decoding costs no shared-memory bandwidth that the MMA needs
+//              for B);
+//   warp D     TMA producer of the code tiles (128 rows x 80 bytes per block);
+//   warp D + 2 TMA producer of B: two 64 x N boxes per block, 128-byte
+//              swizzled (no multicast);
+//   warp D + 1 allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
 //              N = tokens, K = 16) into an fp32 accumulator in TMEM;
-//   warps 0-23 epilogue (six per TMEM lane quarter, split by columns):
+//   warps 0..D-1 epilogue (split by TMEM lane quarter and columns):
 //              tcgen05.ld of the accumulator, scaling, bf16/fp32 store.
+// The single MMA-issuing thread paces a CTA: a tcgen05.mma takes about as
+// long to issue as a 64-token MMA takes to run, and the decode warps on its
+// scheduler slow it further.  Token tiles of at most 128 therefore run with
+// one decode group (NG = 1, 352 threads, 256 TMEM columns) and two CTAs per
+// SM, so that two threads issue MMAs on every SM; 256-token tiles, whose MMAs
+// are long, use two groups (NG = 2) and the whole TMEM of the SM.
 // Stages are handed over with mbarriers; every wait is bounded (2 s), after
 // which the kernel raises HLWQ_DEVERR_TIMEOUT, drains and frees TMEM.
 
@@ -38,14 +44,16 @@ namespace hlwq {
 
 namespace {
 
-constexpr int kTcGroups = 3;                       // decode groups (8 warps each) on alternate blocks
-constexpr int kTcDecWarps = 8 * kTcGroups;
-constexpr int kTcWCodes = kTcDecWarps, kTcWMma = kTcDecWarps + 1, kTcWB = kTcDecWarps + 2;
-constexpr int kTcThreads = 32 * (kTcDecWarps + 3);
+// Warp roles of a CTA with NG decode groups of 8 warps.
+template <int NG>
+struct TcRoles {
+  static constexpr int kDecWarps = 8 * NG;
+  static constexpr int kWCodes = kDecWarps, kWMma = kDecWarps + 1, kWB = kDecWarps + 2;
+  static constexpr int kThreads = 32 * (kDecWarps + 3);
+};
 constexpr int kTcTileRows = 128;
-constexpr int kTcKChunk = 64;                 // K elements per pipeline stage (one half block)
-constexpr int kTcAccCols = 256;               // TMEM columns reserved for the accumulator
-constexpr int kTcAllocCols = 512;   // accumulator (256) + 3 A stages of 64
+constexpr int kTcKChunk = 64;  // K elements per B box (one half block)
+constexpr int kTcStages = 2;   // A/B stages (A: 64 TMEM columns each, after the accumulator)
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -240,17 +248,22 @@ __host__ __device__ constexpr int tc_code_bytes() { return kTcTileRows * F::kByt
 
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcSmemFixed = 1024 /*align slack*/ + 1024 /*centroid table, barriers, misc*/;
-static_assert(4 * TcQ5::kLevels + 8 * (2 * kTcGroups + 4 * kTcGroups + 1) + 8 <= 1024, "barrier block overflows");
+static_assert(4 * TcQ5::kLevels + 8 * (2 * kTcStages + 2 * 4 + 1) + 16 <= 1024, "barrier block overflows");
 constexpr int kTcMaxNb = 64;  // tile norms in shared memory: 128 x nb (in <= 8192)
 
 // Decode groups: G groups of 8 warps take blocks b = g (mod G).  Every ring
 // stage belongs to exactly one group, so each stage is consumed in order by a
 // single consumer and mbarrier parity waits are never ambiguous:
-//   A/B stage of block b   = b mod G               (one per group; A in TMEM, B in smem)
+//   A/B stage of block b   = b mod S (S = 2 stages: one per group when G = 2,
+//                            both of the one group when G = 1)
 //   code stage of block b  = 2 (b mod G) + (b / G) mod 2   (two per group)
-__host__ __device__ inline int tc_groups(int n_box) { return n_box > 128 ? 2 : kTcGroups; }
+// TMEM: the accumulator (128 columns for token tiles <= 128, else 256), then
+// the S A stages; 256 or 512 columns allocated.
+__host__ __device__ inline int tc_groups(int n_box) { return n_box > 128 ? 2 : 1; }
 __host__ __device__ inline int tc_cstages(int n_box) { return 2 * tc_groups(n_box); }
-__host__ __device__ inline int tc_stages(int n_box, int) { return tc_groups(n_box); }
+__host__ __device__ inline int tc_stages(int, int) { return kTcStages; }
+__host__ __device__ inline uint32_t tc_acc_cols(int n_box) { return n_box > 128 ? 256u : 128u; }
+__host__ __device__ inline uint32_t tc_alloc_cols(int n_box) { return n_box > 128 ? 512u : 256u; }
 
 template <class F>
 __host__ __device__ inline int tc_norm_bytes(int nb) {
@@ -263,13 +276,13 @@ __host__ __device__ inline int tc_smem_bytes(int n_box, int nb) {
          tc_norm_bytes<F>(nb);
 }
 
-__host__ __device__ inline int tc_ab_stage(int b, int G) { return b % G; }
-__host__ __device__ inline uint32_t tc_ab_parity(int b, int G) { return static_cast<uint32_t>(b / G) & 1u; }
+__host__ __device__ inline int tc_ab_stage(int b, int S) { return b % S; }
+__host__ __device__ inline uint32_t tc_ab_parity(int b, int S) { return static_cast<uint32_t>(b / S) & 1u; }
 __host__ __device__ inline int tc_code_stage(int b, int G) { return 2 * (b % G) + ((b / G) & 1); }
 __host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static_cast<uint32_t>(b / G / 2) & 1u; }
 
-template <class F>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <class F, int NG>
+__global__ void __launch_bounds__(TcRoles<NG>::kThreads, NG == 1 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
                const typename F::Norm* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
                const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box,
@@ -278,7 +291,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const int G = tc_groups(n_box), S = tc_stages(n_box, nb), CS = tc_cstages(n_box);
+  constexpr int kTcDecWarps = TcRoles<NG>::kDecWarps, kTcWCodes = TcRoles<NG>::kWCodes, kTcWMma = TcRoles<NG>::kWMma,
+                kTcWB = TcRoles<NG>::kWB;
+  constexpr int G = NG, S = kTcStages, CS = 2 * NG;
+  const uint32_t acc_cols = tc_acc_cols(n_box), alloc_cols = tc_alloc_cols(n_box);
   const uint32_t tab = base;                 // 32 fp32 centroids
   const uint32_t bst = base + 1024;
   const uint32_t cst = bst + S * n_box * 256;
@@ -331,7 +347,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kTcWMma) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(misc), "r"(kTcAllocCols)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(misc), "r"(alloc_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -365,7 +381,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // ---------------------------------------------------------- decode
     // two groups of 8 warps take alternate blocks; in a group, warp (q4, hh)
     // decodes half block hh of rows 32 q4 + lane
-    const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod kTcGroups
+    const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod G
     const int r = 32 * q4 + lane;
     const Norm* rown = nrm_s + r * nb;
     float nmax = 0.0f;
@@ -377,7 +393,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     bool ok = true;
     for (int b = kb0 + dg; b < kb1 && dg < G; b += G) {
       const int lb = b - kb0;
-      const int cs = tc_code_stage(lb, G), as = tc_ab_stage(lb, G);
+      const int cs = tc_code_stage(lb, G), as = tc_ab_stage(lb, S);
       const float nsc = F::norm(rown[b]) * rs;
       constexpr int NW = F::kBytes / 16;  // 8-byte words of a half block
       uint2 cw[NW];
@@ -396,9 +412,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const float2 a = fmul2(c, sc2);
         v[p] = cvt_half2(a.x, a.y);
       }
-      if (ok) ok = mbar_wait(empty0 + 8 * as, tc_ab_parity(lb, G) ^ 1u, deadline);
+      if (ok) ok = mbar_wait(empty0 + 8 * as, tc_ab_parity(lb, S) ^ 1u, deadline);
       if (ok && misc_g[1] == 0u) {
-        const uint32_t ta = tm_row + kTcAccCols + 64 * as + 32 * hh;
+        const uint32_t ta = tm_row + acc_cols + 64 * as + 32 * hh;
         uint32_t v0[16], v1[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) { v0[k] = v[k]; v1[k] = v[16 + k]; }
@@ -545,8 +561,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
       bool ok = true;
       int last = -1;  // last block whose copies were issued
       for (int b = kb0; b < kb1; ++b) {
-        const int st = tc_ab_stage(b - kb0, G);
-        ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
+        const int st = tc_ab_stage(b - kb0, S);
+        ok = mbar_wait(empty0 + 8 * st, tc_ab_parity(b - kb0, S) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
         if (fault_skip_tma()) continue;
         mbar_arrive_expect_tx(full0 + 8 * st, 2 * half_bytes);
@@ -563,17 +579,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
       // decode warps arrive on every stage they take, so a stage's phase
       // completes once its bytes have landed)
       const uint64_t dl = globaltimer_ns() + wait_limit_ns();
-      for (int b = std::max(kb0, last - G + 1); b <= last; ++b)
-        mbar_wait(full0 + 8 * tc_ab_stage(b - kb0, G), tc_ab_parity(b - kb0, G), dl);
+      for (int b = std::max(kb0, last - S + 1); b <= last; ++b)
+        mbar_wait(full0 + 8 * tc_ab_stage(b - kb0, S), tc_ab_parity(b - kb0, S), dl);
     }
   } else if (warp == kTcWMma) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(n_box);
       bool ok = true;
-      for (int b = kb0; b < kb1; ++b) {
-        const int st = tc_ab_stage(b - kb0, G);
-        ok = mbar_wait(full0 + 8 * st, tc_ab_parity(b - kb0, G), deadline) && misc_g[1] == 0u;
+      // The MMA thread paces the whole CTA (one tcgen05.mma costs about as
+      // much to issue as a 64-token MMA takes to run), so its loop carries
+      // the stage and parity instead of dividing by G, and does not poll the
+      // abort flag: when another role gives up, this thread's own bounded
+      // wait on the stage it needs runs out.
+      int st = 0;
+      uint32_t par = 0u;
+      for (int b = kb0; b < kb1; ++b, st = (st + 1 == S) ? 0 : st + 1, par ^= (st == 0) ? 1u : 0u) {
+        ok = mbar_wait(full0 + 8 * st, par, deadline);
         if (!ok) break;
         tc_fence_after();
         const uint32_t bstage = bst + st * n_box * 256;
@@ -582,7 +604,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
           const uint64_t bdesc = smem_desc_sw128(bstage + h * n_box * 128);
 #pragma unroll
           for (int kk = 0; kk < kTcKChunk / 16; ++kk)
-            tc_mma_f16(tmem, tmem + kTcAccCols + 64 * st + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk),
+            tc_mma_f16(tmem, tmem + acc_cols + 64 * st + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk),
                        idesc, (b > kb0 || h > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(empty0 + 8 * st);  // frees both the A stage (TMEM) and the B stage (shared memory)
@@ -601,7 +623,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   __syncthreads();
   if (warp == kTcWMma) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcAllocCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(alloc_cols) : "memory");
   }
 }
 
@@ -718,15 +740,23 @@ int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float*
   const int smem = tc_smem_bytes<F>(n_box, nb);
   static PerDeviceOnce attr;
   if (const int st = attr([&] {
-        return cudaFuncSetAttribute(gemm_tc_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        return cudaFuncSetAttribute(gemm_tc_kernel<F, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    227 * 1024) == cudaSuccess &&
+               cudaFuncSetAttribute(gemm_tc_kernel<F, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     227 * 1024) == cudaSuccess;
       }))
     return st;
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const int nfull = P.row_tiles * P.n_tiles - nsplit;
-  gemm_tc_kernel<F><<<nfull + 2 * nsplit, kTcThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s,
-                                                                      Y, ldy, out_bf16 ? 1 : 0, n_box, P.row_tiles,
-                                                                      nfull, part, part_cnt);
+  const int grid = nfull + 2 * nsplit, ob = out_bf16 ? 1 : 0;
+  if (tc_groups(n_box) == 1)
+    gemm_tc_kernel<F, 1><<<grid, TcRoles<1>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
+                                                                       ldy, ob, n_box, P.row_tiles, nfull, part,
+                                                                       part_cnt);
+  else
+    gemm_tc_kernel<F, 2><<<grid, TcRoles<2>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
+                                                                       ldy, ob, n_box, P.row_tiles, nfull, part,
+                                                                       part_cnt);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
 
