@@ -179,18 +179,21 @@ __device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
 // ---------------------------------------------------------------- rotation
 constexpr int kRotThreads = 256;
 
-// One CTA per token: B[m][:] = binary16(x_tilde[m][:] * s_m), inv_s[m] = 1 / s_m;
-// CTA 0 also clears the GEMM's K-split counters.  x_tilde_b = x_b @ H128, or
-// with signs (TQ3; int8 [2][128], negative = -1): s2 * (H128 (s1 * x_b)).
+// One CTA per B row m: B[m][:] = binary16(x_tilde[m][:] * s_m), inv_s[m] = 1 / s_m,
+// for the activation row rows[m] (rows == nullptr: row m; the MoE layer's
+// gather of each assignment's token); CTA 0 also clears the GEMM's K-split
+// counters.  x_tilde_b = x_b @ H128, or with signs (TQ3; int8 [2][128],
+// negative = -1): s2 * (H128 (s1 * x_b)).
 __global__ void __launch_bounds__(kRotThreads)
 rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, const int8_t* __restrict__ signs,
-                uint16_t* __restrict__ B, float* __restrict__ inv_s, unsigned* __restrict__ part_cnt, int nsplit) {
+                const int* __restrict__ rows, uint16_t* __restrict__ B, float* __restrict__ inv_s,
+                unsigned* __restrict__ part_cnt, int nsplit) {
   extern __shared__ __align__(16) float buf[];  // [nb * 128]
   __shared__ float red[kRotThreads / 32];
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (m == 0)  // the K-split counters of the GEMM that follows start at zero
     for (int i = threadIdx.x; i < nsplit; i += kRotThreads) part_cnt[i] = 0u;
-  const uint16_t* x = X + static_cast<int64_t>(m) * ldx;
+  const uint16_t* x = X + static_cast<int64_t>(rows ? __ldg(rows + m) : m) * ldx;
   float s1[4] = {1.0f, 1.0f, 1.0f, 1.0f}, s2[4] = {1.0f, 1.0f, 1.0f, 1.0f};
   if (signs) {
 #pragma unroll
@@ -239,6 +242,63 @@ rotate_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int in, int nb, con
   for (int i = threadIdx.x; i < nb * kBlock; i += kRotThreads) dst[i] = __half_as_ushort(__float2half_rn(buf[i] * sc));
 }
 
+// The MoE layer's down-projection operand: one CTA per assignment row a of
+// G [NA][2F] (gate columns [0, F), up columns [F, 2F), fp32):
+// h = SiLU(g) * u = g / (1 + e^-g) * u, zero past F; then as rotate_x_kernel,
+// Bh[a][:] = binary16(h_tilde * s_a) with h_tilde_b = h_b @ H128, and
+// inv_s[a] = weight[a] / s_a (the down GEMM's output comes out weighted).
+__global__ void __launch_bounds__(kRotThreads)
+silu_rotate_kernel(const float* __restrict__ Gm, int F, int nb, const float* __restrict__ weight,
+                   uint16_t* __restrict__ Bh, float* __restrict__ inv_s) {
+  extern __shared__ __align__(16) float buf[];  // [nb * 128]
+  __shared__ float red[kRotThreads / 32];
+  const int a = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* g = Gm + static_cast<int64_t>(a) * 2 * F;
+  float mx = 0.0f;
+  for (int b = warp; b < nb; b += kRotThreads / 32) {
+    float e4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = kBlock * b + 4 * lane + k;
+      float h = 0.0f;
+      if (i < F) {
+        const float gv = g[i], up = g[F + i];
+        h = gv / (1.0f + expf(-gv)) * up;
+      }
+      e4[k] = h;
+    }
+    float p = e4[0] + e4[1], q = e4[0] - e4[1], r = e4[2] + e4[3], t = e4[2] - e4[3];
+    e4[0] = p + r; e4[1] = q + t; e4[2] = p - r; e4[3] = q - t;
+#pragma unroll
+    for (int hs = 1; hs < 32; hs <<= 1) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float o = __shfl_xor_sync(0xffffffffu, e4[k], hs);
+        e4[k] = (lane & hs) ? o - e4[k] : e4[k] + o;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      buf[kBlock * b + 4 * lane + k] = e4[k];
+      mx = fmaxf(mx, fabsf(e4[k]));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  float tmax = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kRotThreads / 32; ++w) tmax = fmaxf(tmax, red[w]);
+  int e = 0;
+  if (tmax > 0.0f && isfinite(tmax)) frexpf(tmax, &e);
+  const int k = max(-120, min(120, 15 - e));
+  const float sc = ldexpf(1.0f, k);
+  if (threadIdx.x == 0) inv_s[a] = ldexpf(1.0f, -k) * __ldg(weight + a);  // the routing weight rides on the scale
+  uint16_t* dst = Bh + static_cast<int64_t>(a) * nb * kBlock;
+  for (int i = threadIdx.x; i < nb * kBlock; i += kRotThreads) dst[i] = __half_as_ushort(__float2half_rn(buf[i] * sc));
+}
+
 // ---------------------------------------------------------------- main kernel
 // Rings: codes (one 128-row x 80-byte block column per stage, TMA) and A/B
 // stages (one 128-wide K block: A decoded into 64 TMEM columns, B as two
@@ -281,12 +341,27 @@ __host__ __device__ inline uint32_t tc_ab_parity(int b, int S) { return static_c
 __host__ __device__ inline int tc_code_stage(int b, int G) { return 2 * (b % G) + ((b / G) & 1); }
 __host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static_cast<uint32_t>(b / G / 2) & 1u; }
 
+// Grouped mode (the routed MoE layer): the weights are E experts stacked by
+// rows (rows_e rows each) and B holds one row per (token, expert) assignment,
+// grouped by expert.  CTA (slot, row tile j, token tile nt) multiplies the
+// rows of expert active[slot] with the B rows offsets[slot] ..
+// offsets[slot + 1] - 1 and writes Y[assignment][j * 128 + r].  Slots past the
+// active count (meta[0]), the expert id skip_id (handled apart) and token tiles
+// past an expert's assignments exit at once.  active == nullptr: plain mode.
+struct TcGroup {
+  const int* meta;
+  const int* active;
+  const int* offsets;
+  int rows_e, tiles_e, n_tiles, skip_id;
+};
+
 template <class F, int NG>
 __global__ void __launch_bounds__(TcRoles<NG>::kThreads, NG == 1 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
                const typename F::Norm* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
                const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box,
-               int row_tiles, int nfull, float* __restrict__ part, unsigned* __restrict__ part_cnt) {
+               int row_tiles, int nfull, float* __restrict__ part, unsigned* __restrict__ part_cnt,
+               const TcGroup grp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -322,8 +397,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     kb0 = half ? nb / 2 : 0;
     kb1 = half ? nb : nb / 2;
   }
-  const int64_t o0 = static_cast<int64_t>(tt % row_tiles) * kTcTileRows;
-  const int n0 = (tt / row_tiles) * n_box;
+  int64_t o0 = static_cast<int64_t>(tt % row_tiles) * kTcTileRows;  // first weight row of the tile
+  int64_t oend = O;                                                  // end of the rows the tile may read
+  int64_t oy0 = o0;                                                  // output column of the tile's first row
+  int n0 = (tt / row_tiles) * n_box;                                 // first B row of the tile
+  int mend = M;                                                      // end of the tile's valid B rows
+  if (grp.active) {
+    // grouped mode: a CTA-uniform early exit, before any barrier or TMEM
+    const int per = grp.tiles_e * grp.n_tiles;
+    const int slot = static_cast<int>(blockIdx.x) / per, rem = static_cast<int>(blockIdx.x) - slot * per;
+    if (slot >= __ldg(grp.meta)) return;
+    const int e = __ldg(grp.active + slot);
+    if (e == grp.skip_id) return;
+    const int a0 = __ldg(grp.offsets + slot), cnt = __ldg(grp.offsets + slot + 1) - a0;
+    const int j = rem / grp.n_tiles, nt = rem - j * grp.n_tiles;
+    if (nt * n_box >= cnt) return;
+    oy0 = static_cast<int64_t>(j) * kTcTileRows;
+    o0 = static_cast<int64_t>(e) * grp.rows_e + oy0;
+    oend = static_cast<int64_t>(e) * grp.rows_e + grp.rows_e;
+    n0 = a0 + nt * n_box;
+    mend = a0 + cnt;
+  }
   const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
 
   // ---- set-up: codebook, barriers, TMEM
@@ -361,7 +455,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // The tile's norms [128][nb] are one contiguous run of the norm array
     // (rows past O read as zero); they are staged while the producers start
     // on the first code and B boxes, then a barrier of the decode warps only.
-    const int64_t nvalid = std::min<int64_t>(kTcTileRows, O - o0) * nb;
+    const int64_t nvalid = std::min<int64_t>(kTcTileRows, oend - o0) * nb;
     const Norm* nsrc = norms + o0 * nb;
     const int ntot = kTcTileRows * nb;                                   // a multiple of 8
     constexpr int kPer16 = 16 / static_cast<int>(sizeof(Norm));          // norms per 16-byte load
@@ -498,7 +592,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const int m = n0 + c0 + h8 + j;
-              const float yv = m < M ? v[j] * rscale * __ldg(inv_s + m) : 0.0f;
+              const float yv = m < mend ? v[j] * rscale * __ldg(inv_s + m) : 0.0f;
               const int si = (c0 + h8 + j) * kTcTileRows + r;
               if (out_bf16) reinterpret_cast<uint16_t*>(stage)[si] = static_cast<uint16_t>(float_to_bf16_bits(yv));
               else reinterpret_cast<float*>(stage)[si] = yv;
@@ -507,13 +601,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         }
         asm volatile("bar.sync 2, %0;" ::"r"(32 * kTcDecWarps) : "memory");
         if (done && misc_g[1] == 0u) {
-          const int ncols = static_cast<int>(std::min<int64_t>(kTcTileRows, O - o0));  // outputs of the tile
-          const int mrows = std::min(n_box, M - n0);                                   // tokens of the tile
+          const int ncols = static_cast<int>(std::min<int64_t>(kTcTileRows, oend - o0));  // outputs of the tile
+          const int mrows = std::min(n_box, mend - n0);                                   // tokens of the tile
           char* yb = static_cast<char*>(Y);
           if (ncols == kTcTileRows && ((ldy * es) & 15) == 0) {
             const int sh = out_bf16 ? 4 : 5;  // 16-byte pieces per token: 128 x es / 16
             const int64_t pitch = ldy * es;
-            char* yt = yb + (static_cast<int64_t>(n0) * ldy + o0) * es;
+            char* yt = yb + (static_cast<int64_t>(n0) * ldy + oy0) * es;
             for (int q = threadIdx.x; q < (mrows << sh); q += 32 * kTcDecWarps) {
               const int ml = q >> sh, pc = q & ((1 << sh) - 1);
               *reinterpret_cast<uint4*>(yt + ml * pitch + 16 * pc) = reinterpret_cast<const uint4*>(stage)[q];
@@ -522,7 +616,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             for (int q = threadIdx.x; q < mrows * kTcTileRows; q += 32 * kTcDecWarps) {
               const int ml = q >> 7, oc = q & (kTcTileRows - 1);
               if (oc >= ncols) continue;
-              const int64_t off = (n0 + ml) * ldy + o0 + oc;
+              const int64_t off = (n0 + ml) * ldy + oy0 + oc;
               if (out_bf16) reinterpret_cast<uint16_t*>(yb)[off] = reinterpret_cast<const uint16_t*>(stage)[q];
               else reinterpret_cast<float*>(yb)[off] = reinterpret_cast<const float*>(stage)[q];
             }
@@ -687,43 +781,24 @@ size_t tq3_tc_workspace_min_bytes(int64_t O, int64_t in, int64_t M) {
   return tc_workspace_min_bytes<TcTq3>(O, in, M);
 }
 
-// Rotation of X into the workspace, then the tensor-core kernel (in <= 8192;
-// the workspace holds at least the plan's base_bytes).  signs: TQ3's sign
-// vectors, or nullptr for Q5.
+// The tensor-core kernel on a prepared B operand: binary16 [b_rows][nb * 128]
+// (K-major, 16-byte aligned rows), scales inv_s per B row.  Plain mode:
+// row_tiles x token tiles (the last partial wave split in K over nsplit tile
+// pairs); grouped mode: grp.active != nullptr, grid CTAs of the group mapping.
 template <class F>
-int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float* codebook, const int8_t* signs,
-              int64_t O, int in, const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16,
-              void* workspace, size_t ws_bytes, cudaStream_t stream) {
-  const int nb = static_cast<int>(ceil_div(in, kBlock));
-  const TcPlan P = tc_plan<F>(O, in, M);
-  if (ws_bytes < P.base_bytes) return HLWQ_EWORKSPACE;
-  const int nsplit = ws_bytes >= P.split_bytes ? P.nsplit : 0;
-  char* ws = static_cast<char*>(workspace);
-  uint16_t* B = reinterpret_cast<uint16_t*>(ws);
-  float* inv_s = reinterpret_cast<float*>(ws + P.inv_off);
-  unsigned* part_cnt = reinterpret_cast<unsigned*>(ws + P.cnt_off);
-  float* part = nsplit ? reinterpret_cast<float*>(ws + P.part_off) : nullptr;
-  const int rot_smem = nb * kBlock * 4;
-  if (rot_smem > 200 * 1024) return HLWQ_EUNSUPPORTED;
-  static PerDeviceOnce rot_attr;
-  if (const int st = rot_attr([&] {
-        return cudaFuncSetAttribute(rotate_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    200 * 1024) == cudaSuccess;
-      }))
-    return st;
-  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, signs, B, inv_s, part_cnt, nsplit);
-  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
-
-  const int n_box = P.n_box;
+int launch_tc_core(const uint8_t* packed, const typename F::Norm* norms, const float* codebook, int64_t O, int nb,
+                   const uint16_t* B, int64_t b_rows, int M, const float* inv_s, void* Y, int64_t ldy, bool out_bf16,
+                   int n_box, int row_tiles, int nfull, int nsplit, float* part, unsigned* part_cnt,
+                   const TcGroup& grp, cudaStream_t stream) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
   CUtensorMap map;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(nb) * kBlock, static_cast<cuuint64_t>(M)};
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(nb) * kBlock, static_cast<cuuint64_t>(b_rows)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(nb) * kBlock * 2};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcKChunk), static_cast<cuuint32_t>(n_box)};
   const cuuint32_t estr[2] = {1, 1};
-  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, B, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(B), gdim, gstride, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return HLWQ_ECUDA;
   // Codes viewed as a 2-D byte tensor [O][NB * bytes]; one box = 128 rows x
@@ -747,17 +822,111 @@ int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float*
       }))
     return st;
   if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
-  const int nfull = P.row_tiles * P.n_tiles - nsplit;
   const int grid = nfull + 2 * nsplit, ob = out_bf16 ? 1 : 0;
+  if (grid <= 0) return HLWQ_OK;
   if (tc_groups(n_box) == 1)
     gemm_tc_kernel<F, 1><<<grid, TcRoles<1>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
-                                                                       ldy, ob, n_box, P.row_tiles, nfull, part,
-                                                                       part_cnt);
+                                                                       ldy, ob, n_box, row_tiles, nfull, part,
+                                                                       part_cnt, grp);
   else
     gemm_tc_kernel<F, 2><<<grid, TcRoles<2>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
-                                                                       ldy, ob, n_box, P.row_tiles, nfull, part,
-                                                                       part_cnt);
+                                                                       ldy, ob, n_box, row_tiles, nfull, part,
+                                                                       part_cnt, grp);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+}
+
+inline int set_rot_attrs() {
+  static PerDeviceOnce rot_attr;
+  return rot_attr([&] {
+    return cudaFuncSetAttribute(rotate_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(silu_rotate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+               cudaSuccess;
+  });
+}
+
+// Rotation of X into the workspace, then the tensor-core kernel (in <= 8192;
+// the workspace holds at least the plan's base_bytes).  signs: TQ3's sign
+// vectors, or nullptr for Q5.
+template <class F>
+int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float* codebook, const int8_t* signs,
+              int64_t O, int in, const uint16_t* X, int64_t ldx, int M, void* Y, int64_t ldy, bool out_bf16,
+              void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  const int nb = static_cast<int>(ceil_div(in, kBlock));
+  const TcPlan P = tc_plan<F>(O, in, M);
+  if (ws_bytes < P.base_bytes) return HLWQ_EWORKSPACE;
+  const int nsplit = ws_bytes >= P.split_bytes ? P.nsplit : 0;
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* B = reinterpret_cast<uint16_t*>(ws);
+  float* inv_s = reinterpret_cast<float*>(ws + P.inv_off);
+  unsigned* part_cnt = reinterpret_cast<unsigned*>(ws + P.cnt_off);
+  float* part = nsplit ? reinterpret_cast<float*>(ws + P.part_off) : nullptr;
+  const int rot_smem = nb * kBlock * 4;
+  if (rot_smem > 200 * 1024) return HLWQ_EUNSUPPORTED;
+  if (const int st = set_rot_attrs()) return st;
+  rotate_x_kernel<<<M, kRotThreads, rot_smem, stream>>>(X, ldx, in, nb, signs, nullptr, B, inv_s, part_cnt, nsplit);
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  const int nfull = P.row_tiles * P.n_tiles - nsplit;
+  return launch_tc_core<F>(packed, norms, codebook, O, nb, B, M, M, inv_s, Y, ldy, out_bf16, P.n_box, P.row_tiles,
+                           nfull, nsplit, part, part_cnt, TcGroup{}, stream);
+}
+
+// The routed MoE layer on the tensor cores (the grouped path): after the
+// router has grouped the (token, expert) assignments by expert,
+//   1. rotate_x_kernel gathers and rotates each assignment's token (Bg);
+//   2. the grouped kernel multiplies every active expert's gate_up rows with
+//      its assignments' rows of Bg (each expert's codes decoded once for all
+//      its tokens), the shared expert as a plain launch on its T rows;
+//   3. silu_rotate_kernel forms h = SiLU(g) * u and rotates it (Bh), with the
+//      routing weight folded into the row scale;
+//   4. the same for the down rows into the per-assignment partial outputs;
+// the caller then adds the partials per token in a fixed order.
+// EUNSUPPORTED when rows are longer than the tile-norm staging allows.
+int launch_moe_tc(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+                  const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                  const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
+                  int topk, int T, const uint16_t* X, const MoeWs& ws, cudaStream_t stream) {
+  const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
+  if (nbh > kTcMaxNb || nbf > kTcMaxNb) return HLWQ_EUNSUPPORTED;
+  const bool shared = sh_gu_packed != nullptr;
+  const int na_routed = T * topk, na = na_routed + (shared ? T : 0);
+  int n_box = static_cast<int>(std::min<int64_t>(256, (static_cast<int64_t>(T) + 15) / 16 * 16));
+  while (n_box > 16 && tc_smem_bytes<TcQ5>(n_box, std::max(nbh, nbf)) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
+  const int n_tiles = static_cast<int>(ceil_div(T, n_box));  // an expert has at most T assignments
+  if (const int st = set_rot_attrs()) return st;
+  rotate_x_kernel<<<na, kRotThreads, nbh * kBlock * 4, stream>>>(X, H, H, nbh, nullptr, ws.asg_token, ws.bg, ws.inv_g,
+                                                                   nullptr, 0);
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  const int two_f = 2 * F;
+  TcGroup gu{ws.meta, ws.active, ws.offsets, two_f, static_cast<int>(ceil_div(two_f, kTcTileRows)), n_tiles, E};
+  int st = launch_tc_core<TcQ5>(gu_packed, gu_norms, codebook, static_cast<int64_t>(E) * two_f, nbh, ws.bg, na, na,
+                                ws.inv_g, ws.g2, two_f, false, n_box, 1, (E + 1) * gu.tiles_e * n_tiles, 0, nullptr,
+                                nullptr, gu, stream);
+  if (st) return st;
+  if (shared) {
+    const int rt = gu.tiles_e;
+    st = launch_tc_core<TcQ5>(sh_gu_packed, sh_gu_norms, codebook, two_f, nbh,
+                              ws.bg + static_cast<int64_t>(na_routed) * nbh * kBlock, T, T, ws.inv_g + na_routed,
+                              ws.g2 + static_cast<int64_t>(na_routed) * two_f, two_f, false, n_box, rt,
+                              rt * n_tiles, 0, nullptr, nullptr, TcGroup{}, stream);
+    if (st) return st;
+  }
+  silu_rotate_kernel<<<na, kRotThreads, nbf * kBlock * 4, stream>>>(ws.g2, F, nbf, ws.asg_weight, ws.bh, ws.inv_h);
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  TcGroup dn{ws.meta, ws.active, ws.offsets, H, static_cast<int>(ceil_div(H, kTcTileRows)), n_tiles, E};
+  st = launch_tc_core<TcQ5>(dn_packed, dn_norms, codebook, static_cast<int64_t>(E) * H, nbf, ws.bh, na, na, ws.inv_h,
+                            ws.part, H, false, n_box, 1, (E + 1) * dn.tiles_e * n_tiles, 0, nullptr, nullptr, dn,
+                            stream);
+  if (st) return st;
+  if (shared) {
+    const int rt = dn.tiles_e;
+    st = launch_tc_core<TcQ5>(sh_dn_packed, sh_dn_norms, codebook, H, nbf,
+                              ws.bh + static_cast<int64_t>(na_routed) * nbf * kBlock, T, T, ws.inv_h + na_routed,
+                              ws.part + static_cast<int64_t>(na_routed) * H, H, false, n_box, rt, rt * n_tiles, 0,
+                              nullptr, nullptr, TcGroup{}, stream);
+    if (st) return st;
+  }
+  return HLWQ_OK;
 }
 
 int launch_dense(const uint8_t* packed, const uint16_t* norms, const float* codebook, int64_t O, int in,

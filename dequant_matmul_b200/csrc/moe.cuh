@@ -47,6 +47,12 @@ struct MoeWs {
   float* xt_inv;      // [T][NBh] per-block activation scales
   float* h;           // [NA][F]
   float* part;        // [NA][H]
+  // tensor-core grouped path
+  uint16_t* bg;       // [NA][NBh * 128] rotated activation of each assignment's token (binary16)
+  float* inv_g;       // [NA] its scale
+  float* g2;          // [NA][2F] gate and up outputs (fp32)
+  uint16_t* bh;       // [NA][NBf * 128] rotated SiLU(g) * u (binary16)
+  float* inv_h;       // [NA] its scale times the assignment's routing weight
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -73,6 +79,12 @@ size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char
   w.xt_inv = reinterpret_cast<float*>(take(sizeof(float) * T * nbh));
   w.h = reinterpret_cast<float*>(take(sizeof(float) * na * F));
   w.part = reinterpret_cast<float*>(take(sizeof(float) * na * H));
+  const int64_t nbf = ceil_div(F, kBlock);
+  w.bg = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * na * nbh * kBlock));
+  w.inv_g = reinterpret_cast<float*>(take(sizeof(float) * na));
+  w.g2 = reinterpret_cast<float*>(take(sizeof(float) * na * 2 * F));
+  w.bh = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * na * nbf * kBlock));
+  w.inv_h = reinterpret_cast<float*>(take(sizeof(float) * na));
   if (ws) *ws = w;
   return off;
 }
@@ -397,6 +409,12 @@ size_t moe_workspace_bytes(int64_t E, int64_t H, int64_t F, int64_t T, int64_t t
   return moe_layout(E, H, F, T, topk, nullptr, nullptr);
 }
 
+// gemm_tc.cuh: gate_up and down of the grouped path on the tensor cores.
+int launch_moe_tc(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
+                  const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
+                  const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
+                  int topk, int T, const uint16_t* X, const MoeWs& ws, cudaStream_t stream);
+
 int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
                const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
                const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
@@ -405,15 +423,27 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
   MoeWs ws;
   moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
   const bool shared = sh_gu_packed != nullptr;
-  // CTA 0 routes; the others rotate every token's activation, about one
-  // 128-block per warp
-  const int64_t rot_warps = static_cast<int64_t>(T) * ceil_div(H, kBlock);
-  const int rot_ctas = static_cast<int>(std::min<int64_t>(4 * sm_count(), ceil_div(rot_warps, kRouterThreads / 32)));
+  const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
+  // gate_up and down on the tensor cores when the rows fit its tile-norm
+  // staging (in <= 8192), else on the CUDA-core decode engine
+  const bool tc = nbh <= 64 && nbf <= 64;
+  // CTA 0 routes; for the CUDA-core kernels the others rotate every token's
+  // activation, about one 128-block per warp
+  const int64_t rot_warps = static_cast<int64_t>(T) * nbh;
+  const int rot_ctas =
+      tc ? 0 : static_cast<int>(std::min<int64_t>(4 * sm_count(), ceil_div(rot_warps, kRouterThreads / 32)));
   router_kernel<<<1 + rot_ctas, kRouterThreads, 0, stream>>>(logits, X, E, H, T, topk, shared ? 1 : 0, ids_out,
                                                               w_out, ws);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  dim3 cgrid(static_cast<unsigned>(ceil_div(H, 256)), static_cast<unsigned>(T));
+  if (tc) {
+    if (const int st = launch_moe_tc(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+                                     sh_dn_norms, codebook, E, H, F, topk, T, X, ws, stream))
+      return st;
+    combine_kernel<<<cgrid, 256, 0, stream>>>(H, T, topk, ws, Y, out_bf16 ? 1 : 0);
+    return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
+  }
 
-  const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
   const int cg = pick_chunk(nbh), cd = pick_chunk(nbf);
   const int smem_g = engine_layout(kMoePass, nbh, 2 * kJT, (nbh + cg - 1) / cg).total;
   const int smem_d = engine_layout(kMoePass, nbf, kHT, (nbf + cd - 1) / cd).total;
@@ -441,7 +471,6 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
     default: down_kernel<2><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
   }
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
-  dim3 cgrid(static_cast<unsigned>(ceil_div(H, 256)), static_cast<unsigned>(T));
   combine_kernel<<<cgrid, 256, 0, stream>>>(H, T, topk, ws, Y, out_bf16 ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
