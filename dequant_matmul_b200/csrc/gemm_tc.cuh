@@ -308,7 +308,7 @@ __host__ __device__ constexpr int tc_code_bytes() { return kTcTileRows * F::kByt
 
 constexpr int kTcSmemMax = 227 * 1024;
 constexpr int kTcSmemFixed = 1024 /*align slack*/ + 1024 /*centroid table, barriers, misc*/;
-static_assert(4 * TcQ5::kLevels + 8 * (2 * kTcStages + 2 * 4 + 1) + 16 <= 1024, "barrier block overflows");
+static_assert(4 * TcQ5::kLevels + 8 * (2 * kTcStages + 2 * 4 + 1) + 16 <= 512, "barrier block overflows into the row maxima");
 constexpr int kTcMaxNb = 64;  // tile norms in shared memory: 128 x nb (in <= 8192)
 
 // Decode groups: G groups of 8 warps take blocks b = g (mod G).  Every ring
@@ -345,19 +345,22 @@ __host__ __device__ inline uint32_t tc_code_parity(int b, int G) { return static
 // rows (rows_e rows each) and B holds one row per (token, expert) assignment,
 // grouped by expert.  CTA (slot, row tile j, token tile nt) multiplies the
 // rows of expert active[slot] with the B rows offsets[slot] ..
-// offsets[slot + 1] - 1 and writes Y[assignment][j * 128 + r].  Slots past the
-// active count (meta[0]), the expert id skip_id (handled apart) and token tiles
-// past an expert's assignments exit at once.  active == nullptr: plain mode.
+// offsets[slot + 1] - 1 and writes Y[assignment][j * 128 + r].  The expert
+// id shared_id (the shared expert) reads its own matrix (second code map,
+// norms2).  Slots past the active count (meta[0]) and token tiles past an
+// expert's assignments exit at once.  active == nullptr: plain mode.
 struct TcGroup {
   const int* meta;
   const int* active;
   const int* offsets;
-  int rows_e, tiles_e, n_tiles, skip_id;
+  const void* norms2;
+  int rows_e, tiles_e, n_tiles, shared_id;
 };
 
 template <class F, int NG>
 __global__ void __launch_bounds__(TcRoles<NG>::kThreads, NG == 1 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap cmap,
+               const __grid_constant__ CUtensorMap cmap2,
                const typename F::Norm* __restrict__ norms, const float* __restrict__ codebook, int64_t O, int nb, int M,
                const float* __restrict__ inv_s, void* __restrict__ Y, int64_t ldy, int out_bf16, int n_box,
                int row_tiles, int nfull, float* __restrict__ part, unsigned* __restrict__ part_cnt,
@@ -402,31 +405,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   int64_t oy0 = o0;                                                  // output column of the tile's first row
   int n0 = (tt / row_tiles) * n_box;                                 // first B row of the tile
   int mend = M;                                                      // end of the tile's valid B rows
+  bool use2 = false;                                                 // the shared expert's own matrix
   if (grp.active) {
     // grouped mode: a CTA-uniform early exit, before any barrier or TMEM
     const int per = grp.tiles_e * grp.n_tiles;
     const int slot = static_cast<int>(blockIdx.x) / per, rem = static_cast<int>(blockIdx.x) - slot * per;
     if (slot >= __ldg(grp.meta)) return;
     const int e = __ldg(grp.active + slot);
-    if (e == grp.skip_id) return;
+    use2 = e == grp.shared_id;
     const int a0 = __ldg(grp.offsets + slot), cnt = __ldg(grp.offsets + slot + 1) - a0;
     const int j = rem / grp.n_tiles, nt = rem - j * grp.n_tiles;
     if (nt * n_box >= cnt) return;
     oy0 = static_cast<int64_t>(j) * kTcTileRows;
-    o0 = static_cast<int64_t>(e) * grp.rows_e + oy0;
-    oend = static_cast<int64_t>(e) * grp.rows_e + grp.rows_e;
+    const int64_t er = use2 ? 0 : static_cast<int64_t>(e) * grp.rows_e;  // the expert's first row
+    o0 = er + oy0;
+    oend = er + grp.rows_e;
     n0 = a0 + nt * n_box;
     mend = a0 + cnt;
   }
   const uint64_t deadline = globaltimer_ns() + wait_limit_ns();
 
-  // ---- set-up: codebook, barriers, TMEM
-  if (threadIdx.x < F::kLevels) {
-    const float c = __ldg(codebook + threadIdx.x);
-    c32[threadIdx.x] = c;
-    if (threadIdx.x + 1 < F::kLevels && !(c < __ldg(codebook + threadIdx.x + 1)))
-      raise_device_error(HLWQ_DEVERR_CODEBOOK);
-  }
+  // ---- set-up: barriers, TMEM, row maxima cleared (the codebook is loaded
+  // by the decode warps, whose own barrier publishes it)
+  uint32_t* rowmax = reinterpret_cast<uint32_t*>(gbase + 512);  // [128] fp32 bits, inside the first 1 KiB
+  if (threadIdx.x < kTcTileRows) rowmax[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 9);   // 8 decode warps + the B producer (plus its TMA bytes)
@@ -456,19 +458,49 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // (rows past O read as zero); they are staged while the producers start
     // on the first code and B boxes, then a barrier of the decode warps only.
     const int64_t nvalid = std::min<int64_t>(kTcTileRows, oend - o0) * nb;
-    const Norm* nsrc = norms + o0 * nb;
+    const Norm* nsrc = (use2 ? static_cast<const Norm*>(grp.norms2) : norms) + o0 * nb;
+    // Each row's largest norm is gathered on the way (shared-memory atomic
+    // max on the fp32 bits: the norms are >= 0; NaN is left out).
+    if (threadIdx.x < F::kLevels) {
+      const float c = __ldg(codebook + threadIdx.x);
+      c32[threadIdx.x] = c;
+      if (threadIdx.x + 1 < F::kLevels && !(c < __ldg(codebook + threadIdx.x + 1)))
+        raise_device_error(HLWQ_DEVERR_CODEBOOK);
+    }
+    auto row_max = [&](int k, float v) {
+      if (!(v != v)) atomicMax(rowmax + k / nb, __float_as_uint(v));
+    };
     const int ntot = kTcTileRows * nb;                                   // a multiple of 8
     constexpr int kPer16 = 16 / static_cast<int>(sizeof(Norm));          // norms per 16-byte load
     if ((reinterpret_cast<uintptr_t>(nsrc) & 15u) == 0) {
       for (int q = threadIdx.x; q < ntot / kPer16; q += 32 * kTcDecWarps) {
         if (kPer16 * q + kPer16 <= nvalid) {
-          reinterpret_cast<uint4*>(nrm_s)[q] = __ldg(reinterpret_cast<const uint4*>(nsrc) + q);
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(nsrc) + q);
+          reinterpret_cast<uint4*>(nrm_s)[q] = u;
+          const Norm* e = reinterpret_cast<const Norm*>(&u);
+          if (nb % kPer16 == 0) {  // the 16 bytes lie in one row: one atomic
+            float m = 0.0f;
+#pragma unroll
+            for (int k = 0; k < kPer16; ++k) m = fmaxf(m, F::norm(e[k]));
+            row_max(kPer16 * q, m);
+          } else {
+#pragma unroll
+            for (int k = 0; k < kPer16; ++k) row_max(kPer16 * q + k, F::norm(e[k]));
+          }
         } else {
-          for (int k = kPer16 * q; k < kPer16 * q + kPer16; ++k) nrm_s[k] = k < nvalid ? __ldg(nsrc + k) : Norm(0);
+          for (int k = kPer16 * q; k < kPer16 * q + kPer16; ++k) {
+            const Norm v = k < nvalid ? __ldg(nsrc + k) : Norm(0);
+            nrm_s[k] = v;
+            row_max(k, F::norm(v));
+          }
         }
       }
     } else {
-      for (int q = threadIdx.x; q < ntot; q += 32 * kTcDecWarps) nrm_s[q] = q < nvalid ? __ldg(nsrc + q) : Norm(0);
+      for (int q = threadIdx.x; q < ntot; q += 32 * kTcDecWarps) {
+        const Norm v = q < nvalid ? __ldg(nsrc + q) : Norm(0);
+        nrm_s[q] = v;
+        row_max(q, F::norm(v));
+      }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcDecWarps) : "memory");
 
@@ -478,8 +510,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     const int dg = warp >> 3, q4 = warp & 3, hh = (warp >> 2) & 1;  // group dg takes blocks b = dg mod G
     const int r = 32 * q4 + lane;
     const Norm* rown = nrm_s + r * nb;
-    float nmax = 0.0f;
-    for (int b = 0; b < nb; ++b) nmax = fmaxf(nmax, F::norm(rown[b]));
+    const float nmax = __uint_as_float(rowmax[r]);
     int erow = 0;
     if (nmax > 0.0f && isfinite(nmax)) frexpf(nmax, &erow);
     const float rs = ldexpf(1.0f, -erow);
@@ -635,7 +666,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         if (!ok) break;
         if (fault_skip_tma()) continue;
         mbar_arrive_expect_tx(c_full0 + 8 * cs, kCode);
-        tma_load_2d(cst + cs * kCode, &cmap, F::kBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
+        tma_load_2d(cst + cs * kCode, use2 ? &cmap2 : &cmap, F::kBytes * b, static_cast<int>(o0), c_full0 + 8 * cs);
         last = b;
       }
       if (!ok) {
@@ -789,7 +820,7 @@ template <class F>
 int launch_tc_core(const uint8_t* packed, const typename F::Norm* norms, const float* codebook, int64_t O, int nb,
                    const uint16_t* B, int64_t b_rows, int M, const float* inv_s, void* Y, int64_t ldy, bool out_bf16,
                    int n_box, int row_tiles, int nfull, int nsplit, float* part, unsigned* part_cnt,
-                   const TcGroup& grp, cudaStream_t stream) {
+                   const TcGroup& grp, cudaStream_t stream, const uint8_t* packed2 = nullptr, int64_t O2 = 0) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (!encode) return HLWQ_ECUDA;
   CUtensorMap map;
@@ -803,15 +834,19 @@ int launch_tc_core(const uint8_t* packed, const typename F::Norm* norms, const f
     return HLWQ_ECUDA;
   // Codes viewed as a 2-D byte tensor [O][NB * bytes]; one box = 128 rows x
   // one block (80 or 48 bytes: multiples of 16, as is every box's x offset).
-  CUtensorMap cmap;
-  const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(nb) * F::kBytes, static_cast<cuuint64_t>(O)};
+  CUtensorMap cmap, cmap2;
   const cuuint64_t cstride[1] = {static_cast<cuuint64_t>(nb) * F::kBytes};
   const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(F::kBytes), static_cast<cuuint32_t>(kTcTileRows)};
   static_assert(F::kBytes % 16 == 0, "code boxes start on 16-byte boundaries");
-  if (encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), cdim, cstride, cbox, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return HLWQ_ECUDA;
+  for (int k = 0; k < 2; ++k) {
+    const uint8_t* src = k == 0 ? packed : (packed2 ? packed2 : packed);
+    const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(nb) * F::kBytes,
+                                static_cast<cuuint64_t>(k == 0 || !packed2 ? O : O2)};
+    if (encode(k == 0 ? &cmap : &cmap2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(src), cdim, cstride,
+               cbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return HLWQ_ECUDA;
+  }
   const int smem = tc_smem_bytes<F>(n_box, nb);
   static PerDeviceOnce attr;
   if (const int st = attr([&] {
@@ -825,11 +860,11 @@ int launch_tc_core(const uint8_t* packed, const typename F::Norm* norms, const f
   const int grid = nfull + 2 * nsplit, ob = out_bf16 ? 1 : 0;
   if (grid <= 0) return HLWQ_OK;
   if (tc_groups(n_box) == 1)
-    gemm_tc_kernel<F, 1><<<grid, TcRoles<1>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
+    gemm_tc_kernel<F, 1><<<grid, TcRoles<1>::kThreads, smem, stream>>>(map, cmap, cmap2, norms, codebook, O, nb, M, inv_s, Y,
                                                                        ldy, ob, n_box, row_tiles, nfull, part,
                                                                        part_cnt, grp);
   else
-    gemm_tc_kernel<F, 2><<<grid, TcRoles<2>::kThreads, smem, stream>>>(map, cmap, norms, codebook, O, nb, M, inv_s, Y,
+    gemm_tc_kernel<F, 2><<<grid, TcRoles<2>::kThreads, smem, stream>>>(map, cmap, cmap2, norms, codebook, O, nb, M, inv_s, Y,
                                                                        ldy, ob, n_box, row_tiles, nfull, part,
                                                                        part_cnt, grp);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
@@ -876,7 +911,7 @@ int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float*
 //   1. rotate_x_kernel gathers and rotates each assignment's token (Bg);
 //   2. the grouped kernel multiplies every active expert's gate_up rows with
 //      its assignments' rows of Bg (each expert's codes decoded once for all
-//      its tokens), the shared expert as a plain launch on its T rows;
+//      its tokens; the shared expert, the last slot, from its own matrix);
 //   3. silu_rotate_kernel forms h = SiLU(g) * u and rotates it (Bh), with the
 //      routing weight folded into the row scale;
 //   4. the same for the down rows into the per-assignment partial outputs;
@@ -889,7 +924,7 @@ int launch_moe_tc(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint
   const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
   if (nbh > kTcMaxNb || nbf > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const bool shared = sh_gu_packed != nullptr;
-  const int na_routed = T * topk, na = na_routed + (shared ? T : 0);
+  const int na = T * topk + (shared ? T : 0);
   int n_box = static_cast<int>(std::min<int64_t>(256, (static_cast<int64_t>(T) + 15) / 16 * 16));
   while (n_box > 16 && tc_smem_bytes<TcQ5>(n_box, std::max(nbh, nbf)) > kTcSmemMax) n_box = (n_box / 2 + 15) / 16 * 16;
   const int n_tiles = static_cast<int>(ceil_div(T, n_box));  // an expert has at most T assignments
@@ -898,34 +933,21 @@ int launch_moe_tc(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint
                                                                    nullptr, 0);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
   const int two_f = 2 * F;
-  TcGroup gu{ws.meta, ws.active, ws.offsets, two_f, static_cast<int>(ceil_div(two_f, kTcTileRows)), n_tiles, E};
+  const int nslots = E + (shared ? 1 : 0);
+  TcGroup gu{ws.meta, ws.active, ws.offsets, sh_gu_norms, two_f, static_cast<int>(ceil_div(two_f, kTcTileRows)),
+             n_tiles, shared ? E : -1};
   int st = launch_tc_core<TcQ5>(gu_packed, gu_norms, codebook, static_cast<int64_t>(E) * two_f, nbh, ws.bg, na, na,
-                                ws.inv_g, ws.g2, two_f, false, n_box, 1, (E + 1) * gu.tiles_e * n_tiles, 0, nullptr,
-                                nullptr, gu, stream);
+                                ws.inv_g, ws.g2, two_f, false, n_box, 1, nslots * gu.tiles_e * n_tiles, 0, nullptr,
+                                nullptr, gu, stream, sh_gu_packed, two_f);
   if (st) return st;
-  if (shared) {
-    const int rt = gu.tiles_e;
-    st = launch_tc_core<TcQ5>(sh_gu_packed, sh_gu_norms, codebook, two_f, nbh,
-                              ws.bg + static_cast<int64_t>(na_routed) * nbh * kBlock, T, T, ws.inv_g + na_routed,
-                              ws.g2 + static_cast<int64_t>(na_routed) * two_f, two_f, false, n_box, rt,
-                              rt * n_tiles, 0, nullptr, nullptr, TcGroup{}, stream);
-    if (st) return st;
-  }
   silu_rotate_kernel<<<na, kRotThreads, nbf * kBlock * 4, stream>>>(ws.g2, F, nbf, ws.asg_weight, ws.bh, ws.inv_h);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
-  TcGroup dn{ws.meta, ws.active, ws.offsets, H, static_cast<int>(ceil_div(H, kTcTileRows)), n_tiles, E};
+  TcGroup dn{ws.meta, ws.active, ws.offsets, sh_dn_norms, H, static_cast<int>(ceil_div(H, kTcTileRows)), n_tiles,
+             shared ? E : -1};
   st = launch_tc_core<TcQ5>(dn_packed, dn_norms, codebook, static_cast<int64_t>(E) * H, nbf, ws.bh, na, na, ws.inv_h,
-                            ws.part, H, false, n_box, 1, (E + 1) * dn.tiles_e * n_tiles, 0, nullptr, nullptr, dn,
-                            stream);
+                            ws.part, H, false, n_box, 1, nslots * dn.tiles_e * n_tiles, 0, nullptr, nullptr, dn, stream,
+                            sh_dn_packed, H);
   if (st) return st;
-  if (shared) {
-    const int rt = dn.tiles_e;
-    st = launch_tc_core<TcQ5>(sh_dn_packed, sh_dn_norms, codebook, H, nbf,
-                              ws.bh + static_cast<int64_t>(na_routed) * nbf * kBlock, T, T, ws.inv_h + na_routed,
-                              ws.part + static_cast<int64_t>(na_routed) * H, H, false, n_box, rt, rt * n_tiles, 0,
-                              nullptr, nullptr, TcGroup{}, stream);
-    if (st) return st;
-  }
   return HLWQ_OK;
 }
 

@@ -161,7 +161,7 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ lg, i
 __global__ void __launch_bounds__(kRouterThreads, 1)
 router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, int E, int H, int T, int topk,
               int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
-  __shared__ int s_count[1025];
+  __shared__ int s_count[1025], s_cursor[1025], s_wsum[32], s_wact[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (blockIdx.x > 0) {
     // CTAs 1.. rotate the tokens' activations (binary16, per-block power-of-
@@ -192,52 +192,60 @@ router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, 
   }
   __syncthreads();
 
-  // 2. assignments per expert (id E = shared expert, every token).
+  // 2. assignments per expert (id E = shared expert, every token): counts by
+  // shared-memory atomics, active slots and offsets by a block-wide scan,
+  // then every selection placed at its expert's cursor.  The order of an
+  // expert's assignments is not fixed, and nothing depends on it: every
+  // assignment is computed on its own and each token's partials are added
+  // through tok_asg in slot order.
   const int nexp = E + (has_shared ? 1 : 0);
-  for (int e = threadIdx.x; e < nexp; e += kRouterThreads) {
-    int c = 0;
-    if (e == E) c = T;
-    else
-      for (int q = 0; q < T * topk; ++q) c += ws.sel_id[q] == e;
-    s_count[e] = c;
-  }
+  const int nsel = T * topk;
+  for (int e = threadIdx.x; e < nexp; e += kRouterThreads) s_count[e] = (e == E) ? T : 0;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int na = 0, off = 0;
-    for (int e = 0; e < nexp; ++e) {
-      if (s_count[e]) {
-        ws.active[na] = e;
-        ws.offsets[na] = off;
-        off += s_count[e];
-        s_count[e] = na;  // reuse: active slot of expert e
-        ++na;
-      } else {
-        s_count[e] = -1;
-      }
+  for (int q = threadIdx.x; q < nsel; q += kRouterThreads) atomicAdd(&s_count[ws.sel_id[q]], 1);
+  __syncthreads();
+  {
+    // thread t owns experts 2t and 2t + 1 (nexp <= 1025 <= 2 * kRouterThreads)
+    const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+    const int c0 = e0 < nexp ? s_count[e0] : 0, c1 = e1 < nexp ? s_count[e1] : 0;
+    int cnt = c0 + c1, act = (c0 > 0) + (c1 > 0);
+    // inclusive warp scans, then the warps' totals
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, cnt, off), b = __shfl_up_sync(0xffffffffu, act, off);
+      if (lane >= off) { cnt += a; act += b; }
     }
-    ws.offsets[na] = off;
-    ws.meta[0] = na;
+    if (lane == 31) { s_wsum[warp] = cnt; s_wact[warp] = act; }
+    __syncthreads();
+    if (warp == 0) {
+      int wc = s_wsum[lane], wa = s_wact[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, wc, off), b = __shfl_up_sync(0xffffffffu, wa, off);
+        if (lane >= off) { wc += a; wa += b; }
+      }
+      s_wsum[lane] = wc - s_wsum[lane];  // exclusive
+      s_wact[lane] = wa - s_wact[lane];
+      if (lane == 31) { ws.offsets[wa] = wc; ws.meta[0] = wa; }
+    }
+    __syncthreads();
+    int off = s_wsum[warp] + cnt - c0 - c1, slot = s_wact[warp] + act - (c0 > 0) - (c1 > 0);
+    if (c0 > 0) { ws.active[slot] = e0; ws.offsets[slot] = off; s_cursor[e0] = off; off += c0; ++slot; }
+    if (c1 > 0) { ws.active[slot] = e1; ws.offsets[slot] = off; s_cursor[e1] = off; }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < nexp; e += kRouterThreads) {
-    const int slot = s_count[e];
-    if (slot < 0) continue;
-    int pos = ws.offsets[slot];
-    if (e == E) {
-      for (int t = 0; t < T; ++t, ++pos) {
-        ws.asg_token[pos] = t;
-        ws.asg_weight[pos] = 1.0f;
-        ws.tok_asg[t * (topk + 1) + topk] = pos;
-      }
-    } else {
-      for (int q = 0; q < T * topk; ++q) {
-        if (ws.sel_id[q] == e) {
-          ws.asg_token[pos] = q / topk;
-          ws.asg_weight[pos] = ws.sel_w[q];
-          ws.tok_asg[(q / topk) * (topk + 1) + (q % topk)] = pos;
-          ++pos;
-        }
-      }
+  for (int q = threadIdx.x; q < nsel; q += kRouterThreads) {
+    const int pos = atomicAdd(&s_cursor[ws.sel_id[q]], 1);
+    ws.asg_token[pos] = q / topk;
+    ws.asg_weight[pos] = ws.sel_w[q];
+    ws.tok_asg[(q / topk) * (topk + 1) + (q % topk)] = pos;
+  }
+  if (has_shared) {
+    const int base = s_cursor[E];
+    for (int t = threadIdx.x; t < T; t += kRouterThreads) {
+      ws.asg_token[base + t] = t;
+      ws.asg_weight[base + t] = 1.0f;
+      ws.tok_asg[t * (topk + 1) + topk] = base + t;
     }
   }
   if (!has_shared)

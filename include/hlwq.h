@@ -325,14 +325,22 @@ int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * hlwq_moe_gemv with launch flags.  flags = 0 is hlwq_moe_gemv (the fused
- * two-kernel path when its shared memory fits -- few tokens -- else the
- * grouped path).  HLWQ_FLAG_MOE_GROUPED selects the grouped path at any T:
- * four launches (routing and per-expert assignment lists with every token's
- * rotated activation; gate_up over (active expert, 32 columns) units that
- * read each active expert's codes once for all its tokens; down over (active
- * expert, 128 rows) units; a fixed-order combine).  Same arguments, results
- * and workspace; other bits are HLWQ_EINVAL.
+ * hlwq_moe_gemv with launch flags.  flags = 0 is hlwq_moe_gemv: the fused
+ * two-kernel path while 4 * T * topk < 3 * E (fewer assignments than about
+ * three quarters of the experts) and its shared memory fits, else the
+ * grouped path.
+ * HLWQ_FLAG_MOE_GROUPED selects the grouped path at any T.  The grouped path
+ * reads each active expert's codes once for all its tokens:
+ *   routing and per-expert assignment lists;
+ *   for H and F up to 8192, on the tensor cores: each assignment's token
+ *   gathered and rotated, gate_up as one grouped tcgen05 GEMM over (active
+ *   expert, 128-row tile), SiLU(g) * u rotated with the routing weight on its
+ *   scale, down as a grouped GEMM; the shared expert as plain GEMMs;
+ *   for longer rows, on the CUDA cores: gate_up over (active expert, 32
+ *   columns) units, down over (active expert, 128 rows) units;
+ *   a fixed-order combine of each token's partial outputs.
+ * Same arguments, results (to rounding) and workspace; other flag bits are
+ * HLWQ_EINVAL.
  */
 int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_norms,
                      const uint8_t* dn_packed, const uint16_t* dn_norms,
