@@ -28,10 +28,11 @@ def expert_weights(E, H, F, seed):
     return gu, dn
 
 
-def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_only=False, flags=0):
+def run_case(hl, cb, E, H, F, T, topk, shared, seed, odt=torch.float32, used_only=False, flags=0, logits=None):
     """Oracle-quantized experts on both sides (only the experts the oracle's
     router picks are encoded when used_only; the others stay zero on the GPU)."""
-    logits = synth.router_logits(T, E, seed=seed)
+    if logits is None:
+        logits = synth.router_logits(T, E, seed=seed)
     X = synth.activations(T, H, seed=seed + 1)
     ids_ref, _ = O.router_topk(logits, topk)
     need = set(ids_ref.reshape(-1).tolist()) if used_only else set(range(E))
@@ -105,6 +106,16 @@ def test_moe_many_tokens_default_falls_back_to_grouped(hl, cb):
     err_g = run_case(hl, cb, E=32, H=256, F=128, T=400, topk=8, shared=True, seed=612,
                      flags=hl.HLWQ_FLAG_MOE_GROUPED)
     assert err == err_g   # the same kernels ran
+
+
+def test_moe_grouped_path_one_expert_set_for_every_token(hl, cb):
+    """Every token routes to the same top-3 experts (one logit row repeated):
+    those experts get T = 300 assignments each, more than one 256-token tile,
+    and the other 13 experts none."""
+    row = synth.router_logits(1, 16, seed=613)
+    logits = row.repeat(300, 1)
+    run_case(hl, cb, E=16, H=256, F=128, T=300, topk=3, shared=True, seed=613, logits=logits,
+             flags=hl.HLWQ_FLAG_MOE_GROUPED)
 
 
 def test_moe_ex_rejects_unknown_flags(hl, cb):
