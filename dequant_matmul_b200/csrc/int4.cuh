@@ -25,10 +25,13 @@
 // the exact weights (7 rounded butterfly stages whose partial sums are bounded
 // by sum |c|, plus the scaling), so the fp32 results are certain when s and z
 // round to the same bfloat16 for every value within that bound, and every
-// quotient lies farther than E / s + 4e-6 from a half-way point.  A warp with
-// any block that fails these checks recomputes all its blocks in fp64 (the
-// exact path: every step in fp64, the quotient as (w - z) * (1 / s) with the
-// division where that product lies within 8 ulps of a half-way point).
+// quotient lies farther than E / s + 4e-6 from a half-way point.  A block
+// that fails these checks is marked (its scale set to 0xffff, a bfloat16 NaN
+// that no block's scale can be) and left to a second kernel, which gathers the
+// marked blocks eight per warp and takes the exact path for each (every step
+// in fp64, the quotient as (w - z) * (1 / s) with the division where that
+// product lies within 8 ulps of a half-way point).  About 0.2 % of the blocks
+// of a layer are marked, so the fp64 work is that small share.
 //
 // Layout as the dequantizer: four lanes per 128-block, 32 values each; the
 // inverse rotation is 5 register butterfly stages and 2 shuffle stages.
@@ -42,6 +45,7 @@ namespace {
 
 constexpr int kI4Threads = 256;
 constexpr int kI4GroupBytes = kBlock / 2;  // 64
+constexpr uint16_t kI4Unsure = 0xffffu;      // scale mark of a block left to the exact path
 
 // bfloat16 bits of a finite fp64 value, round to nearest even.
 __device__ __forceinline__ uint32_t bf16_rne_from_f64(double x) {
@@ -172,11 +176,59 @@ requantize_int4_kernel(const uint8_t* __restrict__ packed, const uint16_t* __res
         }
       }
     }
-    // ---- exact path (fp64) for every block of a warp with an uncertain one
-    if (__any_sync(0xffffffffu, !sure)) {
+    // the quad's verdict: every lane of the block must be sure
+    sure = __shfl_xor_sync(0xffffffffu, sure, 1) && sure;
+    sure = __shfl_xor_sync(0xffffffffu, sure, 2) && sure;
+    if (active && sure) {
+      *reinterpret_cast<uint4*>(q4 + F * kI4GroupBytes + 16 * q) = make_uint4(out[0], out[1], out[2], out[3]);
+      if (q == 0) {
+        scale[F] = static_cast<uint16_t>(s16);
+        zero[F] = static_cast<uint16_t>(z16);
+      }
+    } else if (active && q == 0) {
+      scale[F] = kI4Unsure;  // the exact kernel takes this block
+    }
+  }
+}
+
+// The exact path for the blocks the fast kernel marked: a warp looks at 32
+// consecutive blocks, gathers the marked ones and encodes them eight at a
+// time (one block per quad of lanes), every step in fp64.
+__global__ void __launch_bounds__(kI4Threads)
+requantize_int4_exact_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
+                             const float* __restrict__ codebook, int64_t nblocks, uint8_t* __restrict__ q4,
+                             uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  __shared__ float cb32[kLevels];
+  if (threadIdx.x < kLevels) cb32[threadIdx.x] = __ldg(codebook + threadIdx.x);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, q = lane & 3, quad = lane >> 2;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kI4Threads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kI4Threads / 32);
+  for (int64_t first = warp * 32; first < nblocks; first += nwarps * 32) {
+    const int64_t mine = first + lane;
+    uint32_t marked = __ballot_sync(0xffffffffu, mine < nblocks && scale[mine] == kI4Unsure);
+    while (marked) {
+      // the quad takes the quad-th marked block of this round (if any)
+      uint32_t m = marked;
+      for (int k = 0; k < quad && m; ++k) m &= m - 1;
+      const bool active = m != 0u;
+      const int64_t F = active ? first + (__ffs(m) - 1) : first;
+      for (int k = 0; k < 8 && marked; ++k) marked &= marked - 1;  // eight blocks per round
+      uint32_t w[5] = {0u, 0u, 0u, 0u, 0u};
+      double nsc = 0.0;
+      if (active) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + F * kBlockBytes + 20 * q);
+#pragma unroll
+        for (int k = 0; k < 5; ++k) w[k] = __ldg(src + k);
+        nsc = static_cast<double>(half_bits_to_float(__ldg(norms + F))) * (1.0 / 128.0);
+      }
       double v[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = static_cast<double>(cb32[code5[e]]);
+      for (int e = 0; e < 32; ++e) {
+        const int bit = 5 * e, k = bit >> 5, sh = bit & 31;
+        const uint32_t c = (sh <= 27) ? ((w[k] >> sh) & 31u) : (__funnelshift_r(w[k], w[k + 1], sh) & 31u);
+        v[e] = static_cast<double>(cb32[c]);
+      }
       stage32_f64<1>(v);
       stage32_f64<2>(v);
       stage32_f64<4>(v);
@@ -193,31 +245,30 @@ requantize_int4_kernel(const uint8_t* __restrict__ packed, const uint16_t* __res
       }
       lo = quad_min_f64(lo);
       hi = quad_max_f64(hi);
-      s16 = bf16_rne_from_f64((hi - lo) / 15.0);
-      z16 = bf16_rne_from_f64(__dadd_rn(lo, 0.0));  // a zero minimum is stored as +0
-      const double s = bf16_bits_to_f64(s16), z = bf16_bits_to_f64(z16);
-      const double rs = s > 0.0 ? 1.0 / s : 0.0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) out[k] = 0u;
+      const uint32_t s16 = bf16_rne_from_f64((hi - lo) / 15.0);
+      const uint32_t z16 = bf16_rne_from_f64(__dadd_rn(lo, 0.0));  // a zero minimum is stored as +0
+      const double sv = bf16_bits_to_f64(s16), z = bf16_bits_to_f64(z16);
+      const double rs = sv > 0.0 ? 1.0 / sv : 0.0;
+      uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         uint32_t code = 0u;
-        if (s > 0.0) {
+        if (sv > 0.0) {
           const double d = v[e] - z;
           double t = d * rs;
           // within 8 ulps of a half-way point: the division decides
           const double f = t - floor(t);
-          if (fabs(f - 0.5) <= 8.0 * 2.220446049250313e-16 * fmax(fabs(t), 1.0)) t = d / s;
+          if (fabs(f - 0.5) <= 8.0 * 2.220446049250313e-16 * fmax(fabs(t), 1.0)) t = d / sv;
           code = static_cast<uint32_t>(fmin(fmax(rint(t), 0.0), 15.0));
         }
         out[e >> 3] |= code << (4 * (e & 7));
       }
-    }
-    if (active) {
-      *reinterpret_cast<uint4*>(q4 + F * kI4GroupBytes + 16 * q) = make_uint4(out[0], out[1], out[2], out[3]);
-      if (q == 0) {
-        scale[F] = static_cast<uint16_t>(s16);
-        zero[F] = static_cast<uint16_t>(z16);
+      if (active) {
+        *reinterpret_cast<uint4*>(q4 + F * kI4GroupBytes + 16 * q) = make_uint4(out[0], out[1], out[2], out[3]);
+        if (q == 0) {
+          zero[F] = static_cast<uint16_t>(z16);
+          scale[F] = static_cast<uint16_t>(s16);
+        }
       }
     }
   }
@@ -231,6 +282,9 @@ int launch_requantize_int4(const uint8_t* packed, const uint16_t* norms, const f
   const int64_t max_ctas = static_cast<int64_t>(sm_count()) * 8;
   const int grid = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(nblocks, kI4Threads / 4)));
   requantize_int4_kernel<<<grid, kI4Threads, 0, stream>>>(packed, norms, codebook, nblocks, q4, scale, zero);
+  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  const int grid2 = static_cast<int>(std::min<int64_t>(max_ctas, ceil_div(nblocks, kI4Threads)));
+  requantize_int4_exact_kernel<<<grid2, kI4Threads, 0, stream>>>(packed, norms, codebook, nblocks, q4, scale, zero);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }
 
