@@ -429,7 +429,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
   // by the decode warps, whose own barrier publishes it)
   uint32_t* rowmax = reinterpret_cast<uint32_t*>(gbase + 512);  // [128] fp32 bits, inside the first 1 KiB
   if (threadIdx.x < kTcTileRows) rowmax[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) {
+  // The code producer initialises the barriers and requests the first code
+  // boxes (one per code stage) before the CTA barrier, so that their memory
+  // latency overlaps the TMEM allocation and the norm loads.
+  const int early = std::min(kb1 - kb0, CS);
+  if (warp == kTcWCodes && lane == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 9);   // 8 decode warps + the B producer (plus its TMA bytes)
       mbar_init(empty0 + 8 * s, 1);  // the MMA commit
@@ -440,7 +444,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     }
     mbar_init(accum, 1);
     misc_g[1] = 0u;  // abort flag
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_barrier_init();
+    for (int lb = 0; lb < early; ++lb) {
+      const int cs = tc_code_stage(lb, G);
+      if (fault_skip_tma()) continue;
+      mbar_arrive_expect_tx(c_full0 + 8 * cs, kCode);
+      tma_load_2d(cst + cs * kCode, use2 ? &cmap2 : &cmap, F::kBytes * (kb0 + lb), static_cast<int>(o0),
+                  c_full0 + 8 * cs);
+    }
   }
   if (warp == kTcWMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(misc), "r"(alloc_cols)
@@ -659,8 +670,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // ---------------------------------------------------------- TMA producer: code tiles
     if (lane == 0) {
       bool ok = true;
-      int last = -1;  // last block whose copy was issued
-      for (int b = kb0; b < kb1; ++b) {
+      int last = early > 0 && !fault_skip_tma() ? kb0 + early - 1 : -1;  // last block whose copy was issued
+      for (int b = kb0 + early; b < kb1; ++b) {
         const int cs = tc_code_stage(b - kb0, G);
         ok = mbar_wait(c_empty0 + 8 * cs, tc_code_parity(b - kb0, G) ^ 1u, deadline) && misc_g[1] == 0u;
         if (!ok) break;
