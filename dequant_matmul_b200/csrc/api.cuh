@@ -307,16 +307,17 @@ extern "C" int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_nor
   const size_t need = hlwq_workspace_bytes(HLWQ_OP_MOE, H, F, T, E, topk);
   if (!workspace || ws_bytes < need) return HLWQ_EWORKSPACE;
   if (!aligned16(workspace)) return HLWQ_EALIGN;
-  // few tokens: two fused kernels on the TMA-fed decode engine; otherwise (or
-  // when the pairs' activations do not fit in shared memory) the four-kernel
-  // path that reads each active expert once for all its tokens
+  // The grouped path (tensor cores, H and F up to 16384) reads each active
+  // expert once for all its tokens; it pays off once the assignments reach
+  // about three quarters of the experts (measured on the 256- and 128-expert
+  // layers: the fused path is faster below, the grouped path from there on).
+  // The fused path also runs when the grouped path cannot; the grouped path
+  // when the fused one's shared memory does not fit.
+  const bool grouped_ok = H <= 16384 && F <= 16384;
+  if ((flags & HLWQ_FLAG_MOE_GROUPED) && !grouped_ok) return HLWQ_EUNSUPPORTED;
   hlwq::MoeWs ws;
   hlwq::moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
-  // The grouped path reads each active expert once for all its tokens; it
-  // pays off once the assignments reach about three quarters of the experts
-  // (measured on the 256- and 128-expert layers: the fused path is faster
-  // below, the grouped path from there on).
-  const bool grouped = (flags & HLWQ_FLAG_MOE_GROUPED) || (4 * T * topk >= 3 * E && H <= 8192 && F <= 8192);
+  const bool grouped = (flags & HLWQ_FLAG_MOE_GROUPED) || (4 * T * topk >= 3 * E && grouped_ok);
   const int st = grouped ? HLWQ_EUNSUPPORTED : hlwq::launch_moe1(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
                                    sh_dn_norms, codebook, static_cast<int>(E), static_cast<int>(H),
                                    static_cast<int>(F), static_cast<int>(topk), static_cast<int>(T), router_logits, X,

@@ -867,7 +867,7 @@ int launch_tc_core(const uint8_t* packed, const typename F::Norm* norms, const f
                                     227 * 1024) == cudaSuccess;
       }))
     return st;
-  if (smem > kTcSmemMax || nb > kTcMaxNb) return HLWQ_EUNSUPPORTED;
+  if (smem > kTcSmemMax) return HLWQ_EUNSUPPORTED;
   const int grid = nfull + 2 * nsplit, ob = out_bf16 ? 1 : 0;
   if (grid <= 0) return HLWQ_OK;
   if (tc_groups(n_box) == 1)
@@ -927,13 +927,12 @@ int launch_tc(const uint8_t* packed, const typename F::Norm* norms, const float*
 //      routing weight folded into the row scale;
 //   4. the same for the down rows into the per-assignment partial outputs;
 // the caller then adds the partials per token in a fixed order.
-// EUNSUPPORTED when rows are longer than the tile-norm staging allows.
+// EUNSUPPORTED when the rows' tile norms do not fit the shared memory.
 int launch_moe_tc(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t* dn_packed,
                   const uint16_t* dn_norms, const uint8_t* sh_gu_packed, const uint16_t* sh_gu_norms,
                   const uint8_t* sh_dn_packed, const uint16_t* sh_dn_norms, const float* codebook, int E, int H, int F,
                   int topk, int T, const uint16_t* X, const MoeWs& ws, cudaStream_t stream) {
   const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
-  if (nbh > kTcMaxNb || nbf > kTcMaxNb) return HLWQ_EUNSUPPORTED;
   const bool shared = sh_gu_packed != nullptr;
   const int na = T * topk + (shared ? T : 0);
   int n_box = static_cast<int>(std::min<int64_t>(256, (static_cast<int64_t>(T) + 15) / 16 * 16));

@@ -10,17 +10,14 @@
 //   g || u = w_hat_gu[e] @ x_t (rows [0, F) gate, [F, 2F) up), h = SiLU(g) * u;
 //   Y[t]   = sum_s p_s * w_hat_dn[ids_s] @ h_s  (+ shared expert with weight 1).
 //
-// Four launches, no atomics, deterministic:
-//   1. router: CTA 0 does top-k + softmax per token and the per-expert
-//      assignment lists sorted by (expert, token); the other CTAs rotate the
-//      activations of every token;
-//   2. gate_up: persistent CTAs over units (active expert, 32 intermediate
-//      columns); each unit decodes its gate and up rows against the tokens
-//      routed to that expert (each expert's codes are read once per call) and
-//      writes h = SiLU(g) * u in fp32;
-//   3. down: units (active expert, 128 output rows); h of the expert's tokens is
-//      rotated in the CTA, the weighted result goes to a per-assignment slot;
-//   4. combine: Y[t] = sum over the token's assignment slots in a fixed order.
+// The grouped path (the fused two-kernel path for few tokens is moe1.cuh):
+//   1. router_kernel (one CTA): top-k + softmax per token, then the
+//      per-expert assignment lists (shared-memory atomics and a block scan);
+//   2. gate_up, SiLU and down on the tensor cores, each active expert's codes
+//      decoded once for all its tokens (launch_moe_tc, gemm_tc.cuh);
+//   3. combine: Y[t] = sum over the token's assignment slots in a fixed order.
+// Deterministic: the order of an expert's assignments varies with the
+// atomics, but each assignment is computed on its own.
 
 #include <algorithm>
 
@@ -31,8 +28,7 @@ namespace hlwq {
 namespace {
 
 constexpr int kRouterThreads = 1024;
-constexpr int kJT = 32;   // intermediate columns per gate_up unit
-constexpr int kHT = 128;  // output rows per down unit
+constexpr int kMoeMaxIn = 16384;  // H and F of the grouped path (tile norms of up to 128 blocks)
 
 struct MoeWs {
   int* meta;          // [0] = number of active experts (shared expert last)
@@ -43,8 +39,6 @@ struct MoeWs {
   int* tok_asg;       // [T][topk + 1] assignment index per (token, slot), -1 = none
   int* sel_id;        // [T][topk]
   float* sel_w;       // [T][topk]
-  uint16_t* xt;       // [T][NBh][kXsStride] rotated tokens (binary16)
-  float* xt_inv;      // [T][NBh] per-block activation scales
   float* h;           // [NA][F]
   float* part;        // [NA][H]
   // tensor-core grouped path
@@ -75,8 +69,6 @@ size_t moe_layout(int64_t E, int64_t H, int64_t F, int64_t T, int64_t topk, char
   w.tok_asg = reinterpret_cast<int*>(take(sizeof(int) * T * (topk + 1)));
   w.sel_id = reinterpret_cast<int*>(take(sizeof(int) * T * topk));
   w.sel_w = reinterpret_cast<float*>(take(sizeof(float) * T * topk));
-  w.xt = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * T * nbh * kXsStride));
-  w.xt_inv = reinterpret_cast<float*>(take(sizeof(float) * T * nbh));
   w.h = reinterpret_cast<float*>(take(sizeof(float) * na * F));
   w.part = reinterpret_cast<float*>(take(sizeof(float) * na * H));
   const int64_t nbf = ceil_div(F, kBlock);
@@ -159,28 +151,10 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ lg, i
 }
 
 __global__ void __launch_bounds__(kRouterThreads, 1)
-router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, int E, int H, int T, int topk,
-              int has_shared, int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
+router_kernel(const float* __restrict__ logits, int E, int T, int topk, int has_shared,
+              int32_t* __restrict__ ids_out, float* __restrict__ w_out, MoeWs ws) {
   __shared__ int s_count[1025], s_cursor[1025], s_wsum[32], s_wact[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (blockIdx.x > 0) {
-    // CTAs 1.. rotate the tokens' activations (binary16, per-block power-of-
-    // two scale), one 128-block per warp at a time
-    const int nbh = (H + kBlock - 1) / kBlock;
-    const int nwarps = (gridDim.x - 1) * (kRouterThreads / 32);
-    for (int q = (blockIdx.x - 1) * (kRouterThreads / 32) + warp; q < T * nbh; q += nwarps) {
-      const int m = q / nbh, b = q - m * nbh;
-      float e4[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = kBlock * b + 4 * lane + k;
-        e4[k] = i < H ? bf16_bits_to_float(__ldg(X + static_cast<int64_t>(m) * H + i)) : 0.0f;
-      }
-      const float inv = rotate_block_store(e4, ws.xt + static_cast<int64_t>(q) * kXsStride);
-      if (lane == 0) ws.xt_inv[q] = inv;
-    }
-    return;
-  }
 
   // 1. top-k + softmax, one warp per token.
   for (int t = warp; t < T; t += kRouterThreads / 32) {
@@ -252,146 +226,6 @@ router_kernel(const float* __restrict__ logits, const uint16_t* __restrict__ X, 
     for (int t = threadIdx.x; t < T; t += kRouterThreads) ws.tok_asg[t * (topk + 1) + topk] = -1;
 }
 
-// One pass of up to MT tokens of a gate_up unit: prefetch codes, stage the
-// tokens' rotated activations, decode (results in slots).
-template <int C, int MT, typename RowFn>
-__device__ __forceinline__ void gate_up_pass(const uint8_t* pk, const uint16_t* nm, int nb, int jt, RowFn rowfn,
-                                             const MoeWs& ws, int a_first, int ntok, const uint32_t* tab,
-                                             uint16_t* xs, float* xinv, float* slots) {
-  auto eng = make_engine<C, MT, 2>(pk, nm, nb, 2 * jt, rowfn);
-  eng.prefetch();
-  const int words = nb * kXsStride / 8;  // uint4 per token
-  for (int q = threadIdx.x; q < MT * words; q += blockDim.x) {
-    const int m = q / words, w = q - m * words;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (m < ntok) {
-      const int t = ws.asg_token[a_first + m];
-      val = reinterpret_cast<const uint4*>(ws.xt + static_cast<int64_t>(t) * nb * kXsStride)[w];
-    }
-    reinterpret_cast<uint4*>(xs)[q] = val;
-  }
-  for (int q = threadIdx.x; q < MT * nb; q += blockDim.x) {
-    const int m = q / nb, b = q - m * nb;
-    xinv[q] = m < ntok ? ws.xt_inv[static_cast<int64_t>(ws.asg_token[a_first + m]) * nb + b] : 0.0f;
-  }
-  __syncthreads();
-  eng.run(tab, xs, xinv, slots);
-  __syncthreads();
-}
-
-// One pass of up to MT assignments of a down unit: prefetch codes, rotate the
-// assignments' h rows in the CTA, decode (results in slots).
-template <int C, int MT, typename RowFn>
-__device__ __forceinline__ void down_pass(const uint8_t* pk, const uint16_t* nm, int nb, int nr, RowFn rowfn,
-                                          const float* hbase, int F, int ntok, const uint32_t* tab, uint16_t* xs,
-                                          float* xinv, float* slots) {
-  auto eng = make_engine<C, MT, 2>(pk, nm, nb, nr, rowfn);
-  eng.prefetch();
-  rotate_tokens_f32([=](int m) { return hbase + static_cast<int64_t>(m) * F; }, F, nb, ntok, MT, xs, xinv);
-  __syncthreads();
-  eng.run(tab, xs, xinv, slots);
-  __syncthreads();
-}
-
-__device__ __forceinline__ int pass_mt(int ntok) { return ntok <= 1 ? 1 : (ntok == 2 ? 2 : 4); }
-constexpr int kMoePass = 4;  // tokens per decode pass of a unit
-
-template <int C>
-__global__ void __launch_bounds__(kEngineThreads, 1)
-gate_up_kernel(const uint8_t* __restrict__ gu_packed, const uint16_t* __restrict__ gu_norms,
-               const uint8_t* __restrict__ sh_packed, const uint16_t* __restrict__ sh_norms,
-               const float* __restrict__ codebook, int E, int H, int F, MoeWs ws) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int nb = (H + kBlock - 1) / kBlock;
-  const int nch = (nb + C - 1) / C;
-  const EngineLayout L = engine_layout(kMoePass, nb, 2 * kJT, nch);
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
-  float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
-  float* slots = reinterpret_cast<float*>(smem + L.slot_off);
-  float* misc = reinterpret_cast<float*>(smem + L.misc_off);
-  uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
-  build_pair_table(tab, c16, codebook);
-  __syncthreads();
-
-  const int tiles = (F + kJT - 1) / kJT;
-  const int units = ws.meta[0] * tiles;
-  const int64_t expert_rows = 2 * static_cast<int64_t>(F);
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int a = u / tiles, tile = u - a * tiles;
-    const int e = ws.active[a];
-    const int j0 = tile * kJT, jt = min(kJT, F - j0);
-    const uint8_t* pk = e < E ? gu_packed + e * expert_rows * nb * kBlockBytes : sh_packed;
-    const uint16_t* nm = e < E ? gu_norms + e * expert_rows * nb : sh_norms;
-    const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
-    for (int m0 = 0; m0 < ne; m0 += kMoePass) {
-      const int ntok = min(kMoePass, ne - m0), mt = pass_mt(ntok);
-      auto rowfn = [=](int v) { return static_cast<int64_t>(v < jt ? j0 + v : F + j0 + (v - jt)); };
-      if (mt == 1) gate_up_pass<C, 1>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
-      else if (mt == 2) gate_up_pass<C, 2>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
-      else gate_up_pass<C, 4>(pk, nm, nb, jt, rowfn, ws, a0 + m0, ntok, tab, xs, xinv, slots);
-      const int nv = 2 * jt;
-      for (int idx = threadIdx.x; idx < ntok * jt; idx += blockDim.x) {
-        const int m = idx / jt, j = idx - m * jt;
-        const float* sg = slots + (m * nv + j) * nch;
-        const float* su = slots + (m * nv + jt + j) * nch;
-        float g = 0.0f, up = 0.0f;
-        for (int ch = 0; ch < nch; ++ch) { g += sg[ch]; up += su[ch]; }
-        const float hval = g / (1.0f + expf(-g)) * up;
-        ws.h[static_cast<int64_t>(a0 + m0 + m) * F + j0 + j] = hval;
-      }
-      __syncthreads();
-    }
-  }
-}
-
-template <int C>
-__global__ void __launch_bounds__(kEngineThreads, 1)
-down_kernel(const uint8_t* __restrict__ dn_packed, const uint16_t* __restrict__ dn_norms,
-            const uint8_t* __restrict__ sh_packed, const uint16_t* __restrict__ sh_norms,
-            const float* __restrict__ codebook, int E, int H, int F, MoeWs ws) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int nb = (F + kBlock - 1) / kBlock;
-  const int nch = (nb + C - 1) / C;
-  const EngineLayout L = engine_layout(kMoePass, nb, kHT, nch);
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
-  float* xinv = reinterpret_cast<float*>(smem + L.xinv_off);
-  float* slots = reinterpret_cast<float*>(smem + L.slot_off);
-  float* misc = reinterpret_cast<float*>(smem + L.misc_off);
-  uint16_t* c16 = reinterpret_cast<uint16_t*>(misc + 64);
-  build_pair_table(tab, c16, codebook);
-  __syncthreads();
-
-  const int tiles = (H + kHT - 1) / kHT;
-  const int units = ws.meta[0] * tiles;
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int a = u / tiles, tile = u - a * tiles;
-    const int e = ws.active[a];
-    const int r0 = tile * kHT, nr = min(kHT, H - r0);
-    const uint8_t* pk = e < E ? dn_packed + static_cast<int64_t>(e) * H * nb * kBlockBytes : sh_packed;
-    const uint16_t* nm = e < E ? dn_norms + static_cast<int64_t>(e) * H * nb : sh_norms;
-    const int a0 = ws.offsets[a], ne = ws.offsets[a + 1] - a0;
-    for (int m0 = 0; m0 < ne; m0 += kMoePass) {
-      const int ntok = min(kMoePass, ne - m0), mt = pass_mt(ntok);
-      const float* hbase = ws.h + static_cast<int64_t>(a0 + m0) * F;
-      auto rowfn = [=](int v) { return static_cast<int64_t>(r0 + v); };
-      if (mt == 1) down_pass<C, 1>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
-      else if (mt == 2) down_pass<C, 2>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
-      else down_pass<C, 4>(pk, nm, nb, nr, rowfn, hbase, F, ntok, tab, xs, xinv, slots);
-      for (int idx = threadIdx.x; idx < ntok * nr; idx += blockDim.x) {
-        const int m = idx / nr, v = idx - m * nr;
-        const float* sl = slots + (m * nr + v) * nch;
-        float sum = 0.0f;
-        for (int ch = 0; ch < nch; ++ch) sum += sl[ch];
-        const int asg = a0 + m0 + m;
-        ws.part[static_cast<int64_t>(asg) * H + r0 + v] = sum * ws.asg_weight[asg];
-      }
-      __syncthreads();
-    }
-  }
-}
-
 __global__ void combine_kernel(int H, int T, int topk, MoeWs ws, void* __restrict__ Y, int out_bf16) {
   const int t = blockIdx.y;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -406,10 +240,6 @@ __global__ void combine_kernel(int H, int T, int topk, MoeWs ws, void* __restric
   else static_cast<float*>(Y)[off] = acc;
 }
 
-template <typename K>
-bool set_smem_attr(K kernel) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) == cudaSuccess;
-}
 
 }  // namespace
 
@@ -431,54 +261,15 @@ int launch_moe(const uint8_t* gu_packed, const uint16_t* gu_norms, const uint8_t
   MoeWs ws;
   moe_layout(E, H, F, T, topk, static_cast<char*>(workspace), &ws);
   const bool shared = sh_gu_packed != nullptr;
-  const int nbh = static_cast<int>(ceil_div(H, kBlock)), nbf = static_cast<int>(ceil_div(F, kBlock));
-  // gate_up and down on the tensor cores when the rows fit its tile-norm
-  // staging (in <= 8192), else on the CUDA-core decode engine
-  const bool tc = nbh <= 64 && nbf <= 64;
-  // CTA 0 routes; for the CUDA-core kernels the others rotate every token's
-  // activation, about one 128-block per warp
-  const int64_t rot_warps = static_cast<int64_t>(T) * nbh;
-  const int rot_ctas =
-      tc ? 0 : static_cast<int>(std::min<int64_t>(4 * sm_count(), ceil_div(rot_warps, kRouterThreads / 32)));
-  router_kernel<<<1 + rot_ctas, kRouterThreads, 0, stream>>>(logits, X, E, H, T, topk, shared ? 1 : 0, ids_out,
-                                                              w_out, ws);
+  // one CTA routes and builds the lists; gate_up and down on the tensor cores
+  // (H and F up to kMoeMaxIn), then the fixed-order combine
+  if (H > kMoeMaxIn || F > kMoeMaxIn) return HLWQ_EUNSUPPORTED;
+  router_kernel<<<1, kRouterThreads, 0, stream>>>(logits, E, T, topk, shared ? 1 : 0, ids_out, w_out, ws);
   if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
-  dim3 cgrid(static_cast<unsigned>(ceil_div(H, 256)), static_cast<unsigned>(T));
-  if (tc) {
-    if (const int st = launch_moe_tc(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
-                                     sh_dn_norms, codebook, E, H, F, topk, T, X, ws, stream))
-      return st;
-    combine_kernel<<<cgrid, 256, 0, stream>>>(H, T, topk, ws, Y, out_bf16 ? 1 : 0);
-    return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
-  }
-
-  const int cg = pick_chunk(nbh), cd = pick_chunk(nbf);
-  const int smem_g = engine_layout(kMoePass, nbh, 2 * kJT, (nbh + cg - 1) / cg).total;
-  const int smem_d = engine_layout(kMoePass, nbf, kHT, (nbf + cd - 1) / cd).total;
-  if (smem_g > 227 * 1024 || smem_d > 227 * 1024) return HLWQ_EUNSUPPORTED;
-  const int grid = sm_count();
-  static PerDeviceOnce attrs;
-  if (const int st = attrs([&] {
-        return set_smem_attr(gate_up_kernel<8>) &&
-               set_smem_attr(gate_up_kernel<4>) &&
-               set_smem_attr(gate_up_kernel<2>) &&
-               set_smem_attr(down_kernel<8>) &&
-               set_smem_attr(down_kernel<4>) &&
-               set_smem_attr(down_kernel<2>);
-      }))
+  if (const int st = launch_moe_tc(gu_packed, gu_norms, dn_packed, dn_norms, sh_gu_packed, sh_gu_norms, sh_dn_packed,
+                                   sh_dn_norms, codebook, E, H, F, topk, T, X, ws, stream))
     return st;
-  switch (cg) {
-    case 8: gate_up_kernel<8><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
-    case 4: gate_up_kernel<4><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
-    default: gate_up_kernel<2><<<grid, kEngineThreads, smem_g, stream>>>(gu_packed, gu_norms, sh_gu_packed, sh_gu_norms, codebook, E, H, F, ws); break;
-  }
-  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
-  switch (cd) {
-    case 8: down_kernel<8><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
-    case 4: down_kernel<4><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
-    default: down_kernel<2><<<grid, kEngineThreads, smem_d, stream>>>(dn_packed, dn_norms, sh_dn_packed, sh_dn_norms, codebook, E, H, F, ws); break;
-  }
-  if (cudaGetLastError() != cudaSuccess) return HLWQ_ECUDA;
+  dim3 cgrid(static_cast<unsigned>(ceil_div(H, 256)), static_cast<unsigned>(T));
   combine_kernel<<<cgrid, 256, 0, stream>>>(H, T, topk, ws, Y, out_bf16 ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? HLWQ_OK : HLWQ_ECUDA;
 }

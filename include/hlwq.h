@@ -330,17 +330,15 @@ int hlwq_moe_gemv(const uint8_t* gu_packed, const uint16_t* gu_norms,
  * three quarters of the experts) and its shared memory fits, else the
  * grouped path.
  * HLWQ_FLAG_MOE_GROUPED selects the grouped path at any T.  The grouped path
- * reads each active expert's codes once for all its tokens:
- *   routing and per-expert assignment lists;
- *   for H and F up to 8192, on the tensor cores: each assignment's token
- *   gathered and rotated, gate_up as one grouped tcgen05 GEMM over (active
- *   expert, 128-row tile), SiLU(g) * u rotated with the routing weight on its
- *   scale, down as a grouped GEMM; the shared expert as plain GEMMs;
- *   for longer rows, on the CUDA cores: gate_up over (active expert, 32
- *   columns) units, down over (active expert, 128 rows) units;
- *   a fixed-order combine of each token's partial outputs.
+ * (H and F up to 16384) reads each active expert's codes once for all its
+ * tokens: routing and per-expert assignment lists; each assignment's token
+ * gathered and rotated; gate_up as one grouped tcgen05 GEMM over (active
+ * expert, 128-row tile), the shared expert from its own matrix in the same
+ * launch; SiLU(g) * u rotated with the routing weight on its scale; down as a
+ * grouped GEMM; a fixed-order combine of each token's partial outputs.
  * Same arguments, results (to rounding) and workspace; other flag bits are
- * HLWQ_EINVAL.
+ * HLWQ_EINVAL; HLWQ_EUNSUPPORTED when the grouped path is asked for with H or
+ * F above 16384, or when neither path fits (very long rows and many tokens).
  */
 int hlwq_moe_gemv_ex(const uint8_t* gu_packed, const uint16_t* gu_norms,
                      const uint8_t* dn_packed, const uint16_t* dn_norms,

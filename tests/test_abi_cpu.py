@@ -140,6 +140,17 @@ def test_tq3_gemm_validation_and_workspace(hl):
     assert hl.workspace_bytes(hl.HLWQ_OP_TQ3_GEMM, 256, 8192, 2) > 0
 
 
+def test_moe_grouped_path_row_limit(hl):
+    """The grouped path takes H and F up to 16384; asked for with longer rows
+    it returns HLWQ_EUNSUPPORTED before launching anything."""
+    L = hl.lib
+    p = ctypes.c_void_p(256)
+    E, H, F, topk, T = 8, 16512, 256, 2, 4
+    need = hl.workspace_bytes(hl.HLWQ_OP_MOE, H, F, T, E, topk)
+    args = [p] * 4 + [None] * 4 + [p, E, H, F, topk, T, p, p, p, hl.HLWQ_F32, None, None, p, need]
+    assert L.hlwq_moe_gemv_ex(*args, hl.HLWQ_FLAG_MOE_GROUPED, None) == hl.HLWQ_EUNSUPPORTED
+
+
 def test_noalloc_validates_arguments_before_sizing_its_scratch(hl):
     L = hl.lib
     p = ctypes.c_void_p(256)

@@ -118,6 +118,13 @@ def test_moe_grouped_path_one_expert_set_for_every_token(hl, cb):
              flags=hl.HLWQ_FLAG_MOE_GROUPED)
 
 
+def test_moe_grouped_path_rows_past_8192(hl, cb):
+    """H = 8320 (65 blocks): the grouped GEMMs stage tile norms of more than 64
+    blocks (up to 128, H and F <= 16384)."""
+    run_case(hl, cb, E=4, H=8320, F=256, T=3, topk=2, shared=True, seed=614, used_only=True,
+             flags=hl.HLWQ_FLAG_MOE_GROUPED)
+
+
 def test_moe_ex_rejects_unknown_flags(hl, cb):
     p = torch.zeros(16, dtype=torch.uint8, device="cuda")
     args = [hl._ptr(p)] * 4 + [None] * 4 + [hl._ptr(cb), 2, 128, 128, 1, 1, hl._ptr(p), hl._ptr(p), hl._ptr(p),
