@@ -75,9 +75,9 @@ def test_moe_small(hl, cb, T, topk, shared):
 
 
 # ----------------------------------------------------------------------------
-# The grouped path (four launches, each active expert read once for all its
-# tokens): selected with HLWQ_FLAG_MOE_GROUPED, and taken by default when the
-# fused path's shared memory does not fit (many tokens).
+# The grouped path (tensor cores, each active expert read once for all its
+# tokens): selected with HLWQ_FLAG_MOE_GROUPED, and taken by default once
+# 4 T topk >= 3 E or when the fused path's shared memory does not fit.
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("T,topk,shared", [(1, 8, True), (5, 2, False), (17, 8, True), (64, 8, True)])
