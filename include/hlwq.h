@@ -18,9 +18,10 @@
  *       first.
  * Dequantisation: w_hat[o][128b + i] = n16[o][b] / 128 * sum_j c[k_obj] H[j][i].
  *
- * Also declared here: the Q5 -> INT4 re-encoder, the Q3 KV-cache encoding,
- * the TQ3 (scalar HIGGS) weight format with its fused GEMV, and the
- * conversion between the packed codes and one code per byte.
+ * Also declared here: the Q5 -> INT4 re-encoder, the Q3 KV-cache encoding
+ * with its residual window, the TQ3 (scalar HIGGS) weight format with its
+ * fused GEMV and small-M GEMM, and the conversion between the packed codes
+ * and one code per byte.
  *
  * Storage contract (all row-major, caller-owned):
  *   packed  uint8  [rows][NB][80]   (0.625 byte per weight, including the pad)
