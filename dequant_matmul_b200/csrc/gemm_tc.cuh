@@ -13,7 +13,9 @@
 // Kernel 1 (rotate_x_kernel): one CTA per token rotates X once per call into
 // the workspace (binary16 B matrix, K-major) and records 1/s_m.
 // Kernel 2 (gemm_tc_kernel<F, NG>): one CTA per 128-row tile of W (and up to
-// 256-token tile of X).  Roles, D = 8 NG decode warps plus three:
+// 256-token tile of X); F is the weight format (HLWQ Q5 or TQ3).  The same
+// kernel runs the routed MoE layer's grouped GEMMs (TcGroup, launch_moe_tc).
+// Roles, D = 8 NG decode warps plus three:
 //   warps 0..D-1 decode, in NG groups of 8 taking blocks b = g (mod NG): each
 //              lane owns one weight row of the tile and decodes one half block
 //              (code -> fp32 centroid from a shared table, times the block
@@ -21,7 +23,9 @@
 //              memory with tcgen05.st (the A operand lives in TMEM, so
 //              decoding costs no shared-memory bandwidth that the MMA needs
 //              for B);
-//   warp D     TMA producer of the code tiles (128 rows x 80 bytes per block);
+//   warp D     initialises the barriers, then TMA producer of the code tiles
+//              (128 rows x one block); its first boxes go out before the
+//              CTA-wide barrier;
 //   warp D + 2 TMA producer of B: two 64 x N boxes per block, 128-byte
 //              swizzled (no multicast);
 //   warp D + 1 allocates TMEM and issues tcgen05.mma (kind::f16, M = 128,
